@@ -1,0 +1,323 @@
+"""Pins of the CPU oracle to facts fixed outside it.
+
+Each pin takes an ``oracle.Oracle`` and raises ``AssertionError`` when the
+oracle disagrees with a value printed on the pages (``tests/golden``), a closed
+form, an invariant, a textbook special case or a brute-force statement.  The
+same pins run against deliberately broken builds of the oracle
+(``test_oracle_mutants.py``) to show that each plausible mistake is caught.
+"""
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def golden(name):
+    """Rows of a fixture: list of (key tokens, value tokens)."""
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, _, vals = line.partition(":")
+            rows.append((key.split(), vals.split()))
+    return rows
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# --------------------------------------------------------------------- text
+
+
+def pin_inv_freq_golden(o):
+    for key, vals in golden("inv_freq.txt"):
+        dim, base, dec = int(key[0]), float(key[1]), int(key[2])
+        got = np.round(o.rope_inv_freq(dim, base).astype(np.float64), dec)
+        want = np.array([float(v) for v in vals])
+        assert got.shape == want.shape and np.array_equal(got, want), (dim, base, got, want)
+
+
+def pin_inv_freq_geometric(o):
+    # The frequencies start at 1 and fall geometrically with ratio base^(2/dim)
+    # ("Interleaved Rotary Position Embedding", RoPE section); fp32 rounding only.
+    for dim, base in [(64, 1e7), (128, 1e6), (36, 1e4), (256, 1e4)]:
+        inv = o.rope_inv_freq(dim, base).astype(np.float64)
+        assert inv.shape == (dim // 2,)
+        assert inv[0] == 1.0
+        ratio = inv[1:] / inv[:-1]
+        assert np.allclose(ratio, base ** (-2.0 / dim), rtol=3e-7, atol=0), (dim, base)
+        assert abs(inv[-1] - base ** (-(dim - 2) / dim)) <= 6e-8 * inv[-1]
+
+
+def pin_axis_acos_golden(o):
+    pos = np.array([[1], [2], [3]])
+    for key, vals in golden("axis_acos.txt"):
+        sec, il = tuple(int(v) for v in key[:3]), int(key[3])
+        cos, sin = o.mrope_cos_sin(pos, np.ones(10, np.float32), sec, il)
+        got = np.rint(np.arccos(np.clip(cos[0], -1, 1))).astype(int)
+        want = np.array([int(v) for v in vals])
+        assert np.array_equal(got, want), (sec, il, got, want)
+        # sin agrees with the same angle
+        assert np.allclose(sin[0], np.sin(want), atol=1e-15)
+
+
+def pin_axis_j7(o):
+    for key, vals in golden("axis_j7.txt"):
+        sec = tuple(int(v) for v in key)
+        lab = o.mrope_axis_labels(10, sec, True)
+        assert lab[7] == int(vals[0]), (sec, lab)
+
+
+def pin_axis_qwen35(o):
+    lab = o.mrope_axis_labels(32, (11, 11, 10), True)
+    names = {"T": 0, "H": 1, "W": 2}
+    seen = np.zeros(32, bool)
+    for key, vals in golden("sections_qwen35.txt"):
+        idx = [int(v) for v in vals]
+        assert np.all(lab[idx] == names[key[0]]), (key, lab)
+        seen[idx] = True
+    assert seen.all()
+
+
+def pin_axis_counts(o):
+    # Each axis gets exactly its mrope_section share of frequencies, in both
+    # layouts; chunked gives contiguous runs T..T H..H W..W.
+    for half, sec in [(64, (24, 20, 20)), (32, (11, 11, 10)), (10, (4, 3, 3)), (10, (6, 2, 2)), (2, (1, 1, 0))]:
+        for il in (True, False):
+            lab = o.mrope_axis_labels(half, sec, il)
+            assert [int((lab == a).sum()) for a in range(3)] == list(sec), (half, sec, il, lab)
+        ch = o.mrope_axis_labels(half, sec, False)
+        assert np.all(np.diff(ch) >= 0)
+    # [24, 20, 20] interleaved: H at 1..58 step 3, W at 2..59 step 3, T elsewhere
+    lab = o.mrope_axis_labels(64, (24, 20, 20), True)
+    want = np.zeros(64, int)
+    want[1:60:3] = 1
+    want[2:60:3] = 2
+    assert np.array_equal(lab, want)
+
+
+def pin_rotary_d4_golden(o):
+    g = {k[0]: np.array([float(v) for v in vals]) for k, vals in golden("rotary_d4.txt")}
+    assert np.array_equal(o.rotate_half(g["rotate_half_in"]), g["rotate_half_out"])
+    inv = np.array([1.0, 0.01], np.float32)
+    pos = np.array([[2], [2], [2]])
+    cos, sin = o.mrope_cos_sin(pos, inv, (1, 1, 0), True)
+    assert np.array_equal(np.round(cos[0], 4), g["cos"]), cos
+    assert np.array_equal(np.round(sin[0], 4), g["sin"]), sin
+    for i in (1, 2):
+        x = g[f"apply_in_{i}"].reshape(1, 1, 4)
+        out = o.apply_rotary(x, cos, sin)[0, 0]
+        assert np.array_equal(np.round(out, 4) + 0.0, g[f"apply_out_{i}"]), (i, out)
+
+
+def pin_text_only_reduces_to_1d(o):
+    # Text tokens (t = h = w): interleaved and chunked give bitwise the same
+    # cos / sin, and the rotation is the textbook 1-D RoPE: pair (j, j + half)
+    # is the complex number x_j + i x_{j+half} multiplied by exp(i p inv_j)
+    # ("M01", step 5; "Interleaved Rotary Position Embedding", RoPE section).
+    rng = _rng(7)
+    half, sec = 32, (11, 11, 10)
+    p = np.sort(rng.integers(0, 200000, 64))
+    pos = np.stack([p, p, p])
+    inv = o.rope_inv_freq(64, 1e7)
+    ci, si = o.mrope_cos_sin(pos, inv, sec, True)
+    cc, sc = o.mrope_cos_sin(pos, inv, sec, False)
+    assert np.array_equal(ci, cc) and np.array_equal(si, sc)
+    x = rng.standard_normal((64, 3, 96))
+    out = o.apply_rotary(x, ci, si)
+    ang = (p[:, None].astype(np.float32) * inv[None, :]).astype(np.float64)   # fp32 products
+    z = (x[:, :, :half] + 1j * x[:, :, half:2 * half]) * np.exp(1j * ang)[:, None, :]
+    assert np.allclose(out[:, :, :half], z.real, rtol=0, atol=1e-12)
+    assert np.allclose(out[:, :, half:2 * half], z.imag, rtol=0, atol=1e-12)
+
+
+def pin_rotation_invariants(o):
+    rng = _rng(11)
+    T, H, D, rot = 40, 5, 48, 32
+    x = rng.standard_normal((T, H, D))
+    pos = rng.integers(0, 5000, (3, T))
+    inv = o.rope_inv_freq(rot, 1e4)
+    cos, sin = o.mrope_cos_sin(pos, inv, (6, 5, 5), True)
+    out = o.apply_rotary(x, cos, sin)
+    h = rot // 2
+    # channels >= rot pass through bit-identically
+    assert np.array_equal(out[:, :, rot:], x[:, :, rot:])
+    # every pair (j, j + rot/2) keeps its length
+    n_in = x[:, :, :h] ** 2 + x[:, :, h:rot] ** 2
+    n_out = out[:, :, :h] ** 2 + out[:, :, h:rot] ** 2
+    assert np.allclose(n_in, n_out, rtol=1e-13, atol=1e-13)
+
+
+def pin_relative_position(o):
+    # q(p) . k(p') depends only on p - p' (RoFormer property quoted on
+    # "Interleaved Rotary Position Embedding", RoPE section).  Frequencies that
+    # are powers of two keep every fp32 angle exact, so the check is exact.
+    rng = _rng(3)
+    half = 8
+    inv = (2.0 ** -np.arange(half)).astype(np.float32)
+    q = rng.standard_normal((1, 1, 2 * half))
+    k = rng.standard_normal((1, 1, 2 * half))
+
+    def rot(x, p):
+        pos = np.array([[p], [p], [p]])
+        c, s = o.mrope_cos_sin(pos, inv, (half, 0, 0), True)
+        return o.apply_rotary(x, c, s)[0, 0]
+
+    for p, pk, shift in [(5, 2, 17), (100, 300, 1000), (0, 9, 4096)]:
+        d0 = rot(q, p) @ rot(k, pk)
+        d1 = rot(q, p + shift) @ rot(k, pk + shift)
+        assert abs(d0 - d1) < 1e-11, (p, pk, shift, d0, d1)
+
+
+def pin_vision_tokens_per_axis(o):
+    # A vision token's rotary angle at frequency j is the selected axis
+    # position times inv_j: [2, 3, 4] for I12 gives 2,3,4,2,3,4,... under
+    # [11, 11, 10] ("Interleaved Rotary Position Embedding", I12 example).
+    inv = np.ones(32, np.float32)
+    cos, sin = o.mrope_cos_sin(np.array([[2], [3], [4]]), inv, (11, 11, 10), True)
+    ang = np.rint(np.mod(np.arctan2(sin[0, :32], cos[0, :32]), 2 * np.pi)).astype(int)
+    want = np.array([[2, 3, 4][j % 3] for j in range(32)])
+    assert np.array_equal(ang, want), ang
+    assert np.array_equal(cos[0, 32:], cos[0, :32])
+
+
+# ------------------------------------------------------------------- vision
+
+
+def _merge_order_rowcol(t, h, w, m):
+    """Brute-force statement of the output order: merge-block row, merge-block
+    column, then the m x m patches inside, for each frame ("cortiq-engine
+    qwen3vis.rs", positions() and rope_angles() loops)."""
+    out = []
+    for _ in range(t):
+        for by in range(h // m):
+            for bx in range(w // m):
+                for iy in range(m):
+                    for ix in range(m):
+                        out.append((by * m + iy, bx * m + ix))
+    return np.array(out, np.int64).reshape(-1, 2)
+
+
+def pin_patch_counts(o):
+    g = {k[0]: [int(v) for v in vals] for k, vals in golden("patch_counts.txt")}
+    assert o.grid_patches(g["grid_thw"], 2) == g["patches"][0]
+    assert o.grid_patches(g["grid_thw"], 2) // 4 == g["merged_tokens"][0]
+    assert o.vis_rot_pos_ids(g["grid_thw"], 2).shape == (3072, 2)
+
+
+def pin_exact_lookup_48(o):
+    # h = w = G: every sample lands on a grid point, weights (1, 0, 0, 0), and
+    # the output is the table itself in merge order.
+    rng = _rng(5)
+    G, C = 48, 24
+    table = rng.standard_normal((G * G, C))
+    out = o.vis_pos_embed_interpolate(table, [(1, 48, 48)], 2)
+    rc = _merge_order_rowcol(1, 48, 48, 2)
+    assert np.array_equal(out, table[rc[:, 0] * G + rc[:, 1]])
+    idx, w = o.vis_interp_plan([(1, 48, 48)], 2, G)
+    assert np.array_equal(w[0], np.ones(48 * 48)) and not w[1:].any()
+    assert np.array_equal(idx[0], rc[:, 0] * G + rc[:, 1])
+
+
+def pin_bilinear_reproduces_bilinear_functions(o):
+    # Bilinear interpolation reproduces a + b y + c x + d x y exactly, sampled
+    # at y = row (G-1)/(h-1), x = col (G-1)/(w-1) (0 when the side is 1).
+    G = 48
+    gy, gx = np.meshgrid(np.arange(G, dtype=np.float64), np.arange(G, dtype=np.float64), indexing="ij")
+    coef = [(0.5, -1.25, 2.0, 0.0), (0.1, 0.0, 0.0, 0.03), (-2.0, 0.7, -0.3, 0.011)]
+    table = np.stack([a + b * gy + c * gx + d * gx * gy for a, b, c, d in coef], -1).reshape(G * G, -1)
+    for grid, m in [((1, 16, 16), 2), ((1, 32, 48), 2), ((2, 28, 28), 2), ((1, 64, 96), 2),
+                    ((1, 80, 56), 2), ((1, 1, 5), 1), ((1, 3, 1), 1), ((1, 6, 9), 3)]:
+        t, h, w = grid
+        out = o.vis_pos_embed_interpolate(table, [grid], m)
+        rc = _merge_order_rowcol(t, h, w, m)
+        y = rc[:, 0] * (G - 1) / (h - 1) if h > 1 else np.zeros(len(rc))
+        x = rc[:, 1] * (G - 1) / (w - 1) if w > 1 else np.zeros(len(rc))
+        want = np.stack([a + b * y + c * x + d * x * y for a, b, c, d in coef], -1)
+        assert np.allclose(out, want, rtol=0, atol=1e-12), grid
+
+
+def pin_interp_weights(o):
+    for grid in [(1, 16, 16), (1, 32, 48), (2, 28, 28), (1, 80, 56), (1, 2, 2)]:
+        idx, w = o.vis_interp_plan([grid], 2, 48)
+        assert np.allclose(w.sum(0), 1.0, rtol=0, atol=1e-15)
+        assert (w >= 0).all() and (w <= 1).all()
+        assert (idx >= 0).all() and (idx < 48 * 48).all()
+        # corners share rows / columns: TL, TR on one row; TL, BL in one column
+        assert np.array_equal(idx[0] // 48, idx[1] // 48) and np.array_equal(idx[2] // 48, idx[3] // 48)
+        assert np.array_equal(idx[0] % 48, idx[2] % 48) and np.array_equal(idx[1] % 48, idx[3] % 48)
+
+
+def pin_frames_and_concat(o):
+    # t frames repeat the same image; images concatenate in grid_thw order.
+    rng = _rng(9)
+    table = rng.standard_normal((48 * 48, 8))
+    grids = [(2, 4, 6), (1, 2, 2), (3, 6, 4)]
+    out = o.vis_pos_embed_interpolate(table, grids, 2)
+    off = 0
+    for t, h, w in grids:
+        single = o.vis_pos_embed_interpolate(table, [(1, h, w)], 2)
+        for f in range(t):
+            assert np.array_equal(out[off + f * h * w: off + (f + 1) * h * w], single)
+        off += t * h * w
+    assert off == out.shape[0]
+
+
+def pin_merge_order_brute_force(o):
+    # The 6-D permute of the interpolation, the broadcast of rot_pos_emb and a
+    # brute-force loop all give the same (row, col) order.
+    G = 48
+    gy, gx = np.meshgrid(np.arange(G), np.arange(G), indexing="ij")
+    # a table whose rows encode their own (row, col) grid point
+    table = np.stack([gy, gx], -1).reshape(G * G, 2).astype(np.float64)
+    for grid in [(1, 2, 2), (1, 4, 6), (2, 6, 4), (1, 2, 8), (2, 8, 2)]:
+        t, h, w = grid
+        rc = _merge_order_rowcol(t, h, w, 2)
+        assert np.array_equal(o.vis_rot_pos_ids([grid], 2), rc)
+    for grid in [(1, 48, 48), (2, 48, 48)]:
+        out = o.vis_pos_embed_interpolate(table, [grid], 2)
+        assert np.array_equal(out.astype(np.int64), _merge_order_rowcol(*grid, 2))
+
+
+def pin_vision_angles_basis(o):
+    # Reading the angles back: q = e_j gives (cos a_j, sin a_j) in channels
+    # (j, j + 36); a_j is row * inv_j for j < 18 and col * inv_(j-18) after
+    # ("cortiq-engine qwen3vis.rs", rope_angles() and attention()).
+    grid = [(1, 4, 6)]
+    pos = o.vis_rot_pos_ids(grid, 2)
+    N, D = pos.shape[0], 72
+    inv = o.rope_inv_freq(36, 1e4)
+    for j in [0, 5, 17, 18, 23, 35]:
+        x = np.zeros((N, 1, D))
+        x[:, 0, j] = 1.0
+        out = o.vis_apply_rotary(x, grid, 2, 1e4)[:, 0]
+        axis, i = (0, j) if j < 18 else (1, j - 18)
+        a = (pos[:, axis].astype(np.float32) * inv[i]).astype(np.float64)
+        assert np.allclose(out[:, j], np.cos(a), atol=1e-15)
+        assert np.allclose(out[:, j + 36], np.sin(a), atol=1e-15)
+        others = np.delete(out, [j, j + 36], axis=1)
+        assert not others.any()
+
+
+def pin_vision_rotation_complex(o):
+    # Whole-head split-half rotation = complex multiply of x_j + i x_(j+36)
+    # by exp(i a_j); norm of every pair preserved.
+    rng = _rng(13)
+    grid = [(2, 4, 4)]
+    pos = o.vis_rot_pos_ids(grid, 2)
+    N = pos.shape[0]
+    x = rng.standard_normal((N, 3, 72))
+    out = o.vis_apply_rotary(x, grid, 2, 1e4)
+    inv = o.rope_inv_freq(36, 1e4)
+    a = np.concatenate([(pos[:, :1].astype(np.float32) * inv[None, :]),
+                        (pos[:, 1:].astype(np.float32) * inv[None, :])], 1).astype(np.float64)
+    z = (x[:, :, :36] + 1j * x[:, :, 36:]) * np.exp(1j * a)[:, None, :]
+    assert np.allclose(out[:, :, :36], z.real, rtol=0, atol=1e-12)
+    assert np.allclose(out[:, :, 36:], z.imag, rtol=0, atol=1e-12)
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
