@@ -1,0 +1,492 @@
+#!/usr/bin/env python
+"""Benchmark of the positional-encoding hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ipe|reference]
+
+One step is one pass of the whole path over one prefill request of the
+large-prefill workload: a 16 x 64 x 64 video (65536 patches) through the
+vision position-table interpolation and the vision 2-D rotary, and the
+language model's interleaved multimodal RoPE on Q [131072, 24, 256] and
+K [131072, 4, 256] (bf16, rotary dim 64, theta 1e7, mrope_section
+[11, 11, 10]).  Inputs are seeded and synthetic, resident in HBM when the
+timed region starts; every input is larger than the 126 MB L2 except the
+5.3 MB position table, which a real vision tower also keeps hot.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own request:
+weak scaling with no data-path collective; the step time is the maximum over
+ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (double precision, one thread) on a
+bounded sample of the same workload instead (rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from datetime import datetime, timedelta
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "prefill_t131072_video"
+METRIC = "Q/K MRoPE tokens/s and pos-interp patches/s; achieved HBM GB/s vs ~8 TB/s"
+UNIT = "tokens/s"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ipe", "reference"], default="ipe")
+    ap.add_argument("--e2e-steps", type=int, default=3, help="steps of the end-to-end (host buffers) measurement")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the per-variant side measurements")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+
+def algorithmic_bytes(w):
+    """Bytes each kernel must move per launch (the roofline numerator)."""
+    v, t = w.vision, w.text
+    import workloads as wl
+    N = wl.n_patches(v)
+    eb_v = 2 if v.dtype == "bf16" else 4
+    G = v.grid_side
+    # table rows any sample touches: every grid row / column that is a corner
+    rows = set()
+    cols = set()
+    for _, h, ww in v.grid_thw:
+        for n, s in ((h, rows), (ww, cols)):
+            for i in range(n):
+                num = i * (G - 1)
+                y0 = 0 if n == 1 else num // (n - 1)
+                s.update((y0, min(y0 + 1, G - 1)))
+    U = len(rows) * len(cols)
+    rot_bytes = (t.hq + t.hk) * t.T * t.rot_dim * 2 * 2
+    return {
+        "vis_pos_interp": U * v.hidden * eb_v + N * v.hidden * eb_v,
+        "vis_rope2d": 2 * N * v.heads * v.head_dim * eb_v * 2,
+        "mrope_apply": rot_bytes + 3 * t.T * 4,
+        "mrope_cos_sin": 3 * t.T * 4 + 2 * t.T * t.rot_dim * 4,
+        "apply_rotary_partial": rot_bytes + 2 * t.T * t.rot_dim * 4,
+    }
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "interpolated_position_encoding_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def dram_traffic(kernel):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or
+    None when the kernels changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(WORKLOAD, {}).get(kernel)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the benchmark runs."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "20",
+                 "-i", str(self.gpu_id)], stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def stop(self, t0, t1):
+        """Summary of the samples taken between host times t0 and t1."""
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = []
+        for line in self.file.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+            except ValueError:
+                continue
+        os.unlink(self.file.name)
+        inside = [r for r in rows if t0 - 0.02 <= r[0] <= t1 + 0.02]
+        used = inside if inside else rows
+        if not used:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in used for i, v in enumerate(r[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in used), "sm_max_mhz": max(r[2] for r in used),
+                "reasons": reasons, "samples": len(used), "window": "timed" if inside else "whole run"}
+
+
+# ------------------------------------------------------------- the oracle
+
+
+def oracle_sample(w, text_tokens, frames, seed_text_offset=8192):
+    """Inputs of a bounded sample of the workload for the CPU oracle: a window
+    of `text_tokens` tokens (from `seed_text_offset`, through the video slices)
+    and the first `frames` frames of the video."""
+    import numpy as np
+    import workloads as wl
+    t, v = w.text, w.vision
+    pos, _ = wl.build_positions(t.segments, t.merge)
+    s0 = min(seed_text_offset, t.T - text_tokens)
+    sl = slice(s0, s0 + text_tokens)
+    key_q, key_k = wl.key_for(w.index, wl.S_Q), wl.key_for(w.index, wl.S_K)
+    q = wl.normal_bf16(key_q + (s0,), (text_tokens, t.hq, t.head_dim))
+    k = wl.normal_bf16(key_k + (s0,), (text_tokens, t.hk, t.head_dim))
+    _, h, ww = v.grid_thw[0]
+    n = frames * h * ww
+    vin = {
+        "table": wl.normal_bf16(wl.key_for(w.index, wl.S_TABLE), (v.grid_side ** 2, v.hidden), v.table_std),
+        "q": wl.normal_bf16(wl.key_for(w.index, wl.S_QV) + (1,), (n, v.heads, v.head_dim)),
+        "k": wl.normal_bf16(wl.key_for(w.index, wl.S_KV) + (1,), (n, v.heads, v.head_dim)),
+    }
+    f64 = lambda b: wl.bf16_bits_to_f32(b).astype(np.float64)  # noqa: E731
+    return {"pos": np.ascontiguousarray(pos[:, sl]), "q": f64(q), "k": f64(k), "table": f64(vin["table"]),
+            "vq": f64(vin["q"]), "vk": f64(vin["k"]), "grid": [(frames, h, ww)]}
+
+
+def run_oracle(orc, w, s):
+    t, v = w.text, w.vision
+    inv = orc.rope_inv_freq(t.rot_dim, t.theta)
+    orc.mrope_apply(s["q"], s["pos"], inv, t.section, True)
+    orc.mrope_apply(s["k"], s["pos"], inv, t.section, True)
+    orc.vis_pos_embed_interpolate(s["table"], s["grid"], v.merge)
+    orc.vis_apply_rotary(s["vq"], s["grid"], v.merge, v.theta)
+    orc.vis_apply_rotary(s["vk"], s["grid"], v.merge, v.theta)
+
+
+def cpu_baseline(w, text_tokens=65536, frames=8):
+    """Oracle throughput on a bounded sample, scaled to tokens/s of the whole step."""
+    import oracle
+    orc = oracle.get()
+    s = oracle_sample(w, text_tokens, frames)
+    t0 = time.perf_counter()
+    run_oracle(orc, w, s)
+    sec = time.perf_counter() - t0
+    import workloads as wl
+    N = wl.n_patches(w.vision)
+    # the sample keeps the step's token : patch ratio (T / N = 2)
+    frac = text_tokens / w.text.T
+    assert abs(frames * 64 * 64 / N - frac) < 1e-9
+    return {"value": text_tokens / sec, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{text_tokens} tokens (Q and K) + {frames} video frames ({frames * 4096} patches: "
+                      f"interpolation, q and k rotary) = 1/{round(1 / frac)} of a step, {sec:.2f} s"}
+
+
+def reference_arm(args):
+    """--impl reference: the CPU oracle as the reference implementation.  Each
+    step is 1/16 of a request: 8192 tokens (Q and K) and one 64 x 64 video
+    frame (4096 patches: interpolation and q, k rotary), the step's own
+    2 : 1 token : patch ratio.  Rank 0 alone runs it."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import oracle
+    import workloads as wl
+    w = wl.WORKLOADS[WORKLOAD]
+    orc = oracle.get()
+    tokens, frames = 8192, 1
+    s = oracle_sample(w, tokens, frames)
+    for _ in range(max(args.warmup, 0)):
+        run_oracle(orc, w, s)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run_oracle(orc, w, s)
+    sec = time.perf_counter() - t0
+    value = tokens * args.steps / sec
+    sample = f"{tokens} tokens (Q and K) + {frames * 4096} patches per step (1/16 of a request)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec / max(args.steps, 1) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "step_sample": sample, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- the GPU
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}: launch N > 1 with torchrun")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=300))
+
+    import interpolated_position_encoding_b200 as ipe
+    import workloads as wl
+
+    w = wl.WORKLOADS[WORKLOAD]
+    t, v = w.text, w.vision
+    N = wl.n_patches(v)
+
+    # ---- inputs (host, seeded; rank r > 0 shifts the stream by r)
+    tin = wl.text_inputs(w)
+    vin = wl.vision_inputs(w)
+    if rank:
+        rng = np.random.default_rng(rank)
+        tin["q"] = np.roll(tin["q"], int(rng.integers(1, 1000)), axis=0)
+        vin["q"] = np.roll(vin["q"], int(rng.integers(1, 1000)), axis=0)
+
+    def dev_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    table = dev_bf16(vin["table"])
+    qv, kv = dev_bf16(vin["q"]), dev_bf16(vin["k"])
+    Q, K = dev_bf16(tin["q"]), dev_bf16(tin["k"])
+    pos = torch.from_numpy(tin["positions"]).to(dev)
+    out = torch.empty(N, v.hidden, dtype=torch.bfloat16, device=dev)
+    inv = ipe.rope_inv_freq(t.rot_dim, t.theta)
+    grid = v.grid_thw
+    stream = torch.cuda.current_stream()
+
+    names = ["vis_pos_interp", "vis_rope2d", "mrope_apply"]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ipe.vis_pos_interp(table, grid, v.merge, out=out, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        ipe.vis_rope2d(qv, kv, grid, v.merge, v.theta, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        ipe.mrope_apply(Q, K, pos, inv, t.section, True, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        tt = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        return float(tt.item())
+
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    sampler = ClockSampler(gpu_id).start()
+    time.sleep(0.1)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    h0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    h1 = time.time()
+    ms_step = start.elapsed_time(end) / args.steps
+    ms_step = max_over_ranks(ms_step)
+    kernel_ms = {n: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j, n in enumerate(names)}
+    clocks = sampler.stop(h0, h1)
+
+    alg = algorithmic_bytes(w)
+    peak, peak_src = measured_peaks()
+    step_bytes = sum(alg[n] for n in names)
+    kernels = {n: {"ms": kernel_ms[n], "alg_bytes": alg[n], "gbs": alg[n] / kernel_ms[n] / 1e6,
+                   "frac": alg[n] / kernel_ms[n] / 1e6 / peak} for n in names}
+    dom = max(names, key=lambda n: kernel_ms[n])
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak, "unit": "GB/s",
+                "frac": kernels[dom]["frac"], "traffic": dram_traffic(dom), "alg_bytes": alg[dom],
+                "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured" else
+                "fallback 6650 GB/s"}
+
+    # ---- side measurements (after the timed region)
+    extras = {}
+    if not args.no_extras:
+        extras = side_measurements(ipe, w, dev, stream, Q, K, pos, inv, table, qv, kv, out, alg, peak,
+                                   max(args.steps // 4, 20))
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = end_to_end(ipe, torch, w, dev, stream, vin, tin, inv, max(args.e2e_steps, 1), max_over_ranks, barrier)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    value = world * t.T / (ms_step / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens_per_step": t.T, "patches_per_step": N,
+                   "text": f"Q [{t.T},{t.hq},{t.head_dim}] K [{t.T},{t.hk},{t.head_dim}] bf16, rot {t.rot_dim}, "
+                           f"theta {t.theta:g}, section {list(t.section)} interleaved, fused mrope_apply",
+                   "vision": f"grid_thw {grid}, table [{v.grid_side ** 2},{v.hidden}] bf16, q/k [{N},{v.heads},"
+                             f"{v.head_dim}] bf16, theta {v.theta:g}",
+                   "l2": "no flush: every input and output but the 5.3 MB table is larger than L2",
+                   "parallelism": f"dp{world} (independent requests)"},
+        "patches_per_s": world * N / (ms_step / 1e3),
+        "step_hbm_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+        "roofline": roofline,
+        "kernels": kernels,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "extras": extras,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def _time(torch, stream, fn, reps):
+    fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def side_measurements(ipe, w, dev, stream, Q, K, pos, inv, table, qv, kv, out, alg, peak, reps):
+    """The unfused MRoPE (tables in HBM) and the one-launch vision variant."""
+    import torch
+    t, v = w.text, w.vision
+    cos = torch.empty(t.T, t.rot_dim, dtype=torch.float32, device=dev)
+    sin = torch.empty_like(cos)
+    res = {}
+    ms_cs = _time(torch, stream, lambda: ipe.mrope_cos_sin(pos, inv, t.section, True, cos, sin, stream=stream), reps)
+    ms_ap = _time(torch, stream, lambda: ipe.apply_rotary_partial(Q, K, cos, sin, stream=stream), reps)
+    ms_fu = _time(torch, stream, lambda: ipe.mrope_apply(Q, K, pos, inv, t.section, True, stream=stream), reps)
+    for n, ms in (("mrope_cos_sin", ms_cs), ("apply_rotary_partial", ms_ap), ("mrope_apply", ms_fu)):
+        res[n] = {"ms": ms, "gbs": alg[n] / ms / 1e6, "frac": alg[n] / ms / 1e6 / peak}
+    res["unfused_over_fused"] = (ms_cs + ms_ap) / ms_fu
+    ms_vf = _time(torch, stream, lambda: ipe.vis_pos_interp_rope2d(table, v.grid_thw, qv, kv, v.merge, v.theta,
+                                                                   out=out, stream=stream), reps)
+    vb = alg["vis_pos_interp"] + alg["vis_rope2d"]
+    res["vis_pos_interp_rope2d"] = {"ms": ms_vf, "gbs": vb / ms_vf / 1e6, "frac": vb / ms_vf / 1e6 / peak}
+    return res
+
+
+def end_to_end(ipe, torch, w, dev, stream, vin, tin, inv, steps, max_over_ranks, barrier):
+    """Same step with host inputs: H2D of every input from pinned memory and
+    D2H of every result inside the timed region."""
+    t, v = w.text, w.vision
+    N = v and sum(a * b * c for a, b, c in v.grid_thw)
+
+    def pinned_bf16(a):
+        return torch.from_numpy(a.view(__import__("numpy").int16)).view(torch.bfloat16).pin_memory()
+
+    h_in = {"table": pinned_bf16(vin["table"]), "qv": pinned_bf16(vin["q"]), "kv": pinned_bf16(vin["k"]),
+            "Q": pinned_bf16(tin["q"]), "K": pinned_bf16(tin["k"]),
+            "pos": torch.from_numpy(tin["positions"]).pin_memory()}
+    d = {k: torch.empty_like(x, device=dev) for k, x in h_in.items()}
+    out = torch.empty(N, v.hidden, dtype=torch.bfloat16, device=dev)
+    h_out = {"out": torch.empty(N, v.hidden, dtype=torch.bfloat16).pin_memory(),
+             "qv": torch.empty_like(h_in["qv"]).pin_memory(), "kv": torch.empty_like(h_in["kv"]).pin_memory(),
+             "Q": torch.empty_like(h_in["Q"]).pin_memory(), "K": torch.empty_like(h_in["K"]).pin_memory()}
+    bi = sum(x.numel() * x.element_size() for x in h_in.values())
+    bo = sum(x.numel() * x.element_size() for x in h_out.values())
+
+    def step():
+        for k, x in h_in.items():
+            d[k].copy_(x, non_blocking=True)
+        ipe.vis_pos_interp(d["table"], v.grid_thw, v.merge, out=out, stream=stream)
+        ipe.vis_rope2d(d["qv"], d["kv"], v.grid_thw, v.merge, v.theta, stream=stream)
+        ipe.mrope_apply(d["Q"], d["K"], d["pos"], inv, t.section, True, stream=stream)
+        h_out["out"].copy_(out, non_blocking=True)
+        for k in ("qv", "kv", "Q", "K"):
+            h_out[k].copy_(d[k], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(a.elapsed_time(b) / steps)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    return {"value": world * t.T / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+            "ms_per_step": ms, "steps": steps}
+
+
+if __name__ == "__main__":
+    main()

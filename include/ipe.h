@@ -1,0 +1,229 @@
+/*
+ * ipe.h -- C ABI of the B200 (sm_100a) interpolated-position-encoding library
+ * (libipe.so): the positional-encoding hot path of Qwen3-VL / Qwen3.5-style
+ * vision-language models.
+ *
+ *   vision tower   vis_pos_interp      bilinear 48x48 position table -> patch grid, 2x2 merge order
+ *                  vis_rope2d          2-D (row, col) rotary over the whole head
+ *                  vis_pos_interp_rope2d  both in one launch
+ *   language model rope_inv_freq       default RoPE inverse frequencies (host)
+ *                  mrope_axis_map      per-frequency T/H/W axis (interleaved or chunked)
+ *                  mrope_cos_sin       multimodal cos / sin tables
+ *                  apply_rotary_partial  rotate_half rotation of the first rot_dim channels
+ *                  mrope_apply         the three above fused; cos / sin never leave registers
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Return value: an ipe_status.  On anything but IPE_OK, ipe_last_error()
+ *   returns a message for the calling thread, and nothing was launched unless
+ *   the status is IPE_ECUDA from the launch itself.
+ * - Every check happens on the host before any launch: sizes, divisibility,
+ *   alignment of vectorised pointers and strides, and that each device pointer
+ *   is device memory of the current device whose allocation covers the bytes
+ *   the call touches.  Kernels never trap or assert.
+ * - Device pointers are caller-owned.  The library allocates no memory and
+ *   keeps no pointer after it returns.  Small host arrays (grid_thw, section,
+ *   inv_freq) are copied by value into kernel parameters before the call
+ *   returns, so the caller may reuse them at once.
+ * - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *   legacy default stream) of the current device.
+ * - Rotations are in place.  vis_pos_interp and mrope_cos_sin write separate
+ *   outputs.  Two calls that touch the same memory on different streams race.
+ * - Element counts and strides are in elements, not bytes.
+ * - Floating-point arithmetic is fp32; bf16 results are rounded once (to
+ *   nearest even) at the end.  sin / cos are CUDA's accurate sincosf.
+ *
+ * Pages cited (title -- section):
+ *   [QVL]  "Qwen3-VL" notes, frankmowj.github.io
+ *   [IRPE] "Interleaved Rotary Position Embedding", taking-lying-flat.github.io
+ *   [M01]  "M01 RMSNorm and multimodal RoPE (interleaved / chunked)", kuanzhou.online
+ *   [VLM]  "VLM", llm.rainlin.net
+ *   [CRT]  cortiq-engine 0.8.52 src/qwen3vis.rs, docs.rs
+ */
+#ifndef IPE_H
+#define IPE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { IPE_F32 = 0, IPE_BF16 = 1 } ipe_dtype;
+
+typedef enum {
+    IPE_OK = 0,
+    IPE_EINVAL = 1,  /* a size, count or pointer the operation does not accept  */
+    IPE_EALIGN = 2,  /* a pointer or stride breaks the vector alignment        */
+    IPE_ELIMIT = 3,  /* above a documented library limit (images, dims, T)     */
+    IPE_ECUDA = 4    /* a CUDA runtime call or the launch failed               */
+} ipe_status;
+
+/* Library limits (IPE_ELIMIT above them). */
+#define IPE_MAX_IMAGES 1024     /* images per vision call                     */
+#define IPE_MAX_HALF 256        /* rot_dim / 2 of the text rotary             */
+#define IPE_MAX_POSITION 16777216 /* positions must lie in [0, 2^24): fl32(pos) is exact */
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char *ipe_last_error(void);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int ipe_version(void);
+
+/* ---------------------------------------------------------------------------
+ * ipe_rope_inv_freq -- default RoPE inverse frequencies, on the host.
+ * [IRPE] compute_default_rope_parameters; [M01] problem summary:
+ *   inv_freq[j] = 1 / theta^(2j / rot_dim),  j = 0 .. rot_dim/2 - 1
+ * with rot_dim = int(head_dim * partial_rotary_factor).  Computed in double,
+ * rounded once to fp32.
+ *   rot_dim        even, 2 .. 2*IPE_MAX_HALF
+ *   theta          > 0 (rope_theta: 1e7 for Qwen3.5 text, 1e6 Qwen3-Omni, 1e4 vision)
+ *   inv_freq_host  host array of rot_dim/2 floats, written.
+ * ------------------------------------------------------------------------- */
+int ipe_rope_inv_freq(int rot_dim, double theta, float *inv_freq_host);
+
+/* ---------------------------------------------------------------------------
+ * ipe_mrope_axis_map -- axis (0 = T, 1 = H, 2 = W) of each of the `half`
+ * frequencies, written on the device by the same device code the rotary
+ * kernels use.
+ * Interleaved ([QVL] apply_interleaved_mrope; [M01] problem summary): H where
+ * j % 3 == 1 and j < 3*section[1]; W where j % 3 == 2 and j < 3*section[2];
+ * T elsewhere.  Chunked ([M01] step-by-step figure, Qwen2-VL / Qwen2.5-Omni):
+ * T for j < section[0], H for j < section[0] + section[1], W after.
+ *   half        1 .. IPE_MAX_HALF
+ *   section     host int32[3] = mrope_section (s_t, s_h, s_w), each >= 0, sum == half
+ *   interleaved 1 for interleaved (Qwen3-VL / Qwen3.5 / Qwen3-Omni), 0 for chunked
+ *   axis_dev    device int8[half], written.
+ * ------------------------------------------------------------------------- */
+int ipe_mrope_axis_map(int half, const int32_t *section, int interleaved, int8_t *axis_dev,
+                       void *stream);
+
+/* ---------------------------------------------------------------------------
+ * ipe_mrope_cos_sin -- multimodal RoPE cos / sin tables.
+ * [QVL] Qwen3VLTextRotaryEmbedding.forward; [M01] shape trace rows 2-7:
+ *   angle[t, j] = fl32(fl32(positions[axis(j), t]) * inv_freq[j])
+ *   cos[t, j] = cos[t, j + half] = cos(angle[t, j]); likewise sin
+ * (emb = cat(f, f); attention_scaling = 1).  Kept in fp32 (no cast to the
+ * activation dtype).
+ *   positions      device int32 [3, T] row-major (rows t, h, w; row stride T),
+ *                  values in [0, IPE_MAX_POSITION) (precondition, not checked
+ *                  on the device)
+ *   T              tokens, >= 0 (T = B*L for a batch of B sequences of length L)
+ *   inv_freq_host  host float[half]
+ *   half           rot_dim / 2, 1 .. IPE_MAX_HALF
+ *   section, interleaved  as for ipe_mrope_axis_map
+ *   cos_out, sin_out  device float [T, 2*half] row-major, written.
+ * ------------------------------------------------------------------------- */
+int ipe_mrope_cos_sin(const int32_t *positions, int64_t T, const float *inv_freq_host, int half,
+                      const int32_t *section, int interleaved, float *cos_out, float *sin_out,
+                      void *stream);
+
+/* ---------------------------------------------------------------------------
+ * ipe_apply_rotary_partial -- rotate_half rotation of the first rot_dim
+ * channels of every head of Q and K, in place; channels >= rot_dim untouched.
+ * [IRPE] rotate_half / apply_rotary_pos_emb (partial rotary); [M01] L1 hints:
+ *   h = rot_dim/2; for j < h:
+ *   x'[j]     = x[j] * cos[t, j]         - x[j + h] * sin[t, j]
+ *   x'[j + h] = x[j + h] * cos[t, j + h] + x[j] * sin[t, j + h]
+ * cos / sin are shared by all heads of a token.
+ *   q, k          device, dtype, token-major [T, hq, head_dim] / [T, hk, head_dim];
+ *                 heads contiguous (head stride = head_dim); token strides
+ *                 q_tok_stride, k_tok_stride (>= heads * head_dim).  k may be
+ *                 NULL iff hk == 0, q NULL iff hq == 0.
+ *   dtype         IPE_BF16 or IPE_F32
+ *   rot_dim       even, 2 .. min(head_dim, 2*IPE_MAX_HALF)
+ *   cos, sin      device float [T, rot_dim] row-major (e.g. from ipe_mrope_cos_sin)
+ * Vector alignment: accesses are as wide as rot_dim/2, head_dim, the strides
+ * and the pointers allow (up to 16 bytes); no alignment is required.
+ * ------------------------------------------------------------------------- */
+int ipe_apply_rotary_partial(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk,
+                             int head_dim, int64_t q_tok_stride, int64_t k_tok_stride,
+                             const float *cos, const float *sin, int rot_dim, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * ipe_mrope_apply -- ipe_mrope_cos_sin followed by ipe_apply_rotary_partial in
+ * one pass: each (token, frequency) angle and its sincosf are computed once
+ * and shared by all hq + hk heads; cos / sin are never written to memory.
+ * Same arguments and results as the two calls it replaces, with
+ * rot_dim = 2 * half.
+ * ------------------------------------------------------------------------- */
+int ipe_mrope_apply(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
+                    int64_t q_tok_stride, int64_t k_tok_stride, const int32_t *positions,
+                    const float *inv_freq_host, int rot_dim, const int32_t *section,
+                    int interleaved, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Vision grids.  grid_thw_host is a host int32 [n_images, 3] array of
+ * (t, h, w) patch grids BEFORE the spatial merge ([VLM] 1.1 Patch; [IRPE]
+ * get_rope_index); h and w must be multiples of `merge` (spatial_merge_size,
+ * 2 in Qwen3-VL).  Patches of all images are concatenated in grid_thw order
+ * (image i starts at row sum_{j<i} t_j h_j w_j, its cu_seqlens offset); within
+ * an image, frame-major, then merge-block row, merge-block column, and the
+ * merge x merge patches of a block row-major ([QVL] fast_pos_embed_interpolate
+ * permute(0, 1, 3, 2, 4, 5); [CRT] positions()).
+ * ------------------------------------------------------------------------- */
+
+/* ---------------------------------------------------------------------------
+ * ipe_vis_interp_plan -- corner ids, weights and (row, col) of every patch in
+ * output order, written by the device code of the interpolation kernels.
+ * [QVL] fast_pos_embed_interpolate: sample y = row (G-1)/(h-1) (0 when h = 1),
+ * y0 = floor(y), y1 = min(y0 + 1, G-1), dy = y - y0 (likewise x); corners
+ * TL, TR, BL, BR = (y0 G + x0, y0 G + x1, y1 G + x0, y1 G + x1), weights
+ * ((1-dy)(1-dx), (1-dy)dx, dy(1-dx), dy dx).  Corners use integer arithmetic
+ * (y0 = row (G-1) div (h-1)); dy = fl32((row (G-1) mod (h-1)) / (h-1)).
+ *   grid_side  G, the side of the learned table (48), 1 .. 256
+ *   idx4       device int32 [4, N] or NULL; w4 device float [4, N] or NULL;
+ *   rowcol     device int32 [2, N] or NULL (row, col of each patch).
+ * ------------------------------------------------------------------------- */
+int ipe_vis_interp_plan(const int32_t *grid_thw_host, int n_images, int merge, int grid_side,
+                        int32_t *idx4, float *w4, int32_t *rowcol, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * ipe_vis_pos_interp -- learned position table interpolated to each image's
+ * patch grid, in merge order ([QVL] fast_pos_embed_interpolate; [CRT]
+ * positions()):  out[k, :] = sum_c w_c(k) table[idx_c(k), :].
+ * Frames of a video repeat frame 0.  Computed in fp32 as the separable form
+ * (1-dx)((1-dy) T[y0,x0] + dy T[y1,x0]) + dx((1-dy) T[y0,x1] + dy T[y1,x1]),
+ * equal to the four-weight sum in exact arithmetic, rounded once.
+ *   table      device [G*G, hidden], dtype (row id = y G + x)
+ *   hidden     channels, multiple of 4 (1152 in Qwen3-VL)
+ *   out        device [N, hidden], dtype, written; N = sum t h w.
+ * ------------------------------------------------------------------------- */
+int ipe_vis_pos_interp(const void *table, ipe_dtype dtype, int grid_side, int hidden,
+                       const int32_t *grid_thw_host, int n_images, int merge, void *out,
+                       void *stream);
+
+/* ---------------------------------------------------------------------------
+ * ipe_vis_rope2d -- vision 2-D rotary over the whole head, in place on q and k.
+ * [QVL] rot_pos_emb + apply_rotary_pos_emb_vision; [CRT] rope_angles(),
+ * attention():  with f = head_dim/4 frequencies inv[i] = fl32(1/theta^(2i/(head_dim/2)))
+ * and (row, col) the patch's grid position, angle a[i] = fl32(row * inv[i]),
+ * a[f + i] = fl32(col * inv[i]) (i < f), and for j < head_dim/2:
+ *   x'[j] = x[j] cos a[j] - x[j + head_dim/2] sin a[j]
+ *   x'[j + head_dim/2] = x[j + head_dim/2] cos a[j] + x[j] sin a[j].
+ * One sincosf per (patch, angle), shared by every head of q and k.
+ *   q, k       device [n_patch, heads, head_dim], dtype; heads contiguous;
+ *              patch strides q_stride, k_stride (>= heads * head_dim); k may be
+ *              NULL (q only)
+ *   n_patch    must equal sum t h w of grid_thw
+ *   head_dim   multiple of 4 (72 in Qwen3-VL); theta > 0 (1e4).
+ * ------------------------------------------------------------------------- */
+int ipe_vis_rope2d(void *q, void *k, ipe_dtype dtype, int64_t n_patch, int heads, int head_dim,
+                   int64_t q_stride, int64_t k_stride, const int32_t *grid_thw_host,
+                   int n_images, int merge, double theta, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * ipe_vis_pos_interp_rope2d -- ipe_vis_pos_interp and ipe_vis_rope2d on the
+ * same images in one launch (one descriptor, one plan decode).  Arguments as
+ * for the two calls; one dtype for table, out, q and k.
+ * ------------------------------------------------------------------------- */
+int ipe_vis_pos_interp_rope2d(const void *table, int grid_side, int hidden, void *out, void *q,
+                              void *k, int heads, int head_dim, int64_t q_stride, int64_t k_stride,
+                              double theta, ipe_dtype dtype, const int32_t *grid_thw_host,
+                              int n_images, int merge, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IPE_H */

@@ -1,0 +1,285 @@
+"""Python binding of libipe.so, the B200 interpolated-position-encoding library.
+
+Argument marshalling only: each function checks that its tensors are on the
+GPU, passes ``data_ptr()``, sizes, strides and the current CUDA stream to the
+C entry point of the same name (``include/ipe.h``) and raises
+``IpeError`` with the library's message on a non-OK status.  Every step of
+the computation runs in the library's CUDA kernels; there is no other path.
+PyTorch is used for device memory and streams only.
+
+Build the library first: ``python -m interpolated_position_encoding_b200.build``.
+"""
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+_LIB_PATH = _build.LIB
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build it with `python -m interpolated_position_encoding_b200.build` "
+        "(nvcc for sm_100a); there is no fallback implementation")
+
+_lib = ctypes.CDLL(_LIB_PATH)
+
+_P, _I, _I64, _D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+
+_SIGS = {
+    "ipe_last_error": (ctypes.c_char_p, []),
+    "ipe_version": (_I, []),
+    "ipe_rope_inv_freq": (_I, [_I, _D, _P]),
+    "ipe_mrope_axis_map": (_I, [_I, _P, _I, _P, _P]),
+    "ipe_mrope_cos_sin": (_I, [_P, _I64, _P, _I, _P, _I, _P, _P, _P]),
+    "ipe_apply_rotary_partial": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, _I, _P]),
+    "ipe_mrope_apply": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, _I, _P, _I, _P]),
+    "ipe_vis_interp_plan": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
+    "ipe_vis_pos_interp": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P]),
+    "ipe_vis_rope2d": (_I, [_P, _P, _I, _I64, _I, _I, _I64, _I64, _P, _I, _I, _D, _P]),
+    "ipe_vis_pos_interp_rope2d": (_I, [_P, _I, _I, _P, _P, _P, _I, _I, _I64, _I64, _D, _I, _P, _I, _I, _P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTS = tuple(_SIGS)
+
+IPE_F32, IPE_BF16 = 0, 1
+IPE_OK, IPE_EINVAL, IPE_EALIGN, IPE_ELIMIT, IPE_ECUDA = 0, 1, 2, 3, 4
+_STATUS = {1: "IPE_EINVAL", 2: "IPE_EALIGN", 3: "IPE_ELIMIT", 4: "IPE_ECUDA"}
+
+
+class IpeError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def _check(rc):
+    if rc != IPE_OK:
+        raise IpeError(rc, _lib.ipe_last_error().decode())
+
+
+def lib():
+    """The loaded ctypes library (raw C entry points)."""
+    return _lib
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return IPE_BF16
+    if t.dtype == torch.float32:
+        return IPE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: bfloat16 or float32")
+
+
+def _cuda(t, name):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    return t
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _i32_host(values, n=None):
+    arr = (ctypes.c_int32 * len(values))(*[int(v) for v in values])
+    if n is not None and len(values) != n:
+        raise ValueError(f"expected {n} values, got {len(values)}")
+    return arr
+
+
+def _grid_host(grid_thw):
+    if isinstance(grid_thw, torch.Tensor):
+        grid_thw = grid_thw.detach().cpu().reshape(-1).tolist()
+    else:
+        grid_thw = [int(v) for g in grid_thw for v in (g if hasattr(g, "__len__") else [g])]
+    if len(grid_thw) % 3:
+        raise ValueError("grid_thw must hold (t, h, w) triples")
+    return _i32_host(grid_thw), len(grid_thw) // 3
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _row_stride(t, heads, head_dim, name):
+    """Token stride of a [rows, heads, head_dim] view with contiguous heads."""
+    if t.dim() != 3 or t.shape[1] != heads or t.shape[2] != head_dim:
+        raise ValueError(f"{name} must be [rows, {heads}, {head_dim}], got {tuple(t.shape)}")
+    if t.stride(2) != 1 or (heads > 1 and t.stride(1) != head_dim):
+        raise ValueError(f"{name}: heads must be contiguous (strides {t.stride()})")
+    return t.stride(0)
+
+
+# --------------------------------------------------------------------- text
+
+
+def rope_inv_freq(rot_dim, theta):
+    """Default RoPE inverse frequencies (fp32, computed on the host by the library)."""
+    out = (ctypes.c_float * (rot_dim // 2))()
+    _check(_lib.ipe_rope_inv_freq(int(rot_dim), float(theta), out))
+    return torch.tensor(list(out), dtype=torch.float32)
+
+
+def mrope_axis_map(half, section, interleaved=True, device="cuda", stream=None):
+    """int8 [half]: axis (0 = T, 1 = H, 2 = W) of each frequency."""
+    out = torch.empty(half, dtype=torch.int8, device=device)
+    _check(_lib.ipe_mrope_axis_map(int(half), _i32_host(section, 3), int(bool(interleaved)), _ptr(out),
+                                   _stream(stream)))
+    return out
+
+
+def _inv_host(inv_freq):
+    vals = inv_freq.detach().float().cpu().tolist() if isinstance(inv_freq, torch.Tensor) else list(inv_freq)
+    return (ctypes.c_float * len(vals))(*vals), len(vals)
+
+
+def mrope_cos_sin(positions, inv_freq, section, interleaved=True, cos=None, sin=None, stream=None):
+    """cos, sin fp32 [T, 2*half] from int32 positions [3, T]."""
+    _cuda(positions, "positions")
+    if positions.dtype != torch.int32 or positions.dim() != 2 or positions.shape[0] != 3 or not positions.is_contiguous():
+        raise ValueError("positions must be a contiguous int32 [3, T] tensor")
+    T = positions.shape[1]
+    inv, half = _inv_host(inv_freq)
+    if cos is None:
+        cos = torch.empty(T, 2 * half, dtype=torch.float32, device=positions.device)
+    if sin is None:
+        sin = torch.empty(T, 2 * half, dtype=torch.float32, device=positions.device)
+    for t, n in ((cos, "cos"), (sin, "sin")):
+        _cuda(t, n)
+        if t.dtype != torch.float32 or tuple(t.shape) != (T, 2 * half) or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous float32 [{T}, {2 * half}] tensor")
+    _check(_lib.ipe_mrope_cos_sin(_ptr(positions), T, inv, half, _i32_host(section, 3), int(bool(interleaved)),
+                                  _ptr(cos), _ptr(sin), _stream(stream)))
+    return cos, sin
+
+
+def _qk_args(q, k):
+    _cuda(q, "q")
+    _cuda(k, "k")
+    ref = q if q is not None else k
+    if ref is None:
+        raise ValueError("q and k are both None")
+    if q is not None and k is not None and q.dtype != k.dtype:
+        raise TypeError("q and k must share a dtype")
+    T, head_dim = ref.shape[0], ref.shape[2]
+    hq = q.shape[1] if q is not None else 0
+    hk = k.shape[1] if k is not None else 0
+    qs = _row_stride(q, hq, head_dim, "q") if q is not None else 0
+    ks = _row_stride(k, hk, head_dim, "k") if k is not None else 0
+    if k is not None and k.shape[0] != T:
+        raise ValueError("q and k must have the same number of rows")
+    return _dtype_code(ref), T, hq, hk, head_dim, qs, ks
+
+
+def apply_rotary_partial(q, k, cos, sin, stream=None):
+    """In place: rotate_half rotation of the first cos.shape[1] channels of q [T, hq, D], k [T, hk, D]."""
+    dt, T, hq, hk, D, qs, ks = _qk_args(q, k)
+    for t, n in ((cos, "cos"), (sin, "sin")):
+        _cuda(t, n)
+        if t.dtype != torch.float32 or t.dim() != 2 or t.shape[0] != T or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous float32 [T, rot_dim] tensor")
+    _check(_lib.ipe_apply_rotary_partial(_ptr(q), _ptr(k), dt, T, hq, hk, D, qs, ks, _ptr(cos), _ptr(sin),
+                                         cos.shape[1], _stream(stream)))
+    return q, k
+
+
+def mrope_apply(q, k, positions, inv_freq, section, interleaved=True, stream=None):
+    """In place: fused multimodal RoPE of q [T, hq, D] and k [T, hk, D] (cos / sin stay in registers)."""
+    dt, T, hq, hk, D, qs, ks = _qk_args(q, k)
+    _cuda(positions, "positions")
+    if positions.dtype != torch.int32 or tuple(positions.shape) != (3, T) or not positions.is_contiguous():
+        raise ValueError("positions must be a contiguous int32 [3, T] tensor")
+    inv, half = _inv_host(inv_freq)
+    _check(_lib.ipe_mrope_apply(_ptr(q), _ptr(k), dt, T, hq, hk, D, qs, ks, _ptr(positions), inv, 2 * half,
+                                _i32_host(section, 3), int(bool(interleaved)), _stream(stream)))
+    return q, k
+
+
+# ------------------------------------------------------------------- vision
+
+
+def vis_interp_plan(grid_thw, merge=2, grid_side=48, device="cuda", stream=None):
+    """(idx4 int32 [4, N], w4 float32 [4, N], rowcol int32 [2, N]) in output order."""
+    g, n = _grid_host(grid_thw)
+    N = sum(g[3 * i] * g[3 * i + 1] * g[3 * i + 2] for i in range(n))
+    idx4 = torch.empty(4, N, dtype=torch.int32, device=device)
+    w4 = torch.empty(4, N, dtype=torch.float32, device=device)
+    rowcol = torch.empty(2, N, dtype=torch.int32, device=device)
+    _check(_lib.ipe_vis_interp_plan(g, n, int(merge), int(grid_side), _ptr(idx4), _ptr(w4), _ptr(rowcol),
+                                    _stream(stream)))
+    return idx4, w4, rowcol
+
+
+def _table_args(table):
+    _cuda(table, "table")
+    if table.dim() != 2 or not table.is_contiguous():
+        raise ValueError("table must be a contiguous [G*G, hidden] tensor")
+    G = int(round(table.shape[0] ** 0.5))
+    if G * G != table.shape[0]:
+        raise ValueError("table rows must be a square grid G*G")
+    return G, table.shape[1]
+
+
+def vis_pos_interp(table, grid_thw, merge=2, out=None, stream=None):
+    """[N, hidden] interpolated position embeddings in merge order, dtype of the table."""
+    G, C = _table_args(table)
+    g, n = _grid_host(grid_thw)
+    N = sum(g[3 * i] * g[3 * i + 1] * g[3 * i + 2] for i in range(n))
+    if out is None:
+        out = torch.empty(N, C, dtype=table.dtype, device=table.device)
+    _cuda(out, "out")
+    if out.dtype != table.dtype or tuple(out.shape) != (N, C) or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous [{N}, {C}] tensor of the table's dtype")
+    _check(_lib.ipe_vis_pos_interp(_ptr(table), _dtype_code(table), G, C, g, n, int(merge), _ptr(out),
+                                   _stream(stream)))
+    return out
+
+
+def vis_rope2d(q, k, grid_thw, merge=2, theta=1e4, stream=None):
+    """In place: vision 2-D rotary of q, k [N, heads, head_dim] (k may be None)."""
+    _cuda(q, "q")
+    _cuda(k, "k")
+    heads, D = q.shape[1], q.shape[2]
+    qs = _row_stride(q, heads, D, "q")
+    ks = _row_stride(k, heads, D, "k") if k is not None else 0
+    if k is not None and (k.dtype != q.dtype or k.shape[0] != q.shape[0]):
+        raise ValueError("k must match q in dtype and rows")
+    g, n = _grid_host(grid_thw)
+    _check(_lib.ipe_vis_rope2d(_ptr(q), _ptr(k), _dtype_code(q), q.shape[0], heads, D, qs, ks, g, n, int(merge),
+                               float(theta), _stream(stream)))
+    return q, k
+
+
+def vis_pos_interp_rope2d(table, grid_thw, q, k, merge=2, theta=1e4, out=None, stream=None):
+    """One launch: interpolated position embeddings (returned) and in-place 2-D rotary of q, k."""
+    G, C = _table_args(table)
+    g, n = _grid_host(grid_thw)
+    N = sum(g[3 * i] * g[3 * i + 1] * g[3 * i + 2] for i in range(n))
+    if out is None:
+        out = torch.empty(N, C, dtype=table.dtype, device=table.device)
+    _cuda(out, "out")
+    _cuda(q, "q")
+    _cuda(k, "k")
+    if out.dtype != table.dtype or q.dtype != table.dtype or (k is not None and k.dtype != table.dtype):
+        raise TypeError("table, out, q and k must share a dtype")
+    if tuple(out.shape) != (N, C) or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous [{N}, {C}] tensor")
+    heads, D = q.shape[1], q.shape[2]
+    qs = _row_stride(q, heads, D, "q")
+    ks = _row_stride(k, heads, D, "k") if k is not None else 0
+    _check(_lib.ipe_vis_pos_interp_rope2d(_ptr(table), G, C, _ptr(out), _ptr(q), _ptr(k), heads, D, qs, ks,
+                                          float(theta), _dtype_code(table), g, n, int(merge), _stream(stream)))
+    return out, q, k
+
+
+__all__ = ["IpeError", "lib", "EXPORTS", "rope_inv_freq", "mrope_axis_map", "mrope_cos_sin", "apply_rotary_partial",
+           "mrope_apply", "vis_interp_plan", "vis_pos_interp", "vis_rope2d", "vis_pos_interp_rope2d"]

@@ -1,0 +1,441 @@
+// C ABI of libipe.so: argument validation, descriptor packing and launches on
+// the caller's stream.  See include/ipe.h for the contract of every entry
+// point.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include <cuda.h>   // CUresult / CUdeviceptr types only; the driver call is resolved at run time
+
+#include "../../include/ipe.h"
+#include "ipe_internal.h"
+
+using namespace ipe;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int ok()
+{
+    g_err.clear();
+    return IPE_OK;
+}
+
+int cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(IPE_ECUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+// cuMemGetAddressRange through the runtime's driver entry point (no link
+// dependency on libcuda, so the library loads on machines without a GPU).
+typedef CUresult (*AddressRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+AddressRangeFn address_range_fn()
+{
+    static AddressRangeFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<AddressRangeFn>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// `p` must be device (or managed) memory of the current device whose
+// allocation covers [p, p + bytes).
+int check_dev(const void *p, size_t bytes, const char *name)
+{
+    if (bytes == 0) return IPE_OK;
+    if (p == nullptr) return fail(IPE_EINVAL, "%s is NULL", name);
+    cudaPointerAttributes at;
+    cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(e, name);
+    }
+    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
+        return fail(IPE_EINVAL, "%s is not device memory", name);
+    int dev = -1;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (at.type == cudaMemoryTypeDevice && at.device != dev)
+        return fail(IPE_EINVAL, "%s lives on device %d, current device is %d", name, at.device, dev);
+    if (AddressRangeFn fn = address_range_fn()) {
+        CUdeviceptr base = 0;
+        size_t size = 0;
+        if (fn(&base, &size, (CUdeviceptr)(uintptr_t)p) == CUDA_SUCCESS) {
+            const uintptr_t end = (uintptr_t)base + size;
+            if ((uintptr_t)p + bytes > end || (uintptr_t)p + bytes < (uintptr_t)p)
+                return fail(IPE_EINVAL, "%s: %zu bytes from the pointer run past its allocation (%zu bytes left)",
+                            name, bytes, (size_t)(end - (uintptr_t)p));
+        }
+    }
+    return IPE_OK;
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int elem_bytes(ipe_dtype dt) { return dt == IPE_BF16 ? 2 : 4; }
+
+int check_dtype(int dt)
+{
+    if (dt != IPE_F32 && dt != IPE_BF16) return fail(IPE_EINVAL, "dtype %d is neither IPE_F32 nor IPE_BF16", dt);
+    return IPE_OK;
+}
+
+int check_section(int half, const int32_t *section)
+{
+    if (section == nullptr) return fail(IPE_EINVAL, "section is NULL");
+    if (section[0] < 0 || section[1] < 0 || section[2] < 0)
+        return fail(IPE_EINVAL, "mrope_section (%d, %d, %d) has a negative count", section[0], section[1], section[2]);
+    if ((long long)section[0] + section[1] + section[2] != half)
+        return fail(IPE_EINVAL, "mrope_section (%d, %d, %d) sums to %lld, not rot_dim/2 = %d", section[0],
+                    section[1], section[2], (long long)section[0] + section[1] + section[2], half);
+    return IPE_OK;
+}
+
+int check_half(int half)
+{
+    if (half < 1) return fail(IPE_EINVAL, "rot_dim/2 = %d must be >= 1", half);
+    if (half > IPE_MAX_HALF) return fail(IPE_ELIMIT, "rot_dim/2 = %d is above IPE_MAX_HALF = %d", half, IPE_MAX_HALF);
+    return IPE_OK;
+}
+
+// Bytes spanned by `rows` rows of `heads` heads of `head_dim` elements.
+size_t span_bytes(long long rows, long long stride, int heads, int head_dim, int eb)
+{
+    if (rows <= 0 || heads <= 0) return 0;
+    return (size_t)(((rows - 1) * stride + (long long)heads * head_dim) * eb);
+}
+
+// Head-row tensors of a rotation call.
+int check_qk(void *q, void *k, ipe_dtype dt, long long rows, int hq, int hk, int head_dim, long long qs,
+             long long ks, const char *qn, const char *kn)
+{
+    if (rows < 0) return fail(IPE_EINVAL, "row count %lld is negative", rows);
+    if (hq < 0 || hk < 0) return fail(IPE_EINVAL, "head counts (%d, %d) must be >= 0", hq, hk);
+    if (head_dim <= 0) return fail(IPE_EINVAL, "head_dim %d must be > 0", head_dim);
+    if (hq > 0 && qs < (long long)hq * head_dim)
+        return fail(IPE_EINVAL, "%s row stride %lld < heads * head_dim = %lld", qn, qs, (long long)hq * head_dim);
+    if (hk > 0 && ks < (long long)hk * head_dim)
+        return fail(IPE_EINVAL, "%s row stride %lld < heads * head_dim = %lld", kn, ks, (long long)hk * head_dim);
+    if (hq > 0 && q == nullptr) return fail(IPE_EINVAL, "%s is NULL but has %d heads", qn, hq);
+    if (hk > 0 && k == nullptr) return fail(IPE_EINVAL, "%s is NULL but has %d heads", kn, hk);
+    const int eb = elem_bytes(dt);
+    if (!aligned(q, eb) || !aligned(k, eb)) return fail(IPE_EALIGN, "%s / %s not aligned to the element size", qn, kn);
+    if (hq > 0) {
+        if (int rc = check_dev(q, span_bytes(rows, qs, hq, head_dim, eb), qn)) return rc;
+    }
+    if (hk > 0) {
+        if (int rc = check_dev(k, span_bytes(rows, ks, hk, head_dim, eb), kn)) return rc;
+    }
+    if (rows > 0 && (long long)(hq + hk) * head_dim > (1LL << 30))
+        return fail(IPE_ELIMIT, "heads * head_dim too large");
+    return IPE_OK;
+}
+
+// Vision descriptor from host grid_thw.
+int build_vis_desc(const int32_t *grid, int n_images, int merge, int grid_side, VisDesc<1024> &d)
+{
+    if (grid == nullptr && n_images > 0) return fail(IPE_EINVAL, "grid_thw is NULL");
+    if (n_images < 0) return fail(IPE_EINVAL, "n_images %d is negative", n_images);
+    if (n_images > IPE_MAX_IMAGES)
+        return fail(IPE_ELIMIT, "n_images %d is above IPE_MAX_IMAGES = %d", n_images, IPE_MAX_IMAGES);
+    if (merge < 1 || merge > 8) return fail(IPE_EINVAL, "merge %d must be in 1 .. 8", merge);
+    if (grid_side < 1 || grid_side > 256) return fail(IPE_EINVAL, "grid_side %d must be in 1 .. 256", grid_side);
+    d.n_images = n_images;
+    d.merge = merge;
+    d.grid_side = grid_side;
+    long long row = 0;
+    long long strips = 0;
+    for (int i = 0; i < n_images; ++i) {
+        const int t = grid[3 * i], h = grid[3 * i + 1], w = grid[3 * i + 2];
+        if (t < 1 || h < 1 || w < 1)
+            return fail(IPE_EINVAL, "grid_thw[%d] = (%d, %d, %d) has a non-positive size", i, t, h, w);
+        if (h % merge || w % merge)
+            return fail(IPE_EINVAL, "grid_thw[%d] = (%d, %d, %d): h and w must be multiples of merge %d", i, t, h,
+                        w, merge);
+        if (h > 65536 || w > 65536 || t > 65536)
+            return fail(IPE_ELIMIT, "grid_thw[%d] = (%d, %d, %d): sides above 65536", i, t, h, w);
+        d.img[i].t = t;
+        d.img[i].h = h;
+        d.img[i].w = w;
+        d.img[i].strip0 = (int)strips;
+        d.img[i].row0 = row;
+        row += (long long)t * h * w;
+        strips += h / merge;
+    }
+    if (row > (1LL << 31) - 1) return fail(IPE_ELIMIT, "more than 2^31 - 1 patches");
+    if (strips > (1LL << 24)) return fail(IPE_ELIMIT, "too many merge-row strips");
+    d.n_patch = row;
+    d.n_strips = (int)strips;
+    return IPE_OK;
+}
+
+int vis_freqs(int head_dim, double theta, VisAngleFreqs &f)
+{
+    if (head_dim <= 0 || head_dim % 4) return fail(IPE_EINVAL, "vision head_dim %d must be a positive multiple of 4", head_dim);
+    if (head_dim / 4 > kMaxVisFreq) return fail(IPE_ELIMIT, "vision head_dim %d above %d", head_dim, 4 * kMaxVisFreq);
+    if (!(theta > 0.0) || !std::isfinite(theta)) return fail(IPE_EINVAL, "theta must be finite and > 0");
+    const int dim = head_dim / 2;
+    f.nf = head_dim / 4;
+    for (int i = 0; i < f.nf; ++i) f.inv[i] = (float)(1.0 / std::pow(theta, (double)(2 * i) / (double)dim));
+    return IPE_OK;
+}
+
+// Per-thread host buffer of the vision descriptor (about 25 KB).
+VisDesc<1024> *desc_buffer()
+{
+    thread_local VisDesc<1024> *dp = nullptr;
+    if (!dp) dp = new VisDesc<1024>();
+    return dp;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ipe_last_error(void) { return g_err.c_str(); }
+
+int ipe_version(void) { return 100; }
+
+int ipe_rope_inv_freq(int rot_dim, double theta, float *inv_freq_host)
+{
+    if (rot_dim < 2 || rot_dim % 2) return fail(IPE_EINVAL, "rot_dim %d must be even and >= 2", rot_dim);
+    if (rot_dim / 2 > IPE_MAX_HALF) return fail(IPE_ELIMIT, "rot_dim %d above 2*IPE_MAX_HALF", rot_dim);
+    if (!(theta > 0.0) || !std::isfinite(theta)) return fail(IPE_EINVAL, "theta must be finite and > 0");
+    if (inv_freq_host == nullptr) return fail(IPE_EINVAL, "inv_freq_host is NULL");
+    for (int j = 0; j < rot_dim / 2; ++j)
+        inv_freq_host[j] = (float)(1.0 / std::pow(theta, (double)(2 * j) / (double)rot_dim));
+    return ok();
+}
+
+int ipe_mrope_axis_map(int half, const int32_t *section, int interleaved, int8_t *axis_dev, void *stream)
+{
+    if (int rc = check_half(half)) return rc;
+    if (int rc = check_section(half, section)) return rc;
+    if (int rc = check_dev(axis_dev, (size_t)half, "axis_dev")) return rc;
+    cudaError_t e = launch_mrope_axis_map(half, section, interleaved ? 1 : 0, axis_dev, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "mrope_axis_map launch");
+}
+
+static int fill_mrope(MropeAngles &a, const int32_t *positions, int64_t T, const float *inv, int half,
+                      const int32_t *section, int interleaved)
+{
+    if (T < 0) return fail(IPE_EINVAL, "T = %lld is negative", (long long)T);
+    if (T > (1LL << 40)) return fail(IPE_ELIMIT, "T = %lld too large", (long long)T);
+    if (int rc = check_half(half)) return rc;
+    if (int rc = check_section(half, section)) return rc;
+    if (inv == nullptr) return fail(IPE_EINVAL, "inv_freq_host is NULL");
+    for (int j = 0; j < half; ++j)
+        if (!std::isfinite(inv[j])) return fail(IPE_EINVAL, "inv_freq[%d] is not finite", j);
+    if (T > 0 && !aligned(positions, 4)) return fail(IPE_EALIGN, "positions not 4-byte aligned");
+    a.positions = positions;
+    a.T = T;
+    a.section[0] = section[0];
+    a.section[1] = section[1];
+    a.section[2] = section[2];
+    a.interleaved = interleaved ? 1 : 0;
+    for (int j = 0; j < half; ++j) a.inv[j] = inv[j];
+    for (int j = half; j < kMaxHalf; ++j) a.inv[j] = 0.f;
+    return IPE_OK;
+}
+
+int ipe_mrope_cos_sin(const int32_t *positions, int64_t T, const float *inv_freq_host, int half,
+                      const int32_t *section, int interleaved, float *cos_out, float *sin_out, void *stream)
+{
+    MropeAngles a;
+    if (int rc = fill_mrope(a, positions, T, inv_freq_host, half, section, interleaved)) return rc;
+    if (T == 0) return ok();
+    if (!aligned(cos_out, 4) || !aligned(sin_out, 4)) return fail(IPE_EALIGN, "cos_out / sin_out not 4-byte aligned");
+    if (int rc = check_dev(positions, (size_t)(3 * T) * 4, "positions")) return rc;
+    if (int rc = check_dev(cos_out, (size_t)T * 2 * half * 4, "cos_out")) return rc;
+    if (int rc = check_dev(sin_out, (size_t)T * 2 * half * 4, "sin_out")) return rc;
+    cudaError_t e = launch_mrope_cos_sin(a, half, cos_out, sin_out, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "mrope_cos_sin launch");
+}
+
+int ipe_apply_rotary_partial(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
+                             int64_t q_tok_stride, int64_t k_tok_stride, const float *cos, const float *sin,
+                             int rot_dim, void *stream)
+{
+    if (int rc = check_dtype(dtype)) return rc;
+    if (rot_dim < 2 || rot_dim % 2) return fail(IPE_EINVAL, "rot_dim %d must be even and >= 2", rot_dim);
+    if (int rc = check_half(rot_dim / 2)) return rc;
+    if (rot_dim > head_dim) return fail(IPE_EINVAL, "rot_dim %d > head_dim %d", rot_dim, head_dim);
+    if (int rc = check_qk(q, k, dtype, T, hq, hk, head_dim, q_tok_stride, k_tok_stride, "q", "k")) return rc;
+    if (T == 0 || hq + hk == 0) return ok();
+    if (!aligned(cos, 4) || !aligned(sin, 4)) return fail(IPE_EALIGN, "cos / sin not 4-byte aligned");
+    if (int rc = check_dev(cos, (size_t)T * rot_dim * 4, "cos")) return rc;
+    if (int rc = check_dev(sin, (size_t)T * rot_dim * 4, "sin")) return rc;
+    RotArgs r{};
+    r.q = hq ? q : nullptr;
+    r.k = hk ? k : nullptr;
+    r.rows = T;
+    r.q_stride = q_tok_stride;
+    r.k_stride = k_tok_stride;
+    r.hq = hq;
+    r.hk = hk;
+    r.head_dim = head_dim;
+    r.half = rot_dim / 2;
+    TableAngles a{cos, sin};
+    cudaError_t e = launch_rotary_table(dtype == IPE_BF16, r, a, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "apply_rotary_partial launch");
+}
+
+int ipe_mrope_apply(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
+                    int64_t q_tok_stride, int64_t k_tok_stride, const int32_t *positions, const float *inv_freq_host,
+                    int rot_dim, const int32_t *section, int interleaved, void *stream)
+{
+    if (int rc = check_dtype(dtype)) return rc;
+    if (rot_dim < 2 || rot_dim % 2) return fail(IPE_EINVAL, "rot_dim %d must be even and >= 2", rot_dim);
+    if (rot_dim > head_dim) return fail(IPE_EINVAL, "rot_dim %d > head_dim %d", rot_dim, head_dim);
+    MropeAngles a;
+    if (int rc = fill_mrope(a, positions, T, inv_freq_host, rot_dim / 2, section, interleaved)) return rc;
+    if (int rc = check_qk(q, k, dtype, T, hq, hk, head_dim, q_tok_stride, k_tok_stride, "q", "k")) return rc;
+    if (T == 0 || hq + hk == 0) return ok();
+    if (int rc = check_dev(positions, (size_t)(3 * T) * 4, "positions")) return rc;
+    RotArgs r{};
+    r.q = hq ? q : nullptr;
+    r.k = hk ? k : nullptr;
+    r.rows = T;
+    r.q_stride = q_tok_stride;
+    r.k_stride = k_tok_stride;
+    r.hq = hq;
+    r.hk = hk;
+    r.head_dim = head_dim;
+    r.half = rot_dim / 2;
+    cudaError_t e = launch_rotary_mrope(dtype == IPE_BF16, r, a, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "mrope_apply launch");
+}
+
+int ipe_vis_interp_plan(const int32_t *grid_thw_host, int n_images, int merge, int grid_side, int32_t *idx4,
+                        float *w4, int32_t *rowcol, void *stream)
+{
+    VisDesc<1024> &d = *desc_buffer();
+    if (int rc = build_vis_desc(grid_thw_host, n_images, merge, grid_side, d)) return rc;
+    const long long N = d.n_patch;
+    if (N == 0) return ok();
+    if (!aligned(idx4, 4) || !aligned(w4, 4) || !aligned(rowcol, 4)) return fail(IPE_EALIGN, "outputs not 4-byte aligned");
+    if (idx4) {
+        if (int rc = check_dev(idx4, (size_t)4 * N * 4, "idx4")) return rc;
+    }
+    if (w4) {
+        if (int rc = check_dev(w4, (size_t)4 * N * 4, "w4")) return rc;
+    }
+    if (rowcol) {
+        if (int rc = check_dev(rowcol, (size_t)2 * N * 4, "rowcol")) return rc;
+    }
+    cudaError_t e = launch_vis_plan(d, idx4, w4, rowcol, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "vis_interp_plan launch");
+}
+
+static int interp_args(const void *table, ipe_dtype dtype, int grid_side, int hidden, void *out,
+                       const VisDesc<1024> &d, InterpArgs &ia)
+{
+    if (int rc = check_dtype(dtype)) return rc;
+    if (hidden <= 0 || hidden % 4) return fail(IPE_EINVAL, "hidden %d must be a positive multiple of 4", hidden);
+    const size_t smem = interp_smem_bytes(dtype == IPE_BF16, d.merge, grid_side);
+    if (smem > 200 * 1024)
+        return fail(IPE_ELIMIT, "merge %d x grid_side %d needs %zu bytes of shared memory per block", d.merge,
+                    grid_side, smem);
+    const int eb = elem_bytes(dtype);
+    if (!aligned(table, 4 * eb) || !aligned(out, 4 * eb))
+        return fail(IPE_EALIGN, "table / out must be aligned to %d bytes", 4 * eb);
+    if (int rc = check_dev(table, (size_t)grid_side * grid_side * hidden * eb, "table")) return rc;
+    if (int rc = check_dev(out, (size_t)d.n_patch * hidden * eb, "out")) return rc;
+    const int cs = 128 / eb;
+    ia.table = table;
+    ia.out = out;
+    ia.hidden = hidden;
+    ia.n_slices = (hidden + cs - 1) / cs;
+    if ((long long)d.n_strips * ia.n_slices > (1LL << 31) - 1) return fail(IPE_ELIMIT, "grid too large");
+    return IPE_OK;
+}
+
+int ipe_vis_pos_interp(const void *table, ipe_dtype dtype, int grid_side, int hidden, const int32_t *grid_thw_host,
+                       int n_images, int merge, void *out, void *stream)
+{
+    VisDesc<1024> &d = *desc_buffer();
+    if (int rc = build_vis_desc(grid_thw_host, n_images, merge, grid_side, d)) return rc;
+    if (d.n_patch == 0) return check_dtype(dtype) ? IPE_EINVAL : ok();
+    InterpArgs ia;
+    if (int rc = interp_args(table, dtype, grid_side, hidden, out, d, ia)) return rc;
+    cudaError_t e = launch_vis_interp(dtype == IPE_BF16, d, ia, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "vis_pos_interp launch");
+}
+
+static int vis_rot_args(void *q, void *k, ipe_dtype dtype, int64_t n_patch, int heads, int head_dim,
+                        int64_t q_stride, int64_t k_stride, const VisDesc<1024> &d, RotArgs &r)
+{
+    if (int rc = check_dtype(dtype)) return rc;
+    if (n_patch != d.n_patch)
+        return fail(IPE_EINVAL, "n_patch %lld != sum t h w of grid_thw = %lld", (long long)n_patch, d.n_patch);
+    if (heads < 1) return fail(IPE_EINVAL, "heads %d must be >= 1", heads);
+    if (q == nullptr) return fail(IPE_EINVAL, "q is NULL");
+    const int hk = k ? heads : 0;
+    if (int rc = check_qk(q, k, dtype, n_patch, heads, hk, head_dim, q_stride, k ? k_stride : 0, "q", "k")) return rc;
+    r = RotArgs{};
+    r.q = q;
+    r.k = k;
+    r.rows = n_patch;
+    r.q_stride = q_stride;
+    r.k_stride = k ? k_stride : 0;
+    r.hq = heads;
+    r.hk = hk;
+    r.head_dim = head_dim;
+    r.half = head_dim / 2;
+    return IPE_OK;
+}
+
+int ipe_vis_rope2d(void *q, void *k, ipe_dtype dtype, int64_t n_patch, int heads, int head_dim, int64_t q_stride,
+                   int64_t k_stride, const int32_t *grid_thw_host, int n_images, int merge, double theta, void *stream)
+{
+    VisDesc<1024> &d = *desc_buffer();
+    if (int rc = build_vis_desc(grid_thw_host, n_images, merge, 1, d)) return rc;
+    VisAngleFreqs f;
+    if (int rc = vis_freqs(head_dim, theta, f)) return rc;
+    if (n_patch == 0 && d.n_patch == 0) return check_dtype(dtype) ? IPE_EINVAL : ok();
+    RotArgs r;
+    if (int rc = vis_rot_args(q, k, dtype, n_patch, heads, head_dim, q_stride, k_stride, d, r)) return rc;
+    cudaError_t e = launch_vis_rope(dtype == IPE_BF16, d, r, f, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "vis_rope2d launch");
+}
+
+int ipe_vis_pos_interp_rope2d(const void *table, int grid_side, int hidden, void *out, void *q, void *k, int heads,
+                              int head_dim, int64_t q_stride, int64_t k_stride, double theta, ipe_dtype dtype,
+                              const int32_t *grid_thw_host, int n_images, int merge, void *stream)
+{
+    VisDesc<1024> &d = *desc_buffer();
+    if (int rc = build_vis_desc(grid_thw_host, n_images, merge, grid_side, d)) return rc;
+    VisAngleFreqs f;
+    if (int rc = vis_freqs(head_dim, theta, f)) return rc;
+    if (d.n_patch == 0) return check_dtype(dtype) ? IPE_EINVAL : ok();
+    InterpArgs ia;
+    if (int rc = interp_args(table, dtype, grid_side, hidden, out, d, ia)) return rc;
+    RotArgs r;
+    if (int rc = vis_rot_args(q, k, dtype, d.n_patch, heads, head_dim, q_stride, k_stride, d, r)) return rc;
+    cudaError_t e = launch_vis_fused(dtype == IPE_BF16, d, ia, r, f, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "vis_pos_interp_rope2d launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+// Language-model multimodal RoPE kernels: axis map, cos / sin tables, and the
+// in-place partial rotate_half rotation (from tables, or fused with the angle
+// computation).
+//
+// "Qwen3-VL" notes (frankmowj.github.io), Qwen3VLTextRotaryEmbedding;
+// "Interleaved Rotary Position Embedding" (taking-lying-flat.github.io),
+// apply_rotary_pos_emb; "M01 RMSNorm and multimodal RoPE" (kuanzhou.online).
+#include <algorithm>
+
+#include "ipe_rotary.cuh"
+
+namespace ipe {
+
+// ------------------------------------------------------------- axis map
+__global__ void mrope_axis_map_kernel(int half, int s0, int s1, int s2, int interleaved, int8_t *axis)
+{
+    const int section[3] = {s0, s1, s2};
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < half; j += gridDim.x * blockDim.x)
+        axis[j] = (int8_t)mrope_axis(j, section, interleaved);
+}
+
+cudaError_t launch_mrope_axis_map(int half, const int *section, int interleaved, int8_t *axis,
+                                  cudaStream_t s)
+{
+    mrope_axis_map_kernel<<<1, 256, 0, s>>>(half, section[0], section[1], section[2], interleaved, axis);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------- cos / sin
+// One thread per (token, frequency); writes both halves of cat(f, f).
+__global__ void __launch_bounds__(256) mrope_cos_sin_kernel(const __grid_constant__ MropeAngles a, int half,
+                                                             float *__restrict__ cos_out,
+                                                             float *__restrict__ sin_out)
+{
+    const long long total = a.T * half;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const long long t = i / half;
+        const int j = (int)(i - t * half);
+        const int ax = mrope_axis(j, a.section, a.interleaved);
+        const int pos = __ldg(a.positions + (long long)ax * a.T + t);
+        const float angle = __fmul_rn(__int2float_rn(pos), a.inv[j]);
+        float s, c;
+        sincosf(angle, &s, &c);
+        const long long o = t * 2 * half + j;
+        cos_out[o] = c;
+        cos_out[o + half] = c;
+        sin_out[o] = s;
+        sin_out[o + half] = s;
+    }
+}
+
+cudaError_t launch_mrope_cos_sin(const MropeAngles &a, int half, float *cos_out, float *sin_out,
+                                 cudaStream_t s)
+{
+    const long long total = a.T * half;
+    const long long need = (total + 255) / 256;
+    const int blocks = (int)std::min<long long>(need, (long long)sm_count() * 8);
+    mrope_cos_sin_kernel<<<blocks, 256, 0, s>>>(a, half, cos_out, sin_out);
+    return cudaGetLastError();
+}
+
+// Widest vector (elements) that divides half, head_dim and both strides and
+// that both base pointers are aligned to.
+int pick_vec(const RotArgs &r, int elem_bytes)
+{
+    const int max_vec = 16 / elem_bytes;
+    for (int v = max_vec; v > 1; v >>= 1) {
+        const uintptr_t align = (uintptr_t)v * elem_bytes;
+        if (r.half % v || r.head_dim % v || r.q_stride % v || r.k_stride % v) continue;
+        if (r.q && ((uintptr_t)r.q % align)) continue;
+        if (r.k && ((uintptr_t)r.k % align)) continue;
+        return v;
+    }
+    return 1;
+}
+
+cudaError_t launch_rotary_mrope(bool bf16, const RotArgs &r, const MropeAngles &a, cudaStream_t s)
+{
+    MropeSrc src{a};
+    return bf16 ? dispatch_vec<__nv_bfloat16>(r, src, s) : dispatch_vec<float>(r, src, s);
+}
+
+cudaError_t launch_rotary_table(bool bf16, const RotArgs &r, const TableAngles &a, cudaStream_t s)
+{
+    TableSrc src{a};
+    return bf16 ? dispatch_vec<__nv_bfloat16>(r, src, s) : dispatch_vec<float>(r, src, s);
+}
+
+}  // namespace ipe

@@ -15,6 +15,8 @@ max(h, w) / m.  Audio is linear in time, which for positions is a text run
 
 bf16 tensors are numpy uint16 arrays of bf16 bit patterns.
 """
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -26,10 +28,11 @@ import numpy as np
 
 def f32_to_bf16_bits(x):
     """Round fp32 to bf16 (nearest, ties to even); returns uint16 bit patterns."""
-    u = np.ascontiguousarray(x, np.float32).view(np.uint32)
-    rounding = np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
-    out = ((u + rounding) >> np.uint32(16)).astype(np.uint16)
-    nan = np.isnan(np.asarray(x, np.float32))
+    x = np.ascontiguousarray(x, np.float32)
+    u = x.view(np.uint32).copy()
+    nan = np.isnan(x)
+    u += np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    out = (u >> np.uint32(16)).astype(np.uint16)
     if nan.any():
         out[nan] = np.uint16(0x7FC0)
     return out
@@ -41,33 +44,53 @@ def bf16_bits_to_f32(b):
 
 
 def rng_for(config_index, stream):
-    """Independent generator per (workload, tensor): seed = 1000 + workload index."""
+    """Generator of one (workload, tensor) pair: seed = 1000 + workload index."""
     return np.random.default_rng([1000 + int(config_index), int(stream)])
 
 
-def normal_f32(rng, shape, std=1.0, chunk=1 << 26):
-    """N(0, std^2) samples in fp32, drawn in chunks to bound peak memory."""
-    n = int(np.prod(shape))
-    out = np.empty(n, np.float32)
-    for s in range(0, n, chunk):
-        e = min(n, s + chunk)
-        out[s:e] = rng.standard_normal(e - s, dtype=np.float32)
-        if std != 1.0:
-            out[s:e] *= np.float32(std)
-    return out.reshape(shape)
+_CHUNK = 1 << 22
 
 
-def normal_bf16(rng, shape, std=1.0, chunk=1 << 26):
-    """N(0, std^2) drawn in fp32 and cast once (RNE) to bf16 bit patterns."""
-    n = int(np.prod(shape))
-    out = np.empty(n, np.uint16)
-    for s in range(0, n, chunk):
-        e = min(n, s + chunk)
-        v = rng.standard_normal(e - s, dtype=np.float32)
+def _fill_normal(key, n, std, to_bf16):
+    """N(0, std^2) samples, chunk c drawn from default_rng(key + (c,)), so the
+    values do not depend on how many threads fill them."""
+    out = np.empty(n, np.uint16 if to_bf16 else np.float32)
+
+    def work(c):
+        s, e = c * _CHUNK, min(n, (c + 1) * _CHUNK)
+        v = np.random.default_rng(list(key) + [c]).standard_normal(e - s, dtype=np.float32)
         if std != 1.0:
             v *= np.float32(std)
-        out[s:e] = f32_to_bf16_bits(v)
+        out[s:e] = f32_to_bf16_bits(v) if to_bf16 else v
+
+    nchunks = (n + _CHUNK - 1) // _CHUNK
+    if nchunks <= 1:
+        for c in range(nchunks):
+            work(c)
+    else:
+        with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+            list(ex.map(work, range(nchunks)))
+    return out
+
+
+def normal_f32(rng, shape, std=1.0):
+    """N(0, std^2) in fp32.  rng: a numpy Generator, or a seed key (tuple of ints)."""
+    n = int(np.prod(shape))
+    if isinstance(rng, tuple):
+        return _fill_normal(rng, n, std, False).reshape(shape)
+    out = rng.standard_normal(n, dtype=np.float32)
+    if std != 1.0:
+        out *= np.float32(std)
     return out.reshape(shape)
+
+
+def normal_bf16(rng, shape, std=1.0):
+    """N(0, std^2) drawn in fp32 and cast once (RNE) to bf16 bit patterns.
+    rng: a numpy Generator, or a seed key (tuple of ints)."""
+    n = int(np.prod(shape))
+    if isinstance(rng, tuple):
+        return _fill_normal(rng, n, std, True).reshape(shape)
+    return f32_to_bf16_bits(normal_f32(rng, (n,), std)).reshape(shape)
 
 
 # --------------------------------------------------------------------------
@@ -175,6 +198,11 @@ def _cfg5_segments(T=131072):
     return segs
 
 
+def key_for(config_index, stream):
+    """Seed key of one (workload, tensor) pair: (1000 + workload index, stream)."""
+    return (1000 + int(config_index), int(stream))
+
+
 def _vision_batch8_grids():
     rng = rng_for(4, 5)
     pick = rng.integers(0, len(VISION_GRID_CHOICES), size=8)
@@ -206,7 +234,7 @@ WORKLOADS = {
                       segments=_cfg5_segments())),
 }
 
-# Streams of rng_for(index, stream)
+# Streams of key_for(index, stream)
 S_TABLE, S_QV, S_KV, S_Q, S_K, S_GRID = 0, 1, 2, 3, 4, 5
 
 
@@ -223,9 +251,9 @@ def vision_inputs(w):
     N = n_patches(v)
     gen = normal_f32 if v.dtype == "f32" else normal_bf16
     return {
-        "table": gen(rng_for(w.index, S_TABLE), (v.grid_side * v.grid_side, v.hidden), v.table_std),
-        "q": gen(rng_for(w.index, S_QV), (N, v.heads, v.head_dim)),
-        "k": gen(rng_for(w.index, S_KV), (N, v.heads, v.head_dim)),
+        "table": gen(key_for(w.index, S_TABLE), (v.grid_side * v.grid_side, v.hidden), v.table_std),
+        "q": gen(key_for(w.index, S_QV), (N, v.heads, v.head_dim)),
+        "k": gen(key_for(w.index, S_KV), (N, v.heads, v.head_dim)),
         "grid_thw": np.asarray(v.grid_thw, np.int32).reshape(-1, 3),
     }
 
@@ -237,6 +265,6 @@ def text_inputs(w, with_qk=True):
     assert pos.shape[1] == t.T, (pos.shape, t.T)
     out = {"positions": pos}
     if with_qk:
-        out["q"] = normal_bf16(rng_for(w.index, S_Q), (t.T, t.hq, t.head_dim))
-        out["k"] = normal_bf16(rng_for(w.index, S_K), (t.T, t.hk, t.head_dim))
+        out["q"] = normal_bf16(key_for(w.index, S_Q), (t.T, t.hq, t.head_dim))
+        out["k"] = normal_bf16(key_for(w.index, S_K), (t.T, t.hk, t.head_dim))
     return out
