@@ -7,7 +7,7 @@ C entry point of the same name (``include/ipe.h``) and raises
 the computation runs in the library's CUDA kernels; there is no other path.
 PyTorch is used for device memory and streams only.
 
-Build the library first: ``python -m interpolated_position_encoding_b200.build``.
+Build the library first: ``python interpolated_position_encoding_b200/build.py``.
 """
 import ctypes
 import os
@@ -20,7 +20,7 @@ _LIB_PATH = _build.LIB
 
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
-        f"{_LIB_PATH} is missing: build it with `python -m interpolated_position_encoding_b200.build` "
+        f"{_LIB_PATH} is missing: build it with `python interpolated_position_encoding_b200/build.py` "
         "(nvcc for sm_100a); there is no fallback implementation")
 
 _lib = ctypes.CDLL(_LIB_PATH)

@@ -1,6 +1,6 @@
 """Build ``libipe.so`` in-tree with nvcc for sm_100a.
 
-    python -m interpolated_position_encoding_b200.build [--force] [--verbose]
+    python interpolated_position_encoding_b200/build.py [--force] [--verbose]
 
 Each ``csrc/*.cu`` compiles to an object in ``_build/`` (in parallel), then
 one link produces ``interpolated_position_encoding_b200/libipe.so`` with the

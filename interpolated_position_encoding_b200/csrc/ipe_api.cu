@@ -138,8 +138,8 @@ int check_qk(void *q, void *k, ipe_dtype dt, long long rows, int hq, int hk, int
         return fail(IPE_EINVAL, "%s row stride %lld < heads * head_dim = %lld", qn, qs, (long long)hq * head_dim);
     if (hk > 0 && ks < (long long)hk * head_dim)
         return fail(IPE_EINVAL, "%s row stride %lld < heads * head_dim = %lld", kn, ks, (long long)hk * head_dim);
-    if (hq > 0 && q == nullptr) return fail(IPE_EINVAL, "%s is NULL but has %d heads", qn, hq);
-    if (hk > 0 && k == nullptr) return fail(IPE_EINVAL, "%s is NULL but has %d heads", kn, hk);
+    if (rows > 0 && hq > 0 && q == nullptr) return fail(IPE_EINVAL, "%s is NULL but has %d heads", qn, hq);
+    if (rows > 0 && hk > 0 && k == nullptr) return fail(IPE_EINVAL, "%s is NULL but has %d heads", kn, hk);
     const int eb = elem_bytes(dt);
     if (!aligned(q, eb) || !aligned(k, eb)) return fail(IPE_EALIGN, "%s / %s not aligned to the element size", qn, kn);
     if (hq > 0) {
