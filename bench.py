@@ -353,6 +353,7 @@ def main():
     h1 = time.time()
     ms_step = start.elapsed_time(end) / args.steps
     ms_step = max_over_ranks(ms_step)
+    ipe.device_status(stream)          # raises if any kernel gave up a bounded wait
     kernel_ms = {n: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j, n in enumerate(names)}
     clocks = sampler.stop(h0, h1)
 

@@ -56,7 +56,8 @@ typedef enum {
     IPE_EINVAL = 1,  /* a size, count or pointer the operation does not accept  */
     IPE_EALIGN = 2,  /* a pointer or stride breaks the vector alignment        */
     IPE_ELIMIT = 3,  /* above a documented library limit (images, dims, T)     */
-    IPE_ECUDA = 4    /* a CUDA runtime call or the launch failed               */
+    IPE_ECUDA = 4,   /* a CUDA runtime call or the launch failed               */
+    IPE_EDEVICE = 5  /* a kernel gave up a bounded wait (ipe_device_status)    */
 } ipe_status;
 
 /* Library limits (IPE_ELIMIT above them). */
@@ -69,6 +70,27 @@ const char *ipe_last_error(void);
 
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
 int ipe_version(void);
+
+/* ---------------------------------------------------------------------------
+ * ipe_device_status -- failure report of the kernels that ran on the current
+ * device.  The TMA-fed rotation kernels wait on shared-memory barriers; every
+ * such wait gives up after a time limit (about one second), records a fault
+ * code in a device status word and lets the kernel return instead of spinning.
+ * This call synchronises `stream`, reads and clears that word, and returns
+ * IPE_OK, or IPE_EDEVICE with a message naming the wait that gave up (the
+ * results of the failed launch are then incomplete).  Not part of any page:
+ * failure reporting of this library.
+ * ------------------------------------------------------------------------- */
+int ipe_device_status(void *stream);
+
+/* ---------------------------------------------------------------------------
+ * ipe_debug_inject -- test hook for the failure path above.  From the next
+ * launch on, the producer of the TMA rotation kernels skips the loads of tile
+ * `skip_tile` (-1: none), so the consumers waiting for it give up after
+ * `wait_cycles` SM clock cycles (0: the default limit).  Host state, not
+ * thread-safe; reset with ipe_debug_inject(-1, 0).
+ * ------------------------------------------------------------------------- */
+int ipe_debug_inject(int64_t skip_tile, int64_t wait_cycles);
 
 /* ---------------------------------------------------------------------------
  * ipe_rope_inv_freq -- default RoPE inverse frequencies, on the host.

@@ -30,6 +30,8 @@ _P, _I, _I64, _D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_doubl
 _SIGS = {
     "ipe_last_error": (ctypes.c_char_p, []),
     "ipe_version": (_I, []),
+    "ipe_device_status": (_I, [_P]),
+    "ipe_debug_inject": (_I, [_I64, _I64]),
     "ipe_rope_inv_freq": (_I, [_I, _D, _P]),
     "ipe_mrope_axis_map": (_I, [_I, _P, _I, _P, _P]),
     "ipe_mrope_cos_sin": (_I, [_P, _I64, _P, _I, _P, _I, _P, _P, _P]),
@@ -48,8 +50,8 @@ for _name, (_res, _args) in _SIGS.items():
 EXPORTS = tuple(_SIGS)
 
 IPE_F32, IPE_BF16 = 0, 1
-IPE_OK, IPE_EINVAL, IPE_EALIGN, IPE_ELIMIT, IPE_ECUDA = 0, 1, 2, 3, 4
-_STATUS = {1: "IPE_EINVAL", 2: "IPE_EALIGN", 3: "IPE_ELIMIT", 4: "IPE_ECUDA"}
+IPE_OK, IPE_EINVAL, IPE_EALIGN, IPE_ELIMIT, IPE_ECUDA, IPE_EDEVICE = 0, 1, 2, 3, 4, 5
+_STATUS = {1: "IPE_EINVAL", 2: "IPE_EALIGN", 3: "IPE_ELIMIT", 4: "IPE_ECUDA", 5: "IPE_EDEVICE"}
 
 
 class IpeError(RuntimeError):
@@ -117,6 +119,16 @@ def _row_stride(t, heads, head_dim, name):
     if t.stride(2) != 1 or (heads > 1 and t.stride(1) != head_dim):
         raise ValueError(f"{name}: heads must be contiguous (strides {t.stride()})")
     return t.stride(0)
+
+
+def device_status(stream=None):
+    """Synchronise the stream and raise IpeError(IPE_EDEVICE) if a kernel gave up a bounded wait."""
+    _check(_lib.ipe_device_status(_stream(stream)))
+
+
+def debug_inject(skip_tile=-1, wait_cycles=0):
+    """Test hook: TMA rotation producers skip tile `skip_tile`; waits give up after `wait_cycles`."""
+    _check(_lib.ipe_debug_inject(int(skip_tile), int(wait_cycles)))
 
 
 # --------------------------------------------------------------------- text
@@ -281,5 +293,5 @@ def vis_pos_interp_rope2d(table, grid_thw, q, k, merge=2, theta=1e4, out=None, s
     return out, q, k
 
 
-__all__ = ["IpeError", "lib", "EXPORTS", "rope_inv_freq", "mrope_axis_map", "mrope_cos_sin", "apply_rotary_partial",
+__all__ = ["IpeError", "lib", "EXPORTS", "device_status", "debug_inject", "rope_inv_freq", "mrope_axis_map", "mrope_cos_sin", "apply_rotary_partial",
            "mrope_apply", "vis_interp_plan", "vis_pos_interp", "vis_rope2d", "vis_pos_interp_rope2d"]

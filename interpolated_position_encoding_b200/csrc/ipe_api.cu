@@ -11,6 +11,7 @@
 
 #include "../../include/ipe.h"
 #include "ipe_internal.h"
+#include "ipe_rotary_tma.cuh"
 
 using namespace ipe;
 
@@ -93,6 +94,34 @@ int check_dev(const void *p, size_t bytes, const char *name)
 }
 
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// ------------------------------------------------- status word, test hooks
+__device__ unsigned g_ipe_status;     // first fault code of any kernel since the last read
+
+long long g_skip_tile = -1;
+long long g_wait_limit = 0;           // 0: default
+constexpr long long kDefaultWaitCycles = 1LL << 31;   // about 1.1 s at 1.9 GHz
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
 
 int elem_bytes(ipe_dtype dt) { return dt == IPE_BF16 ? 2 : 4; }
 
@@ -212,11 +241,118 @@ VisDesc<1024> *desc_buffer()
 
 }  // namespace
 
+namespace ipe {
+
+unsigned *device_status_word()
+{
+    static unsigned *addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_ipe_status) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = static_cast<unsigned *>(p);
+    }
+    return addr[dev];
+}
+
+long long debug_skip_tile() { return g_skip_tile; }
+long long debug_wait_limit() { return g_wait_limit > 0 ? g_wait_limit : kDefaultWaitCycles; }
+
+bool encode_tmap(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
+                 const uint64_t *strides, const uint32_t *box)
+{
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn || rank < 1 || rank > 3 || !aligned(base, 16)) return false;
+    cuuint64_t gdim[3], gstr[2];
+    cuuint32_t bdim[3], estr[3] = {1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        if (dims[i] == 0 || dims[i] > (1ULL << 32) || box[i] == 0 || box[i] > 256) return false;
+        gdim[i] = dims[i];
+        bdim[i] = box[i];
+    }
+    for (int i = 0; i + 1 < rank; ++i) {
+        if (strides[i] % 16 || strides[i] >= (1ULL << 40)) return false;
+        gstr[i] = strides[i];
+    }
+    return fn(map, dt, (cuuint32_t)rank, const_cast<void *>(base), gdim, gstr, bdim, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tma_rot_args(const RotArgs &r, int eb, TmaRotArgs &t)
+{
+    const int rot = 2 * r.half;
+    if ((rot * eb) % 16 || rot > 256 || (r.head_dim * eb) % 16) return false;
+    if (r.hq > 256 || r.hk > 256 || r.rows <= 0 || r.rows > 0x7fffffffLL) return false;
+    // one stage (P rows of q and k) must stay far below the shared memory and
+    // the 2^20-byte transaction count of a barrier phase
+    if ((size_t)kTmaRows * (r.hq + r.hk) * rot * eb > 64 * 1024) return false;
+    const CUtensorMapDataType dt = eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    t = TmaRotArgs{};
+    t.P = kTmaRows;
+    struct Side {
+        CUtensorMap *tile, *one;
+        void *ptr;
+        int heads;
+        long long stride;
+    } sides[2] = {{&t.tq, &t.tq1, r.q, r.hq, r.q_stride}, {&t.tk, &t.tk1, r.k, r.hk, r.k_stride}};
+    for (const Side &sd : sides) {
+        if (!sd.heads) continue;
+        const uint64_t dims[3] = {(uint64_t)r.head_dim, (uint64_t)sd.heads, (uint64_t)r.rows};
+        const uint64_t str[2] = {(uint64_t)r.head_dim * eb, (uint64_t)sd.stride * eb};
+        const uint32_t box_tile[3] = {(uint32_t)rot, (uint32_t)sd.heads, (uint32_t)t.P};
+        const uint32_t box_one[3] = {(uint32_t)rot, (uint32_t)sd.heads, 1};
+        if (!encode_tmap(sd.tile, dt, 3, sd.ptr, dims, str, box_tile)) return false;
+        if (!encode_tmap(sd.one, dt, 3, sd.ptr, dims, str, box_one)) return false;
+    }
+    t.rows = r.rows;
+    t.hq = r.hq;
+    t.hk = r.hk;
+    t.half = r.half;
+    t.wait_limit = debug_wait_limit();
+    t.skip_tile = debug_skip_tile();
+    t.status = device_status_word();
+    return t.status != nullptr;
+}
+
+}  // namespace ipe
+
 extern "C" {
 
 const char *ipe_last_error(void) { return g_err.c_str(); }
 
 int ipe_version(void) { return 100; }
+
+int ipe_device_status(void *stream)
+{
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned v = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, g_ipe_status, sizeof v)) != cudaSuccess) return cuda_fail(e, "status read");
+    if (v == 0) return ok();
+    const unsigned zero = 0;
+    if ((e = cudaMemcpyToSymbol(g_ipe_status, &zero, sizeof zero)) != cudaSuccess) return cuda_fail(e, "status clear");
+    const char *what = v == 1 ? "a consumer warp gave up waiting for a stage's data"
+                     : v == 2 ? "the producer gave up waiting for a free stage"
+                     : v == 3 ? "loads in flight did not land while a block shut down"
+                              : "unknown";
+    return fail(IPE_EDEVICE, "device fault %u: %s", v, what);
+}
+
+int ipe_debug_inject(int64_t skip_tile, int64_t wait_cycles)
+{
+    if (wait_cycles < 0) return fail(IPE_EINVAL, "wait_cycles %lld is negative", (long long)wait_cycles);
+    g_skip_tile = skip_tile < 0 ? -1 : skip_tile;
+    g_wait_limit = wait_cycles;
+    return ok();
+}
 
 int ipe_rope_inv_freq(int rot_dim, double theta, float *inv_freq_host)
 {

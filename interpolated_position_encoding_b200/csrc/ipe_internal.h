@@ -5,6 +5,7 @@
 
 #include <cstdint>
 
+#include <cuda.h>            // CUtensorMap (types only; the encoder is resolved at run time)
 #include <cuda_runtime.h>
 
 namespace ipe {
@@ -70,6 +71,47 @@ struct VisAngleFreqs {             // vision 2-D angles: row * inv[i], col * inv
     int nf;                        // frequencies per axis (= head_dim / 4)
     float inv[kMaxVisFreq];
 };
+
+// ------------------------------------------------------- TMA rotation path
+// In-place rotation fed by tiled TMA loads and drained by TMA stores (see
+// ipe_rotary_tma.cuh).  Each tile is P rows, one per consumer warp.  A stage
+// holds P q-row slots and P k-row slots (each 128-byte aligned, the rotary
+// slice of every head of one row), then the aux boxes.
+struct TmaRotArgs {
+    CUtensorMap tq, tk;      // [rows, heads, head_dim] -> box {rot, heads, P}  (whole-tile loads)
+    CUtensorMap tq1, tk1;    // same tensors, box {rot, heads, 1}             (per-row loads, stores)
+    CUtensorMap taux0;       // positions [3, T] -> box {P, 3}, or cos [T, rot] -> box {rot, P}
+    CUtensorMap taux1;       // sin [T, rot] -> box {rot, P}
+    long long rows;
+    int hq, hk, half;
+    int P;                   // rows per tile = consumer warps
+    int stages;
+    int aux_tma;             // 1 when taux0 (and taux1) are loaded by TMA
+    int dense_q, dense_k;    // 1: one box per tile (slot = row bytes, a multiple of 128)
+    int lane_rows;           // 1: lane i rotates head row i (<= 32 rows); 0: lanes sweep chunks
+    int swap_shift;          // lanes with bit `swap_shift` set read the second half first
+    unsigned slot_q, slot_k; // bytes of one row slot
+    unsigned stage_bytes, off_k, off_aux0, off_aux1;
+    unsigned row_bytes_q, row_bytes_k, aux_bytes;
+    long long wait_limit;    // SM cycles before a barrier wait gives up
+    long long skip_tile;     // test hook: the producer never loads this tile (-1: none)
+    unsigned *status;        // fault word (ipe_device_status)
+};
+
+// Test hooks and the device status word (ipe_api.cu).
+unsigned *device_status_word();
+long long debug_skip_tile();
+long long debug_wait_limit();
+
+// TMA rotation arguments for the q / k of `r` (tensor maps, strides, test
+// hooks, status word).  False when the shapes, strides or alignment do not
+// allow tiled TMA (the caller then uses the vector-load path).
+bool tma_rot_args(const RotArgs &r, int elem_bytes, TmaRotArgs &t);
+
+// Tiled tensor map over `base` (rank <= 3, dims inner first, strides in bytes
+// for dims 1..rank-1).  False if the driver rejects it.
+bool encode_tmap(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
+                 const uint64_t *strides, const uint32_t *box);
 
 // Launchers (return cudaGetLastError() of the launch).
 cudaError_t launch_mrope_cos_sin(const MropeAngles &a, int half, float *cos_out, float *sin_out,

@@ -7,7 +7,7 @@
 // apply_rotary_pos_emb; "M01 RMSNorm and multimodal RoPE" (kuanzhou.online).
 #include <algorithm>
 
-#include "ipe_rotary.cuh"
+#include "ipe_rotary_tma.cuh"
 
 namespace ipe {
 
@@ -75,14 +75,49 @@ int pick_vec(const RotArgs &r, int elem_bytes)
     return 1;
 }
 
+// VEC >= 2 always holds on the TMA path (16-byte rotary rows and strides).
+template <typename T, class Src>
+static cudaError_t dispatch_tma(const TmaRotArgs &t, const RotArgs &r, const Src &src, cudaStream_t s)
+{
+    const int v = pick_vec(r, sizeof(T));
+    if constexpr (sizeof(T) == 2) {
+        if (v == 8) return launch_rotary_tma_vec<T, 8, Src>(t, src, s);
+    }
+    if (v >= 4) return launch_rotary_tma_vec<T, 4, Src>(t, src, s);
+    return launch_rotary_tma_vec<T, 2, Src>(t, src, s);
+}
+
 cudaError_t launch_rotary_mrope(bool bf16, const RotArgs &r, const MropeAngles &a, cudaStream_t s)
 {
+    TmaRotArgs t;
+    if (tma_rot_args(r, bf16 ? 2 : 4, t)) {
+        // positions [3, T] as a {T, 3} tensor: rows must be 16-byte multiples
+        const uint64_t dims[2] = {(uint64_t)a.T, 3};
+        const uint64_t str[1] = {(uint64_t)a.T * 4};
+        const uint32_t box[2] = {(uint32_t)t.P, 3};
+        t.aux_tma = a.T % 4 == 0 && encode_tmap(&t.taux0, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, a.positions, dims, str, box);
+        t.aux_bytes = (unsigned)t.P * 3 * 4;
+        MropeTmaSrc src{a};
+        return bf16 ? dispatch_tma<__nv_bfloat16>(t, r, src, s) : dispatch_tma<float>(t, r, src, s);
+    }
     MropeSrc src{a};
     return bf16 ? dispatch_vec<__nv_bfloat16>(r, src, s) : dispatch_vec<float>(r, src, s);
 }
 
 cudaError_t launch_rotary_table(bool bf16, const RotArgs &r, const TableAngles &a, cudaStream_t s)
 {
+    TmaRotArgs t;
+    if (tma_rot_args(r, bf16 ? 2 : 4, t)) {
+        const int rot = 2 * r.half;
+        const uint64_t dims[2] = {(uint64_t)rot, (uint64_t)r.rows};
+        const uint64_t str[1] = {(uint64_t)rot * 4};
+        const uint32_t box[2] = {(uint32_t)rot, (uint32_t)t.P};
+        t.aux_tma = encode_tmap(&t.taux0, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a.cos, dims, str, box) &&
+                    encode_tmap(&t.taux1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a.sin, dims, str, box);
+        t.aux_bytes = 2u * t.P * rot * 4;
+        TableTmaSrc src{a};
+        return bf16 ? dispatch_tma<__nv_bfloat16>(t, r, src, s) : dispatch_tma<float>(t, r, src, s);
+    }
     TableSrc src{a};
     return bf16 ? dispatch_vec<__nv_bfloat16>(r, src, s) : dispatch_vec<float>(r, src, s);
 }

@@ -1,0 +1,452 @@
+// TMA-fed in-place rotation (sm_100a).
+//
+// Warp 0 is the producer: one lane streams tiles of P rows (tokens or
+// patches) from HBM into a ring of shared-memory stages with tiled TMA loads
+// (cp.async.bulk.tensor over [rows, heads, head_dim] with boxes of
+// {rot, heads, *}, so only the rotary slice of each head row moves), keeping
+// up to `stages` tiles in flight.  Warps 1..P are consumers, one row of the
+// tile each: the warp computes the row's (cos, sin) once into its own
+// shared-memory slot (one sincosf per frequency, shared by every head of q and
+// k), rotates the row's head rows in place in shared memory, and a TMA store
+// writes the row back; once the store has read the slot the warp frees the
+// stage.  No block-wide barrier runs inside the loop.
+//
+// Every wait is bounded (TmaRotArgs::wait_limit cycles): a warp that gives up
+// records a fault in the status word and raises a shared abort flag, the
+// others leave their loops, and the producer waits (bounded) for the loads it
+// still has in flight before the block exits.
+#pragma once
+
+#include "ipe_rotary.cuh"
+#include "ipe_tma.cuh"
+
+namespace ipe {
+
+constexpr int kTmaConsumers = 8;
+constexpr int kTmaRows = kTmaConsumers;             // rows per tile: one per consumer warp
+constexpr int kTmaThreads = 32 * (1 + kTmaConsumers);
+constexpr int kTmaMaxStages = 8;
+constexpr size_t kTmaBlockSmem = 112 * 1024;        // two blocks per SM
+
+__host__ __device__ inline unsigned align128(unsigned v) { return (v + 127u) & ~127u; }
+
+// (cos, sin) slot of one consumer warp, in floats: cos [half], sin [half],
+// -sin [half] (4 floats further, so sin and -sin chunks fall in different
+// banks) and, for tables whose halves may differ, cos_hi [half], sin_hi [half].
+struct CsSlot {
+    float *c, *s, *ns, *ch, *sh;
+};
+
+__host__ __device__ inline size_t tma_cs_floats(int half, bool hi) { return (size_t)half * (hi ? 5 : 3) + (hi ? 8 : 4); }
+
+// Packed fp32 pairs (sm_100a): two independent correctly rounded operations.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// VEC elements <-> VEC/2 fp32 pairs (element 2i in .x, 2i+1 in .y).
+template <typename T, int VEC>
+__device__ __forceinline__ void load_pairs(const T *p, float2 *v)
+{
+    if constexpr (sizeof(T) == 2) {
+        const Pack<uint32_t, VEC / 2> w = ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(p));
+#pragma unroll
+        for (int i = 0; i < VEC / 2; ++i)
+            v[i] = make_float2(__uint_as_float(w.v[i] << 16), __uint_as_float(w.v[i] & 0xffff0000u));
+    } else {
+        const Pack<float2, VEC / 2> f = ld_pack<float2, VEC / 2>(reinterpret_cast<const float2 *>(p));
+#pragma unroll
+        for (int i = 0; i < VEC / 2; ++i) v[i] = f.v[i];
+    }
+}
+
+template <typename T, int VEC>
+__device__ __forceinline__ void store_pairs(T *p, const float2 *v)
+{
+    if constexpr (sizeof(T) == 2) {
+        Pack<uint32_t, VEC / 2> w;
+#pragma unroll
+        for (int i = 0; i < VEC / 2; ++i) {
+            const __nv_bfloat162 b = __floats2bfloat162_rn(v[i].x, v[i].y);   // one rounding each
+            w.v[i] = *reinterpret_cast<const uint32_t *>(&b);
+        }
+        st_pack<uint32_t, VEC / 2>(reinterpret_cast<uint32_t *>(p), w);
+    } else {
+        Pack<float2, VEC / 2> f;
+#pragma unroll
+        for (int i = 0; i < VEC / 2; ++i) f.v[i] = v[i];
+        st_pack<float2, VEC / 2>(reinterpret_cast<float2 *>(p), f);
+    }
+}
+
+template <int VEC>
+__device__ __forceinline__ void load_coef(const float *p, float2 *v)
+{
+    const Pack<float2, VEC / 2> f = ld_pack<float2, VEC / 2>(reinterpret_cast<const float2 *>(p));
+#pragma unroll
+    for (int i = 0; i < VEC / 2; ++i) v[i] = f.v[i];
+}
+
+// ------------------------------------------------------------ angle sources
+// angles(): (cos, sin) of every frequency of tile row c (global row `row`)
+// into the warp's slot.  issue_aux(): TMA loads of per-tile side data.
+
+struct MropeTmaSrc {
+    static constexpr bool kHi = false;
+    MropeAngles a;
+    __device__ __forceinline__ void issue_aux(const TmaRotArgs &r, uint32_t stage, int r0, uint32_t bar) const
+    {
+        tma_load_2d(stage + r.off_aux0, &r.taux0, r0, 0, bar);      // positions [3, P]
+    }
+    __device__ __forceinline__ void angles(const TmaRotArgs &r, const unsigned char *stage, int c, long long row,
+                                           int lane, const CsSlot &cs) const
+    {
+        const int32_t *spos = reinterpret_cast<const int32_t *>(stage + r.off_aux0);
+        for (int j = lane; j < r.half; j += 32) {
+            const int ax = mrope_axis(j, a.section, a.interleaved);
+            const int pos = r.aux_tma ? spos[ax * r.P + c] : __ldg(a.positions + (long long)ax * a.T + row);
+            // fl32(fl32(pos) * inv_freq[j]): one rounded product, no contraction
+            const float angle = __fmul_rn(__int2float_rn(pos), a.inv[j]);
+            float sn, cn;
+            sincosf(angle, &sn, &cn);
+            cs.c[j] = cn;
+            cs.s[j] = sn;
+            cs.ns[j] = -sn;
+        }
+    }
+};
+
+struct TableTmaSrc {
+    static constexpr bool kHi = true;
+    TableAngles a;
+    __device__ __forceinline__ void issue_aux(const TmaRotArgs &r, uint32_t stage, int r0, uint32_t bar) const
+    {
+        tma_load_2d(stage + r.off_aux0, &r.taux0, 0, r0, bar);      // cos [P, rot]
+        tma_load_2d(stage + r.off_aux1, &r.taux1, 0, r0, bar);      // sin [P, rot]
+    }
+    __device__ __forceinline__ void angles(const TmaRotArgs &r, const unsigned char *stage, int c, long long row,
+                                           int lane, const CsSlot &cs) const
+    {
+        const int half = r.half, rot = 2 * half;
+        const float *sc = r.aux_tma ? reinterpret_cast<const float *>(stage + r.off_aux0) + (size_t)c * rot
+                                    : a.cos + row * rot;
+        const float *ss = r.aux_tma ? reinterpret_cast<const float *>(stage + r.off_aux1) + (size_t)c * rot
+                                    : a.sin + row * rot;
+        for (int j = lane; j < half; j += 32) {
+            cs.c[j] = sc[j];
+            cs.s[j] = ss[j];
+            cs.ns[j] = -ss[j];
+            cs.ch[j] = sc[j + half];
+            cs.sh[j] = ss[j + half];
+        }
+    }
+};
+
+template <int MAXIMG>
+struct VisTmaSrc {
+    static constexpr bool kHi = false;
+    VisDesc<MAXIMG> d;
+    VisAngleFreqs f;
+    __device__ __forceinline__ void issue_aux(const TmaRotArgs &, uint32_t, int, uint32_t) const {}
+    __device__ __forceinline__ void angles(const TmaRotArgs &r, const unsigned char *, int, long long row, int lane,
+                                           const CsSlot &cs) const
+    {
+        int prow, pcol;
+        patch_row_col(d, row, prow, pcol);
+        const int nf = f.nf;
+        for (int j = lane; j < r.half; j += 32) {
+            // angles [row * inv (nf) | col * inv (nf)]
+            const int v = j < nf ? prow : pcol;
+            const float angle = __fmul_rn(__int2float_rn(v), f.inv[j < nf ? j : j - nf]);
+            float sn, cn;
+            sincosf(angle, &sn, &cn);
+            cs.c[j] = cn;
+            cs.s[j] = sn;
+            cs.ns[j] = -sn;
+        }
+    }
+};
+
+// One chunk: elements [u VEC, u VEC + VEC) of the first half of head row `p`
+// and the matching chunk of the second half, rotated in place.  With `swap`
+// the lane reads (and writes) the second half first, which spreads
+// neighbouring rows over the banks; the formula is the same either way:
+//   x'[j]     = x[j] cos_j         - x[j+h] sin_j
+//   x'[j + h] = x[j + h] cos_{j+h} + x[j] sin_{j+h}
+// written as  w1 = v1 C1 + v2 S1,  w2 = v2 C2 + v1 S2  on the values v1, v2
+// at the first and second address, with C / S chosen (not computed) per lane.
+template <typename T, int VEC, bool HI>
+__device__ __forceinline__ void rotate_chunk(T *p, int half, int u, bool swap, const CsSlot &cs)
+{
+    static_assert(VEC >= 2, "pairs");
+    T *pa = p + u * VEC, *pb = pa + half;
+    T *p1 = swap ? pb : pa, *p2 = swap ? pa : pb;
+    const int o = u * VEC;
+    const float *C1 = HI ? (swap ? cs.ch : cs.c) + o : cs.c + o;
+    const float *C2 = HI ? (swap ? cs.c : cs.ch) + o : cs.c + o;
+    const float *S1 = (swap ? (HI ? cs.sh : cs.s) : cs.ns) + o;
+    const float *S2 = (swap ? cs.ns : (HI ? cs.sh : cs.s)) + o;
+    float2 v1[VEC / 2], v2[VEC / 2], c1[VEC / 2], c2[VEC / 2], s1[VEC / 2], s2[VEC / 2], w1[VEC / 2], w2[VEC / 2];
+    load_pairs<T, VEC>(p1, v1);
+    load_pairs<T, VEC>(p2, v2);
+    load_coef<VEC>(C1, c1);
+    load_coef<VEC>(S1, s1);
+    load_coef<VEC>(S2, s2);
+    if constexpr (HI) load_coef<VEC>(C2, c2);
+#pragma unroll
+    for (int i = 0; i < VEC / 2; ++i) {
+        w1[i] = fma2(v1[i], c1[i], mul2(v2[i], s1[i]));
+        w2[i] = fma2(v2[i], HI ? c2[i] : c1[i], mul2(v1[i], s2[i]));
+    }
+    store_pairs<T, VEC>(p1, w1);
+    store_pairs<T, VEC>(p2, w2);
+}
+
+// Rotate the head rows of one tile row (q slot then k slot) in shared memory.
+template <typename T, int VEC, bool HI>
+__device__ __forceinline__ void rotate_slots(const TmaRotArgs &a, unsigned char *sq, unsigned char *sk, int lane,
+                                             const CsSlot &cs)
+{
+    const int half = a.half, rot = 2 * half, nvec = half / VEC, H = a.hq + a.hk;
+    T *q = reinterpret_cast<T *>(sq);
+    T *k = reinterpret_cast<T *>(sk);
+    if (a.lane_rows) {
+        // lane i owns head row i; all lanes read the same (cos, sin) chunk
+        if (lane < H) {
+            T *p = lane < a.hq ? q + lane * rot : k + (lane - a.hq) * rot;
+            const bool swap = (lane >> a.swap_shift) & 1;
+            for (int u = 0; u < nvec; ++u) rotate_chunk<T, VEC, HI>(p, half, u, swap, cs);
+        }
+    } else {
+        // lanes sweep (head, chunk) with the chunk fastest; odd heads swap
+        int h = lane / nvec, u = lane - h * nvec;
+        const int dh = 32 / nvec, du = 32 - dh * nvec;
+        while (h < H) {
+            T *p = h < a.hq ? q + h * rot : k + (h - a.hq) * rot;
+            rotate_chunk<T, VEC, HI>(p, half, u, h & 1, cs);
+            u += du;
+            h += dh;
+            if (u >= nvec) {
+                u -= nvec;
+                ++h;
+            }
+        }
+    }
+}
+
+// Shared memory of one block: 128 B alignment slack, the stages, 2 barriers
+// per stage, the abort flag (16 B) and the consumers' (cos, sin) slots.
+__host__ __device__ inline size_t tma_smem_bytes(const TmaRotArgs &a, bool hi)
+{
+    const size_t cs = (tma_cs_floats(a.half, hi) * sizeof(float) + 15) & ~size_t(15);
+    return 128 + (size_t)a.stages * a.stage_bytes + 16 * (size_t)a.stages + 16 + (size_t)kTmaConsumers * cs;
+}
+
+template <typename T, int VEC, class Src>
+__global__ void __launch_bounds__(kTmaThreads) rotary_tma_kernel(const __grid_constant__ TmaRotArgs a,
+                                                                 const __grid_constant__ Src src)
+{
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
+    const int S = a.stages;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)S * a.stage_bytes);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 2 * S);
+    float *slots = reinterpret_cast<float *>(bars + 2 * S + 2);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(smem_addr(&bars[s]), 1);                    // full: the producer's expect_tx
+            mbar_init(smem_addr(&bars[S + s]), kTmaConsumers);    // empty: one arrival per consumer warp
+        }
+        *abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const long long ntiles = (a.rows + a.P - 1) / a.P;
+
+    if (warp == 0) {
+        if (lane != 0) return;
+        // ------------------------------------------------------- producer
+        if (a.hq) prefetch_tmap(a.dense_q ? &a.tq : &a.tq1);
+        if (a.hk) prefetch_tmap(a.dense_k ? &a.tk : &a.tk1);
+        long long last_round[kTmaMaxStages];
+        for (int s = 0; s < kTmaMaxStages; ++s) last_round[s] = -1;
+        bool aborted = false;
+        long long it = 0;
+        for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+            const int s = (int)(it % S);
+            const long long round = it / S;
+            if (!mbar_wait(smem_addr(&bars[S + s]), (uint32_t)((round & 1) ^ 1), a.wait_limit, abort)) {
+                if (!*abort) record_fault(a.status, kFaultEmptyWait);
+                *abort = 1;
+                aborted = true;
+                break;
+            }
+            if (tile == a.skip_tile) continue;    // test hook: this stage never fills
+            const uint32_t full = smem_addr(&bars[s]);
+            const uint32_t st = smem_addr(smem + (size_t)s * a.stage_bytes);
+            const int r0 = (int)(tile * a.P);
+            const int valid = (int)min((long long)a.P, a.rows - r0);
+            // a whole-tile box counts all P rows (rows past the end are
+            // zero-filled); per-row boxes are issued for valid rows only
+            const unsigned tx = (a.dense_q ? a.P : valid) * a.row_bytes_q + (a.dense_k ? a.P : valid) * a.row_bytes_k +
+                                (a.aux_tma ? a.aux_bytes : 0u);
+            mbar_arrive_expect_tx(full, tx);
+            if (a.hq) {
+                if (a.dense_q) tma_load_3d(st, &a.tq, 0, 0, r0, full);
+                else
+                    for (int p = 0; p < valid; ++p) tma_load_3d(st + p * a.slot_q, &a.tq1, 0, 0, r0 + p, full);
+            }
+            if (a.hk) {
+                if (a.dense_k) tma_load_3d(st + a.off_k, &a.tk, 0, 0, r0, full);
+                else
+                    for (int p = 0; p < valid; ++p)
+                        tma_load_3d(st + a.off_k + p * a.slot_k, &a.tk1, 0, 0, r0 + p, full);
+            }
+            if (a.aux_tma) src.issue_aux(a, st, r0, full);
+            last_round[s] = round;
+        }
+        if (aborted || *abort) {
+            // loads still in flight must land before the block releases its memory
+            for (int s = 0; s < S; ++s)
+                if (last_round[s] >= 0 &&
+                    !mbar_wait(smem_addr(&bars[s]), (uint32_t)(last_round[s] & 1), a.wait_limit, nullptr))
+                    record_fault(a.status, kFaultDrainWait);
+        }
+        return;
+    }
+
+    // ----------------------------------------------------------- consumers
+    const int c = warp - 1;
+    const size_t cs_stride = (tma_cs_floats(a.half, Src::kHi) + 3) & ~size_t(3);
+    CsSlot cs;
+    cs.c = slots + (size_t)c * cs_stride;
+    cs.s = cs.c + a.half;
+    cs.ns = cs.s + a.half + 4;
+    cs.ch = Src::kHi ? cs.ns + a.half + 4 : cs.c;
+    cs.sh = Src::kHi ? cs.ch + a.half : cs.s;
+    long long it = 0;
+    for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        const int s = (int)(it % S);
+        bool ok = mbar_wait(smem_addr(&bars[s]), (uint32_t)((it / S) & 1), a.wait_limit, abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+            if (lane == 0) {
+                if (!*abort) record_fault(a.status, kFaultFullWait);
+                *abort = 1;
+            }
+            break;
+        }
+        unsigned char *stage = smem + (size_t)s * a.stage_bytes;
+        const long long row = tile * a.P + c;
+        if (row < a.rows) {
+            unsigned char *sq = stage + (size_t)c * a.slot_q;
+            unsigned char *sk = stage + a.off_k + (size_t)c * a.slot_k;
+            src.angles(a, stage, c, row, lane, cs);
+            __syncwarp();
+            rotate_slots<T, VEC, Src::kHi>(a, sq, sk, lane, cs);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                if (a.hq) tma_store_3d(&a.tq1, smem_addr(sq), 0, 0, (int)row);
+                if (a.hk) tma_store_3d(&a.tk1, smem_addr(sk), 0, 0, (int)row);
+                bulk_commit();
+                bulk_wait_read_all();     // the slot may be refilled once the store has read it
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&bars[S + s]));
+    }
+    if (lane == 0) bulk_wait_all();
+}
+
+// --------------------------------------------------------------- launch
+// Lanes with bit `shift` of their index set read the second half first; the
+// shift with the fewest shared-memory bank conflicts for lane-per-row access
+// (row stride, half offset and access width in bytes).
+inline int best_swap_shift(unsigned row_bytes, unsigned half_bytes, unsigned access_bytes)
+{
+    int best = 3, best_cost = 1 << 30;
+    const unsigned lanes_per_wave = access_bytes >= 16 ? 8 : access_bytes == 8 ? 16 : 32;
+    for (int shift = 1; shift <= 4; ++shift) {
+        int cost = 0;
+        for (unsigned w0 = 0; w0 < 32; w0 += lanes_per_wave) {
+            int load[32] = {0};
+            for (unsigned l = w0; l < w0 + lanes_per_wave; ++l) {
+                const unsigned off = l * row_bytes + (((l >> shift) & 1) ? half_bytes : 0);
+                for (unsigned b = 0; b < access_bytes; b += 4) ++load[((off + b) / 4) % 32];
+            }
+            int worst = 0;
+            for (int b = 0; b < 32; ++b) worst = load[b] > worst ? load[b] : worst;
+            cost += worst;
+        }
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = shift;
+        }
+    }
+    return best;
+}
+
+// Fills the stage layout of `a`, picks the stage count for the shared-memory
+// budget and launches on the SMs.
+template <typename T, int VEC, class Src>
+cudaError_t launch_rotary_tma_vec(TmaRotArgs a, const Src &src, cudaStream_t s)
+{
+    const unsigned eb = sizeof(T);
+    const unsigned rot = 2u * a.half;
+    a.row_bytes_q = a.hq * rot * eb;
+    a.row_bytes_k = a.hk * rot * eb;
+    a.dense_q = a.row_bytes_q % 128 == 0;
+    a.dense_k = a.row_bytes_k % 128 == 0;
+    a.slot_q = align128(a.row_bytes_q);
+    a.slot_k = align128(a.row_bytes_k);
+    a.off_k = a.P * a.slot_q;
+    a.off_aux0 = a.off_k + a.P * a.slot_k;
+    const unsigned aux0 = a.aux_tma ? a.aux_bytes - (Src::kHi ? a.aux_bytes / 2 : 0) : 0;
+    a.off_aux1 = a.off_aux0 + align128(aux0);
+    a.stage_bytes = a.off_aux1 + align128(a.aux_tma && Src::kHi ? a.aux_bytes / 2 : 0);
+    const int H = a.hq + a.hk;
+    a.lane_rows = H <= 32 && (rot * eb) % 128 != 0;
+    a.swap_shift = best_swap_shift(rot * eb, a.half * eb, VEC * eb);
+    a.stages = 2;
+    for (int st = kTmaMaxStages; st >= 2; --st) {
+        a.stages = st;
+        if (tma_smem_bytes(a, Src::kHi) <= kTmaBlockSmem) break;
+    }
+    const size_t smem = tma_smem_bytes(a, Src::kHi);
+    auto kern = rotary_tma_kernel<T, VEC, Src>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kTmaThreads, smem);
+    if (e != cudaSuccess) return e;
+    const long long ntiles = (a.rows + a.P - 1) / a.P;
+    const long long cap = (long long)sm_count() * std::max(per_sm, 1);
+    const int blocks = (int)std::max<long long>(1, std::min(ntiles, cap));
+    kern<<<blocks, kTmaThreads, smem, s>>>(a, src);
+    return cudaGetLastError();
+}
+
+}  // namespace ipe

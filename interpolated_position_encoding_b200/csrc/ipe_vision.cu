@@ -4,7 +4,7 @@
 // "Qwen3-VL" notes (frankmowj.github.io), fast_pos_embed_interpolate,
 // rot_pos_emb, apply_rotary_pos_emb_vision; cortiq-engine qwen3vis.rs
 // (docs.rs), positions(), rope_angles(), attention().
-#include "ipe_rotary.cuh"
+#include "ipe_rotary_tma.cuh"
 
 namespace ipe {
 
@@ -200,6 +200,17 @@ cudaError_t launch_vis_interp(bool bf16, const VisDesc<1024> &d, const InterpArg
 template <typename T, int MAXIMG>
 static cudaError_t rope_impl(const VisDesc<1024> &d, const RotArgs &r, const VisAngleFreqs &f, cudaStream_t s)
 {
+    TmaRotArgs t;
+    if (tma_rot_args(r, sizeof(T), t)) {
+        t.aux_tma = 0;
+        VisTmaSrc<MAXIMG> src{shrink<MAXIMG>(d), f};
+        const int v = pick_vec(r, sizeof(T));
+        if constexpr (sizeof(T) == 2) {
+            if (v == 8) return launch_rotary_tma_vec<T, 8>(t, src, s);
+        }
+        if (v >= 4) return launch_rotary_tma_vec<T, 4>(t, src, s);
+        return launch_rotary_tma_vec<T, 2>(t, src, s);   // VEC >= 2 on the TMA path
+    }
     VisSrc<MAXIMG> src{shrink<MAXIMG>(d), f};
     return dispatch_vec<T>(r, src, s);
 }
