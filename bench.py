@@ -48,10 +48,29 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-variant side measurements")
+    ap.add_argument("--extras-reps", type=int, default=20, help="timed repetitions of each side measurement")
     return ap.parse_args()
 
 
 # ------------------------------------------------------------------ helpers
+
+
+def algorithmic_bytes_vision(v):
+    """Interpolation bytes: table rows the samples touch, read once, plus the output."""
+    import workloads as wl
+    N = wl.n_patches(v)
+    eb_v = 2 if v.dtype == "bf16" else 4
+    G = v.grid_side
+    touched = set()
+    for _, h, ww in v.grid_thw:
+        rows, cols = set(), set()
+        for n, s in ((h, rows), (ww, cols)):
+            for i in range(n):
+                num = i * (G - 1)
+                y0 = 0 if n == 1 else num // (n - 1)
+                s.update((y0, min(y0 + 1, G - 1)))
+        touched.update((y, x) for y in rows for x in cols)
+    return len(touched) * v.hidden * eb_v + N * v.hidden * eb_v
 
 
 def algorithmic_bytes(w):
@@ -60,20 +79,9 @@ def algorithmic_bytes(w):
     import workloads as wl
     N = wl.n_patches(v)
     eb_v = 2 if v.dtype == "bf16" else 4
-    G = v.grid_side
-    # table rows any sample touches: every grid row / column that is a corner
-    rows = set()
-    cols = set()
-    for _, h, ww in v.grid_thw:
-        for n, s in ((h, rows), (ww, cols)):
-            for i in range(n):
-                num = i * (G - 1)
-                y0 = 0 if n == 1 else num // (n - 1)
-                s.update((y0, min(y0 + 1, G - 1)))
-    U = len(rows) * len(cols)
     rot_bytes = (t.hq + t.hk) * t.T * t.rot_dim * 2 * 2
     return {
-        "vis_pos_interp": U * v.hidden * eb_v + N * v.hidden * eb_v,
+        "vis_pos_interp": algorithmic_bytes_vision(v),
         "vis_rope2d": 2 * N * v.heads * v.head_dim * eb_v * 2,
         "mrope_apply": rot_bytes + 3 * t.T * 4,
         "mrope_cos_sin": 3 * t.T * 4 + 2 * t.T * t.rot_dim * 4,
@@ -372,7 +380,8 @@ def main():
     extras = {}
     if not args.no_extras:
         extras = side_measurements(ipe, w, dev, stream, Q, K, pos, inv, table, qv, kv, out, alg, peak,
-                                   max(args.steps // 4, 20))
+                                   args.extras_reps)
+        extras["workloads"] = per_workload(ipe, dev, stream, peak, args.extras_reps)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -440,6 +449,92 @@ def side_measurements(ipe, w, dev, stream, Q, K, pos, inv, table, qv, kv, out, a
                                                                    out=out, stream=stream), reps)
     vb = alg["vis_pos_interp"] + alg["vis_rope2d"]
     res["vis_pos_interp_rope2d"] = {"ms": ms_vf, "gbs": vb / ms_vf / 1e6, "frac": vb / ms_vf / 1e6 / peak}
+    return res
+
+
+def _time_flushed(torch, stream, fn, reps, flush):
+    """Mean device time of fn.  Before each call (untimed) a buffer twice the
+    L2 is written and then read back, so the kernel starts with its inputs out
+    of L2 and with no dirty lines of the flush left to write back."""
+    fn()
+    total = 0.0
+    for _ in range(reps):
+        flush.zero_()
+        flush.max()
+        # keep the GPU busy while the host marshals the call, so the start
+        # event is not recorded before the kernel is queued
+        torch.cuda._sleep(1_000_000)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        total += a.elapsed_time(b)
+    return total / reps
+
+
+def per_workload(ipe, dev, stream, peak, reps):
+    """Every kernel of the library on each of the five workloads (L2 flushed
+    between timed calls): ms, algorithmic GB/s and fraction of the peak."""
+    import numpy as np
+    import torch
+    import workloads as wl
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+
+    def dev_t(a, dtype):
+        if dtype == "bf16":
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(a).to(dev)
+
+    def entry(ms, nbytes):
+        return {"ms": ms, "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / peak}
+
+    for name, w in wl.WORKLOADS.items():
+        r = {}
+        if w.vision is not None:
+            v = w.vision
+            vin = wl.vision_inputs(w)
+            N = wl.n_patches(v)
+            eb = 2 if v.dtype == "bf16" else 4
+            table, q, k = dev_t(vin["table"], v.dtype), dev_t(vin["q"], v.dtype), dev_t(vin["k"], v.dtype)
+            out = torch.empty(N, v.hidden, dtype=table.dtype, device=dev)
+            ib = algorithmic_bytes_vision(v)
+            rb = 2 * N * v.heads * v.head_dim * eb * 2
+            r["vis_pos_interp"] = entry(_time_flushed(
+                torch, stream, lambda: ipe.vis_pos_interp(table, v.grid_thw, v.merge, out=out, stream=stream), reps,
+                flush), ib)
+            r["vis_rope2d"] = entry(_time_flushed(
+                torch, stream, lambda: ipe.vis_rope2d(q, k, v.grid_thw, v.merge, v.theta, stream=stream), reps,
+                flush), rb)
+            r["vis_pos_interp_rope2d"] = entry(_time_flushed(
+                torch, stream, lambda: ipe.vis_pos_interp_rope2d(table, v.grid_thw, q, k, v.merge, v.theta, out=out,
+                                                                 stream=stream), reps, flush), ib + rb)
+            r["patches"] = N
+        if w.text is not None:
+            t = w.text
+            tin = wl.text_inputs(w)
+            Q, K = dev_t(tin["q"], "bf16"), dev_t(tin["k"], "bf16")
+            pos = torch.from_numpy(tin["positions"]).to(dev)
+            inv = ipe.rope_inv_freq(t.rot_dim, t.theta)
+            cos = torch.empty(t.T, t.rot_dim, dtype=torch.float32, device=dev)
+            sin = torch.empty_like(cos)
+            rot = (t.hq + t.hk) * t.T * t.rot_dim * 2 * 2
+            for layout in t.layouts:
+                il = layout == "interleaved"
+                r[f"mrope_apply/{layout}"] = entry(_time_flushed(
+                    torch, stream, lambda: ipe.mrope_apply(Q, K, pos, inv, t.section, il, stream=stream), reps,
+                    flush), rot + 3 * t.T * 4)
+                r[f"mrope_cos_sin/{layout}"] = entry(_time_flushed(
+                    torch, stream, lambda: ipe.mrope_cos_sin(pos, inv, t.section, il, cos, sin, stream=stream), reps,
+                    flush), 3 * t.T * 4 + 2 * t.T * t.rot_dim * 4)
+                r[f"apply_rotary_partial/{layout}"] = entry(_time_flushed(
+                    torch, stream, lambda: ipe.apply_rotary_partial(Q, K, cos, sin, stream=stream), reps, flush),
+                    rot + 2 * t.T * t.rot_dim * 4)
+            r["tokens"] = t.T
+        res[name] = r
+        torch.cuda.empty_cache()
+    ipe.device_status(stream)
     return res
 
 

@@ -86,26 +86,48 @@ def _cuda(t, name):
     return t
 
 
+try:
+    _raw_stream = torch._C._cuda_getCurrentRawStream
+except AttributeError:  # pragma: no cover - older torch
+    _raw_stream = None
+
+
 def _stream(stream):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream)
+    if _raw_stream is not None:
+        return ctypes.c_void_p(_raw_stream(torch.cuda.current_device()))
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+# Small caches of host arrays passed by value (keys are immutable tuples).
+_HOST_CACHE = {}
+
+
+def _cached(key, make):
+    v = _HOST_CACHE.get(key)
+    if v is None:
+        if len(_HOST_CACHE) > 256:
+            _HOST_CACHE.clear()
+        v = _HOST_CACHE[key] = make()
+    return v
 
 
 def _i32_host(values, n=None):
-    arr = (ctypes.c_int32 * len(values))(*[int(v) for v in values])
+    values = tuple(int(v) for v in values)
     if n is not None and len(values) != n:
         raise ValueError(f"expected {n} values, got {len(values)}")
-    return arr
+    return _cached(("i32",) + values, lambda: (ctypes.c_int32 * len(values))(*values))
 
 
 def _grid_host(grid_thw):
     if isinstance(grid_thw, torch.Tensor):
-        grid_thw = grid_thw.detach().cpu().reshape(-1).tolist()
+        flat = tuple(grid_thw.detach().cpu().reshape(-1).tolist())
     else:
-        grid_thw = [int(v) for g in grid_thw for v in (g if hasattr(g, "__len__") else [g])]
-    if len(grid_thw) % 3:
+        flat = tuple(int(v) for g in grid_thw for v in (g if hasattr(g, "__len__") else [g]))
+    if len(flat) % 3:
         raise ValueError("grid_thw must hold (t, h, w) triples")
-    return _i32_host(grid_thw), len(grid_thw) // 3
+    return _i32_host(flat), len(flat) // 3
 
 
 def _ptr(t):
@@ -150,8 +172,14 @@ def mrope_axis_map(half, section, interleaved=True, device="cuda", stream=None):
 
 
 def _inv_host(inv_freq):
-    vals = inv_freq.detach().float().cpu().tolist() if isinstance(inv_freq, torch.Tensor) else list(inv_freq)
-    return (ctypes.c_float * len(vals))(*vals), len(vals)
+    if isinstance(inv_freq, torch.Tensor):
+        if inv_freq.is_cuda:
+            raise TypeError("inv_freq must be a host tensor or sequence (it travels as a kernel parameter)")
+        vals = tuple(inv_freq.detach().float().reshape(-1).tolist())
+    else:
+        vals = tuple(float(v) for v in inv_freq)
+    arr = _cached(("inv",) + vals, lambda: (ctypes.c_float * len(vals))(*vals))
+    return arr, len(vals)
 
 
 def mrope_cos_sin(positions, inv_freq, section, interleaved=True, cos=None, sin=None, stream=None):

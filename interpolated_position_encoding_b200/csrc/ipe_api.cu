@@ -293,7 +293,7 @@ bool tma_rot_args(const RotArgs &r, int eb, TmaRotArgs &t)
     if (r.hq > 256 || r.hk > 256 || r.rows <= 0 || r.rows > 0x7fffffffLL) return false;
     // one stage (P rows of q and k) must stay far below the shared memory and
     // the 2^20-byte transaction count of a barrier phase
-    if ((size_t)kTmaRows * (r.hq + r.hk) * rot * eb > 64 * 1024) return false;
+    if ((size_t)kTmaRows * (r.hq + r.hk) * rot * eb > 96 * 1024) return false;
     const CUtensorMapDataType dt = eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     t = TmaRotArgs{};
     t.P = kTmaRows;

@@ -27,37 +27,73 @@ cudaError_t launch_mrope_axis_map(int half, const int *section, int interleaved,
 }
 
 // ---------------------------------------------------------- cos / sin
-// One thread per (token, frequency); writes both halves of cat(f, f).
+// Block (G, 256 / G): threadIdx.x is one of the G = half / V groups of V
+// consecutive frequencies of a token, threadIdx.y a token.  Each thread
+// takes U tokens per pass (their position loads in flight together) and
+// writes both halves of cat(f, f) for cos and sin with V-wide stores.
+template <int V>
 __global__ void __launch_bounds__(256) mrope_cos_sin_kernel(const __grid_constant__ MropeAngles a, int half,
                                                              float *__restrict__ cos_out,
                                                              float *__restrict__ sin_out)
 {
-    const long long total = a.T * half;
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
-        const long long t = i / half;
-        const int j = (int)(i - t * half);
-        const int ax = mrope_axis(j, a.section, a.interleaved);
-        const int pos = __ldg(a.positions + (long long)ax * a.T + t);
-        const float angle = __fmul_rn(__int2float_rn(pos), a.inv[j]);
-        float s, c;
-        sincosf(angle, &s, &c);
-        const long long o = t * 2 * half + j;
-        cos_out[o] = c;
-        cos_out[o + half] = c;
-        sin_out[o] = s;
-        sin_out[o + half] = s;
+    constexpr int U = 2;
+    const int j0 = threadIdx.x * V;
+    int ax[V];
+    float inv[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) {          // fixed per thread: its frequencies
+        ax[e] = mrope_axis(j0 + e, a.section, a.interleaved);
+        inv[e] = a.inv[j0 + e];
     }
+    const long long stride = (long long)gridDim.x * blockDim.y;
+    for (long long t0 = (long long)blockIdx.x * blockDim.y + threadIdx.y; t0 < a.T; t0 += U * stride) {
+        int p0[U], p1[U], p2[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long t = t0 + u * stride;
+            if (t < a.T) {
+                p0[u] = __ldg(a.positions + t);
+                p1[u] = __ldg(a.positions + a.T + t);
+                p2[u] = __ldg(a.positions + 2 * a.T + t);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long t = t0 + u * stride;
+            if (t >= a.T) break;
+            Pack<float, V> c, s;
+#pragma unroll
+            for (int e = 0; e < V; ++e) {
+                const int pos = ax[e] == 0 ? p0[u] : (ax[e] == 1 ? p1[u] : p2[u]);
+                const float angle = __fmul_rn(__int2float_rn(pos), inv[e]);
+                sincosf(angle, &s.v[e], &c.v[e]);
+            }
+            float *co = cos_out + t * 2 * half + j0;
+            float *so = sin_out + t * 2 * half + j0;
+            st_pack<float, V>(co, c);
+            st_pack<float, V>(co + half, c);
+            st_pack<float, V>(so, s);
+            st_pack<float, V>(so + half, s);
+        }
+    }
+}
+
+template <int V>
+static cudaError_t cos_sin_vec(const MropeAngles &a, int half, float *cos_out, float *sin_out, cudaStream_t s)
+{
+    const int gx = half / V;
+    const int gy = std::max(1, 256 / gx);
+    const long long need = (a.T + 2LL * gy - 1) / (2LL * gy);     // 2 tokens per thread and pass
+    const int blocks = (int)std::max<long long>(1, std::min(need, (long long)sm_count() * 8));
+    mrope_cos_sin_kernel<V><<<blocks, dim3(gx, gy), 0, s>>>(a, half, cos_out, sin_out);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_mrope_cos_sin(const MropeAngles &a, int half, float *cos_out, float *sin_out,
                                  cudaStream_t s)
 {
-    const long long total = a.T * half;
-    const long long need = (total + 255) / 256;
-    const int blocks = (int)std::min<long long>(need, (long long)sm_count() * 8);
-    mrope_cos_sin_kernel<<<blocks, 256, 0, s>>>(a, half, cos_out, sin_out);
-    return cudaGetLastError();
+    const bool v4 = half % 4 == 0 && (uintptr_t)cos_out % 16 == 0 && (uintptr_t)sin_out % 16 == 0;
+    return v4 ? cos_sin_vec<4>(a, half, cos_out, sin_out, s) : cos_sin_vec<1>(a, half, cos_out, sin_out, s);
 }
 
 // Widest vector (elements) that divides half, head_dim and both strides and

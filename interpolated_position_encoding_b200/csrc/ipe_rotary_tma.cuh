@@ -260,11 +260,12 @@ __host__ __device__ inline size_t tma_smem_bytes(const TmaRotArgs &a, bool hi)
     return 128 + (size_t)a.stages * a.stage_bytes + 16 * (size_t)a.stages + 16 + (size_t)kTmaConsumers * cs;
 }
 
+// The whole pipeline of one block over tiles bid, bid + nb, ... (the caller
+// passes its dynamic shared memory).
 template <typename T, int VEC, class Src>
-__global__ void __launch_bounds__(kTmaThreads) rotary_tma_kernel(const __grid_constant__ TmaRotArgs a,
-                                                                 const __grid_constant__ Src src)
+__device__ __forceinline__ void rotary_tma_block(const TmaRotArgs &a, const Src &src, unsigned char *smem_raw,
+                                                 long long bid, long long nb)
 {
-    extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
     const int S = a.stages;
@@ -294,7 +295,7 @@ __global__ void __launch_bounds__(kTmaThreads) rotary_tma_kernel(const __grid_co
         for (int s = 0; s < kTmaMaxStages; ++s) last_round[s] = -1;
         bool aborted = false;
         long long it = 0;
-        for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        for (long long tile = bid; tile < ntiles; tile += nb, ++it) {
             const int s = (int)(it % S);
             const long long round = it / S;
             if (!mbar_wait(smem_addr(&bars[S + s]), (uint32_t)((round & 1) ^ 1), a.wait_limit, abort)) {
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(kTmaThreads) rotary_tma_kernel(const __grid_co
     cs.ch = Src::kHi ? cs.ns + a.half + 4 : cs.c;
     cs.sh = Src::kHi ? cs.ch + a.half : cs.s;
     long long it = 0;
-    for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    for (long long tile = bid; tile < ntiles; tile += nb, ++it) {
         const int s = (int)(it % S);
         bool ok = mbar_wait(smem_addr(&bars[s]), (uint32_t)((it / S) & 1), a.wait_limit, abort);
         ok = __all_sync(0xffffffffu, ok);
@@ -381,6 +382,14 @@ __global__ void __launch_bounds__(kTmaThreads) rotary_tma_kernel(const __grid_co
     if (lane == 0) bulk_wait_all();
 }
 
+template <typename T, int VEC, class Src>
+__global__ void __launch_bounds__(kTmaThreads) rotary_tma_kernel(const __grid_constant__ TmaRotArgs a,
+                                                                 const __grid_constant__ Src src)
+{
+    extern __shared__ unsigned char smem_raw[];
+    rotary_tma_block<T, VEC, Src>(a, src, smem_raw, blockIdx.x, gridDim.x);
+}
+
 // --------------------------------------------------------------- launch
 // Lanes with bit `shift` of their index set read the second half first; the
 // shift with the fewest shared-memory bank conflicts for lane-per-row access
@@ -409,10 +418,10 @@ inline int best_swap_shift(unsigned row_bytes, unsigned half_bytes, unsigned acc
     return best;
 }
 
-// Fills the stage layout of `a`, picks the stage count for the shared-memory
-// budget and launches on the SMs.
+// Fills the stage layout of `a` and picks the stage count for the
+// shared-memory budget.
 template <typename T, int VEC, class Src>
-cudaError_t launch_rotary_tma_vec(TmaRotArgs a, const Src &src, cudaStream_t s)
+void tma_layout(TmaRotArgs &a)
 {
     const unsigned eb = sizeof(T);
     const unsigned rot = 2u * a.half;
@@ -430,11 +439,23 @@ cudaError_t launch_rotary_tma_vec(TmaRotArgs a, const Src &src, cudaStream_t s)
     const int H = a.hq + a.hk;
     a.lane_rows = H <= 32 && (rot * eb) % 128 != 0;
     a.swap_shift = best_swap_shift(rot * eb, a.half * eb, VEC * eb);
-    a.stages = 2;
-    for (int st = kTmaMaxStages; st >= 2; --st) {
-        a.stages = st;
-        if (tma_smem_bytes(a, Src::kHi) <= kTmaBlockSmem) break;
+    // deepest ring within ~112 KB (two blocks per SM); rows too wide for two
+    // stages there get up to ~220 KB (one block per SM)
+    for (size_t budget : {kTmaBlockSmem, size_t(220 * 1024)}) {
+        a.stages = 2;
+        for (int st = kTmaMaxStages; st >= 2; --st) {
+            a.stages = st;
+            if (tma_smem_bytes(a, Src::kHi) <= budget) break;
+        }
+        if (tma_smem_bytes(a, Src::kHi) <= budget) break;
     }
+}
+
+// Lays out `a` and launches the pipeline on the SMs.
+template <typename T, int VEC, class Src>
+cudaError_t launch_rotary_tma_vec(TmaRotArgs a, const Src &src, cudaStream_t s)
+{
+    tma_layout<T, VEC, Src>(a);
     const size_t smem = tma_smem_bytes(a, Src::kHi);
     auto kern = rotary_tma_kernel<T, VEC, Src>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -13,10 +13,13 @@ constexpr int kInterpThreads = 256;
 // Channels of one interpolation block: 128 bytes of every output row.
 template <typename T> constexpr int interp_slice() { return 128 / (int)sizeof(T); }
 
+// Column samples cached per block (images at most this wide).
+constexpr int kColCache = 1024;
+
 size_t interp_smem_bytes(bool bf16, int merge, int grid_side)
 {
     const int cs = bf16 ? interp_slice<__nv_bfloat16>() : interp_slice<float>();
-    return (size_t)merge * grid_side * cs * sizeof(float);
+    return (size_t)merge * grid_side * cs * sizeof(float) + kColCache * sizeof(int2);
 }
 
 // ---------------------------------------------------------------- plan
@@ -62,92 +65,200 @@ __global__ void vis_plan_kernel(const __grid_constant__ VisDesc<MAXIMG> d, int32
 //            table column the strip samples (shared memory, fp32);
 //   phase 2  out = (1-dx) R[iy][x0] + dx R[iy][x1], rounded once, written to
 //            every frame (frames of a video repeat frame 0).
-// Each table entry is read once per block instead of once per corner.
-template <typename T, int MAXIMG>
+// Each table entry is read once per block instead of once per corner; lanes
+// move E channels per access (16 bytes when rows are 16-byte aligned).
+template <typename T, int E, int M, int MAXIMG>
 __device__ __forceinline__ void interp_block(const VisDesc<MAXIMG> &d, const InterpArgs &ia, int strip,
-                                             int slice, float4 *R)
+                                             int slice, unsigned char *smem)
 {
-    constexpr int CS = interp_slice<T>();
-    constexpr int NV = CS / 4;                        // 4-channel vectors of a full slice
-    const VisImage &im = d.img[find_image_of_strip(d, strip)];
-    const int m = d.merge, G = d.grid_side, C = ia.hidden;
-    const int by = strip - im.strip0;
+    constexpr int CS = interp_slice<T>();             // E: channels per lane access (4, or 8 for bf16)
+    constexpr int NVM = CS / E;                       // lanes of one row slice (a power of two)
+    constexpr int NV4 = CS / 4;                       // float4 of one R entry
+    // image fields in registers (a dynamic index into the parameter block
+    // would otherwise be re-read inside the loops)
+    const int ii = find_image_of_strip(d, strip);
+    const int im_t = d.img[ii].t, im_h = d.img[ii].h, im_w = d.img[ii].w, strip0 = d.img[ii].strip0;
+    const long long row0 = d.img[ii].row0;
+    const int m = M ? M : d.merge, G = d.grid_side, C = ia.hidden;
+    float4 *R = reinterpret_cast<float4 *>(smem);
+    int2 *cols = reinterpret_cast<int2 *>(smem + (size_t)m * G * CS * sizeof(float));
+    const int by = strip - strip0;
     const int c0 = slice * CS;
-    const int nv = min(CS, C - c0) / 4;
+    const int cw = min(CS, C - c0);
+    const int nv = (cw + E - 1) / E;                  // lanes in use for this slice
     int xl0, xl1;
     float dl;
-    grid_sample(im.w - 1, im.w, G, xl0, xl1, dl);
+    grid_sample(im_w - 1, im_w, G, xl0, xl1, dl);
     const int ncols = xl1 + 1;                        // columns 0 .. x1 of the last sample
+    const int v = threadIdx.x % NVM;
+    const int rstep = blockDim.x / NVM;
 
-    const T *tab = static_cast<const T *>(ia.table);
-    for (int i = threadIdx.x; i < m * ncols * nv; i += blockDim.x) {
-        const int v = i % nv;
-        const int t2 = i / nv;
-        const int gx = t2 % ncols, iy = t2 / ncols;
-        int y0, y1;
-        float dy;
-        grid_sample(by * m + iy, im.h, G, y0, y1, dy);
-        const float omdy = __fsub_rn(1.f, dy);
-        const Pack<T, 4> a = ld_pack<T, 4>(tab + (size_t)(y0 * G + gx) * C + c0 + 4 * v);
-        const Pack<T, 4> b = ld_pack<T, 4>(tab + (size_t)(y1 * G + gx) * C + c0 + 4 * v);
-        float4 r;
-        r.x = __fmaf_rn(dy, to_f32(b.v[0]), __fmul_rn(omdy, to_f32(a.v[0])));
-        r.y = __fmaf_rn(dy, to_f32(b.v[1]), __fmul_rn(omdy, to_f32(a.v[1])));
-        r.z = __fmaf_rn(dy, to_f32(b.v[2]), __fmul_rn(omdy, to_f32(a.v[2])));
-        r.w = __fmaf_rn(dy, to_f32(b.v[3]), __fmul_rn(omdy, to_f32(a.v[3])));
-        R[(iy * ncols + gx) * NV + v] = r;
+    // column samples once per block (phase 2 reads them back)
+    const bool cached = im_w <= kColCache;
+    if (cached)
+        for (int x = threadIdx.x; x < im_w; x += blockDim.x) {
+            int x0, x1;
+            float dx;
+            grid_sample(x, im_w, G, x0, x1, dx);
+            cols[x] = make_int2(x0 | (x1 << 16), __float_as_int(dx));
+        }
+
+    // phase 1: y-blend of the strip's m patch rows.  R entry (iy, gx) holds
+    // NV4 float4; lane v keeps its E / 4 chunks at float4 v + NVM q, so
+    // neighbouring lanes touch neighbouring banks in both phases.
+    int ry0[M ? M : 1], ry1[M ? M : 1];
+    float rdy[M ? M : 1];
+    if constexpr (M != 0) {
+#pragma unroll
+        for (int iy = 0; iy < M; ++iy) grid_sample(by * M + iy, im_h, G, ry0[iy], ry1[iy], rdy[iy]);
+    }
+    auto row_sample = [&](int iy, int &y0, int &y1, float &dy) {
+        if constexpr (M != 0) {
+            y0 = ry0[0];
+            y1 = ry1[0];
+            dy = rdy[0];
+#pragma unroll
+            for (int k = 1; k < M; ++k)
+                if (iy == k) {
+                    y0 = ry0[k];
+                    y1 = ry1[k];
+                    dy = rdy[k];
+                }
+        } else {
+            grid_sample(by * m + iy, im_h, G, y0, y1, dy);
+        }
+    };
+    const T *tab_v = static_cast<const T *>(ia.table) + c0 + E * v;
+    const int nrows = m * ncols;
+    const bool full = E * v + E <= cw;           // else: the 4-channel tail of the last slice
+    if (v < nv) {
+        int r = threadIdx.x / NVM;
+        int iy = r / ncols, gx = r - iy * ncols;
+        for (; r < nrows; r += rstep) {
+            int y0, y1;
+            float dy;
+            row_sample(iy, y0, y1, dy);
+            const float2 DY = make_float2(dy, dy);
+            const float omdy = __fsub_rn(1.f, dy);
+            const float2 OMDY = make_float2(omdy, omdy);
+            const T *ra = tab_v + (size_t)(y0 * G + gx) * C;
+            const T *rb = tab_v + (size_t)(y1 * G + gx) * C;
+            float4 *dst = R + r * NV4 + v;
+            if (full) {
+                float2 a[E / 2], b[E / 2];
+                load_pairs<T, E>(ra, a);
+                load_pairs<T, E>(rb, b);
+#pragma unroll
+                for (int q = 0; q < E / 4; ++q) {
+                    // (1-dy) a + dy b, as fma(dy, b, (1-dy) a)
+                    const float2 lo = fma2(DY, b[2 * q], mul2(OMDY, a[2 * q]));
+                    const float2 hi = fma2(DY, b[2 * q + 1], mul2(OMDY, a[2 * q + 1]));
+                    dst[NVM * q] = make_float4(lo.x, lo.y, hi.x, hi.y);
+                }
+            } else {
+                float2 a[2], b[2];
+                load_pairs<T, 4>(ra, a);
+                load_pairs<T, 4>(rb, b);
+                const float2 lo = fma2(DY, b[0], mul2(OMDY, a[0]));
+                const float2 hi = fma2(DY, b[1], mul2(OMDY, a[1]));
+                dst[0] = make_float4(lo.x, lo.y, hi.x, hi.y);
+            }
+            gx += rstep;                           // next row of this thread
+            while (gx >= ncols) {
+                gx -= ncols;
+                ++iy;
+            }
+        }
     }
     __syncthreads();
 
-    const long long hw = (long long)im.h * im.w;
-    const long long strip_row0 = im.row0 + (long long)by * m * im.w;
-    T *out = static_cast<T *>(ia.out);
-    for (int i = threadIdx.x; i < m * im.w * nv; i += blockDim.x) {
-        const int v = i % nv;
-        const int p = i / nv;                         // patch of the strip, merge order
-        const int bx = p / (m * m), rr = p - bx * m * m;
-        const int iy = rr / m, ix = rr - iy * m;
-        int x0, x1;
-        float dx;
-        grid_sample(bx * m + ix, im.w, G, x0, x1, dx);
-        const float omdx = __fsub_rn(1.f, dx);
-        const float4 r0 = R[(iy * ncols + x0) * NV + v];
-        const float4 r1 = R[(iy * ncols + x1) * NV + v];
-        Pack<T, 4> o;
-        o.v[0] = from_f32<T>(__fmaf_rn(dx, r1.x, __fmul_rn(omdx, r0.x)));
-        o.v[1] = from_f32<T>(__fmaf_rn(dx, r1.y, __fmul_rn(omdx, r0.y)));
-        o.v[2] = from_f32<T>(__fmaf_rn(dx, r1.z, __fmul_rn(omdx, r0.z)));
-        o.v[3] = from_f32<T>(__fmaf_rn(dx, r1.w, __fmul_rn(omdx, r0.w)));
-        T *dst = out + (size_t)(strip_row0 + p) * C + c0 + 4 * v;
-        for (int f = 0; f < im.t; ++f)
-            st_pack<T, 4>(dst + (size_t)f * hw * C, o);
+    // phase 2: x-blend, one rounding, every frame
+    const size_t frame = (size_t)im_h * im_w * C;    // elements between frames
+    T *out_v = static_cast<T *>(ia.out) + (size_t)(row0 + (long long)by * m * im_w) * C + c0 + E * v;
+    if (v < nv) {
+        for (int p = threadIdx.x / NVM; p < m * im_w; p += rstep) {
+            int bx, iy, ix;                       // patch of the strip, merge order
+            if constexpr (M == 2) {
+                bx = p >> 2;
+                iy = (p >> 1) & 1;
+                ix = p & 1;
+            } else {
+                bx = p / (m * m);
+                const int rr = p - bx * m * m;
+                iy = rr / m;
+                ix = rr - iy * m;
+            }
+            const int col = bx * m + ix;
+            int x0, x1;
+            float dx;
+            if (cached) {
+                const int2 cc = cols[col];
+                x0 = cc.x & 0xffff;
+                x1 = cc.x >> 16;
+                dx = __int_as_float(cc.y);
+            } else {
+                grid_sample(col, im_w, G, x0, x1, dx);
+            }
+            const float2 DX = make_float2(dx, dx);
+            const float omdx = __fsub_rn(1.f, dx);
+            const float2 OMDX = make_float2(omdx, omdx);
+            const float4 *r0 = R + (iy * ncols + x0) * NV4 + v;
+            const float4 *r1 = R + (iy * ncols + x1) * NV4 + v;
+            T *dst = out_v + (size_t)p * C;
+            if (full) {
+                float2 o[E / 2];
+#pragma unroll
+                for (int q = 0; q < E / 4; ++q) {
+                    const float4 a = r0[NVM * q], b = r1[NVM * q];
+                    o[2 * q] = fma2(DX, make_float2(b.x, b.y), mul2(OMDX, make_float2(a.x, a.y)));
+                    o[2 * q + 1] = fma2(DX, make_float2(b.z, b.w), mul2(OMDX, make_float2(a.z, a.w)));
+                }
+                for (int f = 0; f < im_t; ++f) store_pairs<T, E>(dst + f * frame, o);
+            } else {
+                const float4 a = r0[0], b = r1[0];
+                float2 o[2];
+                o[0] = fma2(DX, make_float2(b.x, b.y), mul2(OMDX, make_float2(a.x, a.y)));
+                o[1] = fma2(DX, make_float2(b.z, b.w), mul2(OMDX, make_float2(a.z, a.w)));
+                for (int f = 0; f < im_t; ++f) store_pairs<T, 4>(dst + f * frame, o);
+            }
+        }
     }
 }
 
-template <typename T, int MAXIMG>
-__global__ void __launch_bounds__(kInterpThreads) vis_interp_kernel(const __grid_constant__ VisDesc<MAXIMG> d,
+template <typename T, int E, int M, int MAXIMG>
+__global__ void __launch_bounds__(kInterpThreads, 6) vis_interp_kernel(const __grid_constant__ VisDesc<MAXIMG> d,
                                                                     const __grid_constant__ InterpArgs ia)
 {
-    extern __shared__ float4 R[];
+    extern __shared__ __align__(16) unsigned char smem[];
     const int b = blockIdx.x;
-    interp_block<T, MAXIMG>(d, ia, b / ia.n_slices, b % ia.n_slices, R);
+    interp_block<T, E, M, MAXIMG>(d, ia, b / ia.n_slices, b % ia.n_slices, smem);
+}
+
+// 16-byte accesses need 16-byte-aligned rows and base pointers.
+template <typename T>
+static bool interp_wide(const InterpArgs &ia)
+{
+    constexpr int E = 16 / (int)sizeof(T);
+    return ia.hidden % E == 0 && (uintptr_t)ia.table % 16 == 0 && (uintptr_t)ia.out % 16 == 0;
 }
 
 // --------------------------------------------------------------- fused
-// Blocks [0, n_strips * n_slices) interpolate; the rest rotate q and k.
-template <typename T, int VEC, int MAXIMG>
-__global__ void __launch_bounds__(kRotThreads) vis_fused_kernel(const __grid_constant__ VisSrc<MAXIMG> src,
+// One persistent launch: every block first takes interpolation work items
+// (strip x channel slice) in a grid-stride loop, using its shared memory as
+// the blend buffer, then runs the TMA rotary pipeline over its tiles of q, k.
+template <typename T, int VEC, int E, int M, int MAXIMG>
+__global__ void __launch_bounds__(kTmaThreads, 2) vis_fused_kernel(const __grid_constant__ VisTmaSrc<MAXIMG> src,
                                                                 const __grid_constant__ InterpArgs ia,
-                                                                const __grid_constant__ RotArgs r)
+                                                                const __grid_constant__ TmaRotArgs r)
 {
-    extern __shared__ __align__(16) unsigned char smem[];
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *R = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const int n_interp = src.d.n_strips * ia.n_slices;
-    if ((int)blockIdx.x < n_interp) {
-        interp_block<T, MAXIMG>(src.d, ia, blockIdx.x / ia.n_slices, blockIdx.x % ia.n_slices,
-                                reinterpret_cast<float4 *>(smem));
-    } else {
-        rotary_tiles<T, VEC, VisSrc<MAXIMG>>(r, src, blockIdx.x - n_interp, gridDim.x - n_interp, smem);
+    for (int item = blockIdx.x; item < n_interp; item += gridDim.x) {
+        interp_block<T, E, M, MAXIMG>(src.d, ia, item / ia.n_slices, item % ia.n_slices, R);
+        __syncthreads();          // R is reused by the next item / the pipeline
     }
+    rotary_tma_block<T, VEC, VisTmaSrc<MAXIMG>>(r, src, smem_raw, blockIdx.x, gridDim.x);
 }
 
 // ------------------------------------------------------------- launches
@@ -181,7 +292,9 @@ template <typename T, int MAXIMG>
 static cudaError_t interp_impl(const VisDesc<1024> &d, const InterpArgs &ia, cudaStream_t s)
 {
     const size_t smem = interp_smem_bytes(sizeof(T) == 2, d.merge, d.grid_side);
-    auto kern = vis_interp_kernel<T, MAXIMG>;
+    const bool wide = interp_wide<T>(ia), m2 = d.merge == 2;
+    auto kern = wide ? (m2 ? vis_interp_kernel<T, 16 / sizeof(T), 2, MAXIMG> : vis_interp_kernel<T, 16 / sizeof(T), 0, MAXIMG>)
+                     : (m2 ? vis_interp_kernel<T, 4, 2, MAXIMG> : vis_interp_kernel<T, 4, 0, MAXIMG>);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
@@ -224,39 +337,49 @@ cudaError_t launch_vis_rope(bool bf16, const VisDesc<1024> &d, const RotArgs &r,
 }
 
 template <typename T, int VEC, int MAXIMG>
-static cudaError_t fused_vec(const VisDesc<1024> &d, const InterpArgs &ia, RotArgs r, const VisAngleFreqs &f,
+static cudaError_t fused_vec(const VisDesc<1024> &d, const InterpArgs &ia, TmaRotArgs t, const VisAngleFreqs &f,
                              cudaStream_t s)
 {
-    r.rows_per_tile = pick_rows_per_tile(r, VEC);
-    const size_t smem = std::max(interp_smem_bytes(sizeof(T) == 2, d.merge, d.grid_side),
-                                 rot_smem_bytes(r.rows_per_tile, r.half, false));
-    auto kern = vis_fused_kernel<T, VEC, MAXIMG>;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRotThreads, smem);
+    tma_layout<T, VEC, VisTmaSrc<MAXIMG>>(t);
+    const size_t smem = std::max(interp_smem_bytes(sizeof(T) == 2, d.merge, d.grid_side) + 128,
+                                 tma_smem_bytes(t, false));
+    const bool wide = interp_wide<T>(ia), m2 = d.merge == 2;
+    auto kern = wide ? (m2 ? vis_fused_kernel<T, VEC, 16 / sizeof(T), 2, MAXIMG> : vis_fused_kernel<T, VEC, 16 / sizeof(T), 0, MAXIMG>)
+                     : (m2 ? vis_fused_kernel<T, VEC, 4, 2, MAXIMG> : vis_fused_kernel<T, VEC, 4, 0, MAXIMG>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const long long ntiles = (r.rows + r.rows_per_tile - 1) / r.rows_per_tile;
-    const long long n_rope = std::max<long long>(1, std::min(ntiles, (long long)sm_count() * std::max(per_sm, 1)));
-    const long long n_interp = (long long)d.n_strips * ia.n_slices;
-    VisSrc<MAXIMG> src{shrink<MAXIMG>(d), f};
-    kern<<<(unsigned)(n_interp + n_rope), kRotThreads, smem, s>>>(src, ia, r);
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kTmaThreads, smem);
+    if (e != cudaSuccess) return e;
+    const long long ntiles = (t.rows + t.P - 1) / t.P;
+    const long long work = std::max(ntiles, (long long)d.n_strips * ia.n_slices);
+    const long long cap = (long long)sm_count() * std::max(per_sm, 1);
+    const int blocks = (int)std::max<long long>(1, std::min(work, cap));
+    VisTmaSrc<MAXIMG> src{shrink<MAXIMG>(d), f};
+    kern<<<blocks, kTmaThreads, smem, s>>>(src, ia, t);
     return cudaGetLastError();
 }
 
+// The fused launch needs the TMA rotary path; shapes it cannot take run as
+// two launches (interpolation, then the vector-load rotary).
 template <typename T, int MAXIMG>
 static cudaError_t fused_impl(const VisDesc<1024> &d, const InterpArgs &ia, const RotArgs &r,
                               const VisAngleFreqs &f, cudaStream_t s)
 {
-    const int v = pick_vec(r, sizeof(T));
-    if constexpr (sizeof(T) == 2) {
-        if (v == 8) return fused_vec<T, 8, MAXIMG>(d, ia, r, f, s);
+    TmaRotArgs t;
+    if (tma_rot_args(r, sizeof(T), t) && interp_smem_bytes(sizeof(T) == 2, d.merge, d.grid_side) + 128 <= 200 * 1024) {
+        t.aux_tma = 0;
+        const int v = pick_vec(r, sizeof(T));
+        if constexpr (sizeof(T) == 2) {
+            if (v == 8) return fused_vec<T, 8, MAXIMG>(d, ia, t, f, s);
+        }
+        if (v >= 4) return fused_vec<T, 4, MAXIMG>(d, ia, t, f, s);
+        return fused_vec<T, 2, MAXIMG>(d, ia, t, f, s);
     }
-    if (v >= 4) return fused_vec<T, 4, MAXIMG>(d, ia, r, f, s);
-    if (v == 2) return fused_vec<T, 2, MAXIMG>(d, ia, r, f, s);
-    return fused_vec<T, 1, MAXIMG>(d, ia, r, f, s);
+    cudaError_t e = interp_impl<T, MAXIMG>(d, ia, s);
+    if (e != cudaSuccess) return e;
+    VisSrc<MAXIMG> src{shrink<MAXIMG>(d), f};
+    return dispatch_vec<T>(r, src, s);
 }
 
 cudaError_t launch_vis_fused(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, const RotArgs &r,
