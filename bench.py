@@ -55,6 +55,26 @@ def parse_args():
 # ------------------------------------------------------------------ helpers
 
 
+def job_time_and_value(ms_local, units_per_rank, world, reduce_max=None):
+    """Step time of the job (max over ranks) and the whole-job throughput.
+
+    Every rank runs its own request (weak scaling): the job processes
+    world * units_per_rank units per step, in the time of the slowest rank.
+    reduce_max(x) returns the maximum of x over ranks (None: one rank)."""
+    ms = reduce_max(ms_local) if (reduce_max is not None and world > 1) else ms_local
+    return ms, world * units_per_rank / (ms / 1e3)
+
+
+def dist_max(value, device):
+    """Maximum of a float over the ranks of the default process group."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+
 def algorithmic_bytes_vision(v):
     """Interpolation bytes: table rows the samples touch, read once, plus the output."""
     import workloads as wl
@@ -332,11 +352,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        tt = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        return float(tt.item())
+        return x if world == 1 else dist_max(x, dev)
 
     props = torch.cuda.get_device_properties(dev)
     gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
@@ -359,8 +375,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     h1 = time.time()
-    ms_step = start.elapsed_time(end) / args.steps
-    ms_step = max_over_ranks(ms_step)
+    ms_step, value = job_time_and_value(start.elapsed_time(end) / args.steps, t.T, world, max_over_ranks)
     ipe.device_status(stream)          # raises if any kernel gave up a bounded wait
     kernel_ms = {n: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j, n in enumerate(names)}
     clocks = sampler.stop(h0, h1)
@@ -392,7 +407,6 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
 
-    value = world * t.T / (ms_step / 1e3)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -578,9 +592,9 @@ def end_to_end(ipe, torch, w, dev, stream, vin, tin, inv, steps, max_over_ranks,
     b.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = max_over_ranks(a.elapsed_time(b) / steps)
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    return {"value": world * t.T / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+    ms, value = job_time_and_value(a.elapsed_time(b) / steps, t.T, world, max_over_ranks)
+    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
             "ms_per_step": ms, "steps": steps}
 
 

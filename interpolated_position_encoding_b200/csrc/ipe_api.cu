@@ -9,7 +9,7 @@
 
 #include <cuda.h>   // CUresult / CUdeviceptr types only; the driver call is resolved at run time
 
-#include "../../include/ipe.h"
+#include "ipe.h"
 #include "ipe_internal.h"
 #include "ipe_rotary_tma.cuh"
 

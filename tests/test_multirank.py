@@ -1,0 +1,48 @@
+"""The multi-rank logic of bench.py on CPU: two gloo ranks, no GPU.
+
+The path shards without a data-path collective (every rank runs its own
+request); the only cross-rank steps are a barrier and the max-reduction of
+the step time, which sets the whole-job throughput.
+"""
+import os
+import socket
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, ms_by_rank, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    dist.barrier()
+    ms, value = bench.job_time_and_value(ms_by_rank[rank], 131072, world, lambda x: bench.dist_max(x, "cpu"))
+    dist.barrier()
+    out[rank] = (ms, value)
+    dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_slowest_rank():
+    world = 2
+    ms_by_rank = [0.40, 0.55]
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank, args=(world, _free_port(), ms_by_rank, out), nprocs=world, join=True)
+        res = dict(out)
+    for r in range(world):
+        ms, value = res[r]
+        assert ms == pytest.approx(0.55)
+        assert value == pytest.approx(world * 131072 / 0.55e-3)
+
+
+def test_single_rank_needs_no_group():
+    import bench
+    ms, value = bench.job_time_and_value(0.5, 1000, 1, None)
+    assert ms == 0.5 and value == pytest.approx(2e6)
