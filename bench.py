@@ -545,6 +545,12 @@ def per_workload(ipe, dev, stream, peak, reps):
                 r[f"apply_rotary_partial/{layout}"] = entry(_time_flushed(
                     torch, stream, lambda: ipe.apply_rotary_partial(Q, K, cos, sin, stream=stream), reps, flush),
                     rot + 2 * t.T * t.rot_dim * 4)
+                if layout == t.layouts[0]:
+                    wq = torch.ones(t.head_dim, dtype=torch.bfloat16, device=dev)
+                    full = (t.hq + t.hk) * t.T * t.head_dim * 2 * 2 + 3 * t.T * 4 + 2 * t.head_dim * 2
+                    r["qk_norm_mrope"] = entry(_time_flushed(
+                        torch, stream, lambda: ipe.qk_norm_mrope(Q, K, wq, wq, pos, inv, t.section, il, stream=stream),
+                        reps, flush), full)
             r["tokens"] = t.T
         res[name] = r
         torch.cuda.empty_cache()

@@ -175,6 +175,28 @@ int ipe_mrope_apply(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk
                     int interleaved, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * ipe_qk_norm_mrope -- RMSNorm of every head row of Q and K followed by the
+ * multimodal rotation of ipe_mrope_apply, in one pass, in place.
+ * [M01] problem summary and hints (rms_norm; the vllm-omni note on fusing it
+ * with the rotary); [IRPE] RoPE section ("projection and Q norm done" before
+ * the rotation):
+ *   xn = x * rsqrt(mean(x^2) + eps)      fp32, mean over the head_dim channels
+ *   y  = dtype(dtype(xn) * weight)       cast back to the dtype, then the weight
+ *   out = y rotated as ipe_mrope_apply (first rot_dim channels); channels
+ *         >= rot_dim are y.  All head_dim channels are written.
+ * q_weight / k_weight: device [head_dim], dtype (the q_norm / k_norm weights).
+ * head_dim: 16-byte chunks per row a power of two in 2 .. 32 (bf16: 16 .. 256,
+ * fp32: 8 .. 128); rot_dim / 2 a multiple of 8 (bf16) or 4 (fp32); q, k,
+ * weights and token strides 16-byte aligned (IPE_EALIGN otherwise).
+ * eps >= 0.  Other arguments as ipe_mrope_apply.
+ * ------------------------------------------------------------------------- */
+int ipe_qk_norm_mrope(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
+                      int64_t q_tok_stride, int64_t k_tok_stride, const void *q_weight,
+                      const void *k_weight, float eps, const int32_t *positions,
+                      const float *inv_freq_host, int rot_dim, const int32_t *section,
+                      int interleaved, void *stream);
+
+/* ---------------------------------------------------------------------------
  * Vision grids.  grid_thw_host is a host int32 [n_images, 3] array of
  * (t, h, w) patch grids BEFORE the spatial merge ([VLM] 1.1 Patch; [IRPE]
  * get_rope_index); h and w must be multiples of `merge` (spatial_merge_size,

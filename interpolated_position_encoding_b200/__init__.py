@@ -37,6 +37,8 @@ _SIGS = {
     "ipe_mrope_cos_sin": (_I, [_P, _I64, _P, _I, _P, _I, _P, _P, _P]),
     "ipe_apply_rotary_partial": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, _I, _P]),
     "ipe_mrope_apply": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, _I, _P, _I, _P]),
+    "ipe_qk_norm_mrope": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, ctypes.c_float, _P, _P, _I, _P, _I,
+                               _P]),
     "ipe_vis_interp_plan": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
     "ipe_vis_pos_interp": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P]),
     "ipe_vis_rope2d": (_I, [_P, _P, _I, _I64, _I, _I, _I64, _I64, _P, _I, _I, _D, _P]),
@@ -244,6 +246,25 @@ def mrope_apply(q, k, positions, inv_freq, section, interleaved=True, stream=Non
     return q, k
 
 
+def qk_norm_mrope(q, k, q_weight, k_weight, positions, inv_freq, section, interleaved=True, eps=1e-6, stream=None):
+    """In place: RMSNorm of every head row (cast back, then the weight) and the
+    fused multimodal rotation of its first 2 * len(inv_freq) channels."""
+    dt, T, hq, hk, D, qs, ks = _qk_args(q, k)
+    for w, nm in ((q_weight, "q_weight"), (k_weight, "k_weight")):
+        _cuda(w, nm)
+        ref = q if q is not None else k
+        if w.dtype != ref.dtype or tuple(w.shape) != (D,) or not w.is_contiguous():
+            raise ValueError(f"{nm} must be a contiguous [{D}] tensor of the activation dtype")
+    _cuda(positions, "positions")
+    if positions.dtype != torch.int32 or tuple(positions.shape) != (3, T) or not positions.is_contiguous():
+        raise ValueError("positions must be a contiguous int32 [3, T] tensor")
+    inv, half = _inv_host(inv_freq)
+    _check(_lib.ipe_qk_norm_mrope(_ptr(q), _ptr(k), dt, T, hq, hk, D, qs, ks, _ptr(q_weight), _ptr(k_weight),
+                                  float(eps), _ptr(positions), inv, 2 * half, _i32_host(section, 3),
+                                  int(bool(interleaved)), _stream(stream)))
+    return q, k
+
+
 # ------------------------------------------------------------------- vision
 
 
@@ -322,4 +343,4 @@ def vis_pos_interp_rope2d(table, grid_thw, q, k, merge=2, theta=1e4, out=None, s
 
 
 __all__ = ["IpeError", "lib", "EXPORTS", "device_status", "debug_inject", "rope_inv_freq", "mrope_axis_map", "mrope_cos_sin", "apply_rotary_partial",
-           "mrope_apply", "vis_interp_plan", "vis_pos_interp", "vis_rope2d", "vis_pos_interp_rope2d"]
+           "mrope_apply", "qk_norm_mrope", "vis_interp_plan", "vis_pos_interp", "vis_rope2d", "vis_pos_interp_rope2d"]

@@ -464,6 +464,49 @@ int ipe_mrope_apply(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk
     return e == cudaSuccess ? ok() : cuda_fail(e, "mrope_apply launch");
 }
 
+int ipe_qk_norm_mrope(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim, int64_t q_tok_stride,
+                      int64_t k_tok_stride, const void *q_weight, const void *k_weight, float eps,
+                      const int32_t *positions, const float *inv_freq_host, int rot_dim, const int32_t *section,
+                      int interleaved, void *stream)
+{
+    if (int rc = check_dtype(dtype)) return rc;
+    const int eb = elem_bytes(dtype), ec = 16 / eb;
+    if (head_dim <= 0 || head_dim % ec) return fail(IPE_EINVAL, "head_dim %d must be a multiple of %d", head_dim, ec);
+    const int lpr = head_dim / ec;
+    if (lpr < 2 || lpr > 32 || (lpr & (lpr - 1)))
+        return fail(IPE_ELIMIT, "head_dim %d: %d-element chunks per row must be a power of two in 2 .. 32", head_dim, ec);
+    if (rot_dim < 2 || rot_dim % 2 || rot_dim > head_dim)
+        return fail(IPE_EINVAL, "rot_dim %d must be even and in 2 .. head_dim", rot_dim);
+    if ((rot_dim / 2) % ec) return fail(IPE_EINVAL, "rot_dim / 2 = %d must be a multiple of %d", rot_dim / 2, ec);
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(IPE_EINVAL, "eps must be finite and >= 0");
+    MropeAngles a;
+    if (int rc = fill_mrope(a, positions, T, inv_freq_host, rot_dim / 2, section, interleaved)) return rc;
+    if (int rc = check_qk(q, k, dtype, T, hq, hk, head_dim, q_tok_stride, k_tok_stride, "q", "k")) return rc;
+    if ((hq && (q_tok_stride % ec || !aligned(q, 16))) || (hk && (k_tok_stride % ec || !aligned(k, 16))))
+        return fail(IPE_EALIGN, "q / k and their token strides must be 16-byte aligned");
+    if (!aligned(q_weight, 16) || !aligned(k_weight, 16)) return fail(IPE_EALIGN, "norm weights must be 16-byte aligned");
+    if (T == 0 || hq + hk == 0) return ok();
+    if (int rc = check_dev(q_weight, (size_t)head_dim * eb, "q_weight")) return rc;
+    if (int rc = check_dev(k_weight, (size_t)head_dim * eb, "k_weight")) return rc;
+    if (int rc = check_dev(positions, (size_t)(3 * T) * 4, "positions")) return rc;
+    QkNormArgs n{};
+    n.q = hq ? q : nullptr;
+    n.k = hk ? k : nullptr;
+    n.q_weight = q_weight;
+    n.k_weight = k_weight;
+    n.T = T;
+    n.q_stride = q_tok_stride;
+    n.k_stride = k_tok_stride;
+    n.hq = hq;
+    n.hk = hk;
+    n.head_dim = head_dim;
+    n.half = rot_dim / 2;
+    n.half_pad = (n.half + 3) & ~3;
+    n.eps = eps;
+    cudaError_t e = launch_qk_norm_mrope(dtype == IPE_BF16, n, a, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "qk_norm_mrope launch");
+}
+
 int ipe_vis_interp_plan(const int32_t *grid_thw_host, int n_images, int merge, int grid_side, int32_t *idx4,
                         float *w4, int32_t *rowcol, void *stream)
 {

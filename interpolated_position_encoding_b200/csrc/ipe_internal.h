@@ -98,6 +98,18 @@ struct TmaRotArgs {
     unsigned *status;        // fault word (ipe_device_status)
 };
 
+// ----------------------------------------------- fused QK-RMSNorm + MRoPE
+struct QkNormArgs {
+    void *q, *k;                      // [T, hq, D], [T, hk, D], rewritten in place
+    const void *q_weight, *k_weight;  // [D] norm weights, activation dtype
+    long long T;
+    long long q_stride, k_stride;
+    int hq, hk, head_dim, half, half_pad;
+    float eps;
+};
+
+cudaError_t launch_qk_norm_mrope(bool bf16, const QkNormArgs &n, const MropeAngles &a, cudaStream_t s);
+
 // Test hooks and the device status word (ipe_api.cu).
 unsigned *device_status_word();
 long long debug_skip_tile();

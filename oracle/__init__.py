@@ -44,6 +44,7 @@ class Oracle:
             "orc_vis_interp_plan": (_I, [_P, _I, _I, _I, _P, _P]),
             "orc_vis_rot_pos_ids": (_I, [_P, _I, _I, _P]),
             "orc_vis_rotary_cos_sin": (_I, [_P, _I64, _I, _D, _P, _P]),
+            "orc_rms_norm": (_I, [_P, _I64, _I, _P, _D, _I, _P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -106,6 +107,25 @@ class Oracle:
     def mrope_apply(self, x, positions, inv_freq, section, interleaved, with_mag=False):
         cos, sin = self.mrope_cos_sin(positions, inv_freq, section, interleaved)
         return self.apply_rotary(x, cos, sin, with_mag)
+
+    def rms_norm(self, x, weight, eps, dtype):
+        """RMSNorm over the last axis: x [..., D] -> rounded to `dtype` ("f32" | "bf16")."""
+        x = np.ascontiguousarray(x, np.float64)
+        w = np.ascontiguousarray(weight, np.float64)
+        D = x.shape[-1]
+        assert w.shape == (D,)
+        out = np.zeros_like(x)
+        R = x.size // D
+        if self._lib.orc_rms_norm(_ptr(x), R, D, _ptr(w), float(eps), {"f32": 0, "bf16": 1}[dtype], _ptr(out)):
+            raise ValueError("rms_norm: bad arguments")
+        return out
+
+    def qk_norm_mrope(self, x, weight, eps, dtype, positions, inv_freq, section, interleaved, with_mag=False):
+        """RMSNorm of every head row, then the multimodal rotation of its first
+        2 * len(inv_freq) channels (x: [T, H, D])."""
+        y = self.rms_norm(x, weight, eps, dtype)
+        out = self.mrope_apply(y, positions, inv_freq, section, interleaved, with_mag)
+        return (out[0], out[1], y) if with_mag else (out, y)
 
     # -------------------------------------------------------------- vision
     def grid_patches(self, grid_thw, merge):

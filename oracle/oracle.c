@@ -453,3 +453,50 @@ int orc_vis_rotary_cos_sin(const int64_t *pos_ids, int64_t N, int head_dim, doub
     free(inv);
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * RMSNorm over the last axis, in the order the drill page fixes.
+ * [M01] problem summary and L2 hints (rms_norm):
+ *   x32 = float(x); xn = x32 * rsqrt(mean(x32^2, -1, keepdim) + eps)
+ *   y = xn.to(x.dtype) * weight            (cast back first, then the weight)
+ * Reading: mean, rsqrt and the product are taken in double; the two casts are
+ * the dtype's own rounding (dtype 0: fp32, 1: bf16, round to nearest even),
+ * the second applied to the exact product of the two rounded values.
+ * x, out: [R][D]; weight: [D] (values of the weight's dtype).
+ * ---------------------------------------------------------------------- */
+static double round_to(double v, int dtype)
+{
+    if (dtype == 0)
+        return (double)(float)v;
+    /* bf16: round the fp32-representable value v to 8 significant bits, ties
+     * to even, through its fp32 bit pattern (v is first rounded to fp32, as
+     * the dtype conversion of a fp32 tensor does) */
+    float f = (float)v;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u)
+        return (double)f;
+    uint32_t r = u + 0x7fffu + ((u >> 16) & 1u);
+    r &= 0xffff0000u;
+    float g;
+    memcpy(&g, &r, sizeof g);
+    return (double)g;
+}
+
+int orc_rms_norm(const double *x, int64_t R, int D, const double *weight, double eps, int dtype, double *out)
+{
+    if (R < 0 || D <= 0 || (dtype != 0 && dtype != 1) || eps < 0)
+        return -1;
+    for (int64_t r = 0; r < R; ++r) {
+        const double *xr = x + r * D;
+        double ss = 0.0;
+        for (int d = 0; d < D; ++d)
+            ss += xr[d] * xr[d];
+        double inv = 1.0 / sqrt(ss / D + eps);
+        for (int d = 0; d < D; ++d) {
+            double xn = round_to(xr[d] * inv, dtype);            /* .to(x.dtype) */
+            out[r * D + d] = round_to(xn * weight[d], dtype);    /* * weight */
+        }
+    }
+    return 0;
+}

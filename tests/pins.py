@@ -185,6 +185,29 @@ def pin_vision_tokens_per_axis(o):
     assert np.array_equal(cos[0, 32:], cos[0, :32])
 
 
+def pin_rms_norm_golden(o):
+    g = {k[0]: np.array([float(v) for v in vals]) for k, vals in golden("rms_norm.txt")}
+    out = o.rms_norm(g["x"].reshape(2, 2), g["weight"], 0.0, "f32")
+    assert np.array_equal(np.round(out.reshape(-1), 4), g["out"]), out
+
+
+def pin_rms_norm_closed_forms(o):
+    # eps sits inside the square root: x = [1, 1], eps = 3 -> 1 / sqrt(1 + 3) = 0.5
+    out = o.rms_norm(np.array([[1.0, 1.0]]), np.array([1.0, 3.0]), 3.0, "f32")
+    assert np.array_equal(out, [[0.5, 1.5]])
+    # a zero row with eps > 0 stays zero; with unit weight the row RMS is 1
+    assert not o.rms_norm(np.zeros((1, 8)), np.ones(8), 1e-6, "f32").any()
+    rng = _rng(17)
+    x = rng.standard_normal((16, 64))
+    y = o.rms_norm(x, np.ones(64), 0.0, "f32")
+    assert np.allclose(np.sqrt((y ** 2).mean(-1)), 1.0, rtol=0, atol=2e-7)
+    # scale invariance, and the bf16 result is bf16-representable
+    y2 = o.rms_norm(7.25 * x, np.ones(64), 0.0, "f32")
+    assert np.allclose(y, y2, rtol=2 ** -22, atol=0)
+    yb = o.rms_norm(x, np.full(64, 1.5), 1e-6, "bf16").astype(np.float32)
+    assert not (yb.view(np.uint32) & 0xFFFF).any()
+
+
 # ------------------------------------------------------------------- vision
 
 

@@ -54,6 +54,10 @@ MUTANTS = {
     # vision exponent 2i / head_dim instead of 2i / (head_dim / 2): the same
     # 18 values as base sqrt(theta) over dim (written so, to stay in bounds)
     "vision_inv_dim": ("orc_rope_inv_freq(dim, theta, inv);", "orc_rope_inv_freq(dim, sqrt(theta), inv);"),
+    # RMSNorm: eps added after the square root
+    "rms_eps_outside": ("double inv = 1.0 / sqrt(ss / D + eps);", "double inv = 1.0 / (sqrt(ss / D) + eps);"),
+    # RMSNorm: sum of squares instead of the mean
+    "rms_sum_not_mean": ("double inv = 1.0 / sqrt(ss / D + eps);", "double inv = 1.0 / sqrt(ss + eps);"),
 }
 
 
