@@ -12,12 +12,18 @@
 // (EC elements = 16 bytes per lane), its sum of squares reduced with
 // shuffles inside those lanes, and the rotary partner of a chunk fetched from
 // the lane half a rotary slice away.  All D channels are written back.
-#include "ipe_rotary.cuh"
+#include "ipe_rotary_tma.cuh"
 
 namespace ipe {
 
+#ifndef IPE_QK_UNROLL
+#define IPE_QK_UNROLL 4
+#endif
+#ifndef IPE_QK_MIN_BLOCKS
+#define IPE_QK_MIN_BLOCKS 3
+#endif
 constexpr int kQkWarps = 8;
-constexpr int kQkUnroll = 2;          // head rows per lane in flight
+constexpr int kQkUnroll = IPE_QK_UNROLL;     // head rows per lane in flight
 
 template <typename T> struct QkElem;
 template <> struct QkElem<__nv_bfloat16> {
@@ -27,15 +33,53 @@ template <> struct QkElem<float> {
     static constexpr int EC = 4;
 };
 
-// Round to the activation dtype (identity for fp32).
-__device__ __forceinline__ float round_dtype(float v, __nv_bfloat16 *) { return __bfloat162float(__float2bfloat16_rn(v)); }
-__device__ __forceinline__ float round_dtype(float v, float *) { return v; }
+// A 16-byte chunk (4 words) as EC/2 fp32 pairs, and back (one rounding to
+// the dtype per element).
+template <typename T> __device__ __forceinline__ void chunk_to_pairs(const uint32_t *w, float2 *p);
+template <> __device__ __forceinline__ void chunk_to_pairs<__nv_bfloat16>(const uint32_t *w, float2 *p)
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+}
+template <> __device__ __forceinline__ void chunk_to_pairs<float>(const uint32_t *w, float2 *p)
+{
+#pragma unroll
+    for (int i = 0; i < 2; ++i) p[i] = make_float2(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]));
+}
+template <typename T> __device__ __forceinline__ void pairs_to_chunk(const float2 *p, uint32_t *w);
+template <> __device__ __forceinline__ void pairs_to_chunk<__nv_bfloat16>(const float2 *p, uint32_t *w)
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(p[i].x, p[i].y);
+        w[i] = *reinterpret_cast<const uint32_t *>(&b);
+    }
+}
+template <> __device__ __forceinline__ void pairs_to_chunk<float>(const float2 *p, uint32_t *w)
+{
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        w[2 * i] = __float_as_uint(p[i].x);
+        w[2 * i + 1] = __float_as_uint(p[i].y);
+    }
+}
+
+// Product of two bf16 pairs rounded once to bf16 (the exact product of two
+// bf16 values fits in fp32, so this equals rounding the fp32 product).
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
 
 template <typename T, int LPR>
-__global__ void __launch_bounds__(32 * kQkWarps) qk_norm_mrope_kernel(const __grid_constant__ QkNormArgs n,
-                                                                      const __grid_constant__ MropeAngles a)
+__global__ void __launch_bounds__(32 * kQkWarps, IPE_QK_MIN_BLOCKS)
+    qk_norm_mrope_kernel(const __grid_constant__ QkNormArgs n, const __grid_constant__ MropeAngles a)
 {
+    constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr int EC = QkElem<T>::EC;
+    constexpr int NP = EC / 2;                        // fp32 pairs of a 16-byte chunk
     constexpr int RPW = 32 / LPR;                     // head rows per warp access
     extern __shared__ float4 qk_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -48,22 +92,38 @@ __global__ void __launch_bounds__(32 * kQkWarps) qk_norm_mrope_kernel(const __gr
     const bool rotary = e0 < rot;
     const bool first_half = e0 < half;
     const int j0 = first_half ? e0 : e0 - half;       // frequency of element e0
-    const int partner = first_half ? lane + half / EC : lane - half / EC;
+    const int partner = rotary ? (first_half ? lane + half / EC : lane - half / EC) : lane;
+    // D = LPR * EC is a power of two: multiplying by 1/D is the exact division
+    const float inv_d = __frcp_rn((float)D);
 
-    // norm weights of this chunk, as fp32
-    float wq[EC], wk[EC];
-    {
-        const Pack<T, EC> pq = ld_pack<T, EC>(static_cast<const T *>(n.q_weight) + e0);
-        const Pack<T, EC> pk = ld_pack<T, EC>(static_cast<const T *>(n.k_weight) + e0);
-#pragma unroll
-        for (int e = 0; e < EC; ++e) {
-            wq[e] = to_f32(pq.v[e]);
-            wk[e] = to_f32(pk.v[e]);
-        }
-    }
+    // norm weights of this chunk, as words
+    const Pack<uint32_t, 4> wq = ld_pack<uint32_t, 4>(reinterpret_cast<const uint32_t *>(static_cast<const T *>(n.q_weight) + e0));
+    const Pack<uint32_t, 4> wk = ld_pack<uint32_t, 4>(reinterpret_cast<const uint32_t *>(static_cast<const T *>(n.k_weight) + e0));
     const int H = n.hq + n.hk;
     const long long stride = (long long)gridDim.x * kQkWarps;
     for (long long t = (long long)blockIdx.x * kQkWarps + warp; t < n.T; t += stride) {
+        Pack<uint32_t, 4> x[kQkUnroll];
+        // this lane's chunk of head row h of token t
+        auto chunk_ptr = [&](int h) {
+            T *row = h < n.hq ? static_cast<T *>(n.q) + t * n.q_stride + (long long)h * D
+                              : static_cast<T *>(n.k) + t * n.k_stride + (long long)(h - n.hq) * D;
+            return reinterpret_cast<uint32_t *>(row + e0);
+        };
+        // rows h0 + u * RPW + sub of token t (zeros past the last head)
+        auto load_group = [&](int h0) {
+#pragma unroll
+            for (int u = 0; u < kQkUnroll; ++u) {
+                const int h = h0 + u * RPW + sub;
+                if (h < H) {
+                    x[u] = ld_pack<uint32_t, 4>(chunk_ptr(h));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) x[u].v[i] = 0u;
+                }
+            }
+        };
+        // the first rows are in flight while the angles are computed
+        load_group(0);
         // (cos, sin) of every frequency of token t
         for (int j = lane; j < half; j += 32) {
             const int ax = mrope_axis(j, a.section, a.interleaved);
@@ -72,63 +132,57 @@ __global__ void __launch_bounds__(32 * kQkWarps) qk_norm_mrope_kernel(const __gr
             sincosf(angle, &cs_s[j], &cs_c[j]);
         }
         __syncwarp();
-        float co[EC], si[EC];
-        if (rotary) {
+        // cos and the signed sine of this chunk (pass-through: 1 and 0)
+        float2 co[NP], si[NP];
 #pragma unroll
-            for (int e = 0; e < EC; ++e) {
-                co[e] = cs_c[j0 + e];
-                si[e] = cs_s[j0 + e];
-            }
+        for (int i = 0; i < NP; ++i) {
+            co[i] = rotary ? make_float2(cs_c[j0 + 2 * i], cs_c[j0 + 2 * i + 1]) : make_float2(1.f, 1.f);
+            const float2 sv = rotary ? make_float2(cs_s[j0 + 2 * i], cs_s[j0 + 2 * i + 1]) : make_float2(0.f, 0.f);
+            si[i] = first_half ? make_float2(-sv.x, -sv.y) : sv;
         }
         for (int h0 = 0; h0 < H; h0 += RPW * kQkUnroll) {
-            Pack<T, EC> x[kQkUnroll];
-            T *ptr[kQkUnroll];
+            if (h0 > 0) load_group(h0);
 #pragma unroll
             for (int u = 0; u < kQkUnroll; ++u) {
+                // every lane of the warp takes part in the shuffles, rows past
+                // H included (zeros; never stored)
                 const int h = h0 + u * RPW + sub;
-                ptr[u] = nullptr;
-                if (h < H) {
-                    ptr[u] = (h < n.hq ? static_cast<T *>(n.q) + t * n.q_stride + (long long)h * D
-                                       : static_cast<T *>(n.k) + t * n.k_stride + (long long)(h - n.hq) * D) + e0;
-                    x[u] = ld_pack<T, EC>(ptr[u]);
-                }
-            }
+                float2 xv[NP];
+                chunk_to_pairs<T>(x[u].v, xv);
+                float2 acc = mul2(xv[0], xv[0]);
 #pragma unroll
-            for (int u = 0; u < kQkUnroll; ++u) {
-                const int h = h0 + u * RPW + sub;
-                // rows of one warp access are uniform in (h < H) per RPW group;
-                // the shuffles below stay inside each row's LPR lanes
-                float xf[EC];
-                float ss = 0.f;
-#pragma unroll
-                for (int e = 0; e < EC; ++e) {
-                    xf[e] = h < H ? to_f32(x[u].v[e]) : 0.f;
-                    ss = __fmaf_rn(xf[e], xf[e], ss);
-                }
+                for (int i = 1; i < NP; ++i) acc = fma2(xv[i], xv[i], acc);
+                float ss = __fadd_rn(acc.x, acc.y);
 #pragma unroll
                 for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off, LPR);
-                const float r = __frsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)D), n.eps));
+                const float r = __frsqrt_rn(__fadd_rn(__fmul_rn(ss, inv_d), n.eps));
                 const bool is_q = h < n.hq;
-                float y[EC];
+                // y = dtype(dtype(x r) * w): cast back first, then the weight
+                const float2 r2 = make_float2(r, r);
 #pragma unroll
-                for (int e = 0; e < EC; ++e) {
-                    // cast back to the dtype first, then the weight (one more rounding)
-                    const float xn = round_dtype(__fmul_rn(xf[e], r), (T *)nullptr);
-                    y[e] = round_dtype(__fmul_rn(xn, is_q ? wq[e] : wk[e]), (T *)nullptr);
+                for (int i = 0; i < NP; ++i) xv[i] = mul2(xv[i], r2);
+                Pack<uint32_t, 4> y;
+                pairs_to_chunk<T>(xv, y.v);
+                if constexpr (BF16) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) y.v[i] = mul_bf16x2(y.v[i], is_q ? wq.v[i] : wk.v[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        y.v[i] = __float_as_uint(__fmul_rn(__uint_as_float(y.v[i]), __uint_as_float(is_q ? wq.v[i] : wk.v[i])));
                 }
-                float yp[EC];
+                Pack<uint32_t, 4> yp;
 #pragma unroll
-                for (int e = 0; e < EC; ++e) yp[e] = __shfl_sync(0xffffffffu, y[e], rotary ? partner : lane);
-                Pack<T, EC> o;
+                for (int i = 0; i < 4; ++i) yp.v[i] = __shfl_sync(0xffffffffu, y.v[i], partner);
+                // y[j] cos - y[j+h] sin ; y[j+h] cos + y[j] sin, the sign in si
+                float2 yv[NP], pv[NP];
+                chunk_to_pairs<T>(y.v, yv);
+                chunk_to_pairs<T>(yp.v, pv);
 #pragma unroll
-                for (int e = 0; e < EC; ++e) {
-                    float v = y[e];
-                    if (rotary)   // x[j] cos - x[j+h] sin ; x[j+h] cos + x[j] sin
-                        v = first_half ? __fmaf_rn(y[e], co[e], -__fmul_rn(yp[e], si[e]))
-                                       : __fmaf_rn(y[e], co[e], __fmul_rn(yp[e], si[e]));
-                    o.v[e] = from_f32<T>(v);
-                }
-                if (ptr[u]) st_pack<T, EC>(ptr[u], o);
+                for (int i = 0; i < NP; ++i) yv[i] = fma2(yv[i], co[i], mul2(pv[i], si[i]));
+                Pack<uint32_t, 4> o;
+                pairs_to_chunk<T>(yv, o.v);
+                if (h < H) st_pack<uint32_t, 4>(chunk_ptr(h), o);
             }
         }
         __syncwarp();
