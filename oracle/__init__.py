@@ -45,6 +45,7 @@ class Oracle:
             "orc_vis_rot_pos_ids": (_I, [_P, _I, _I, _P]),
             "orc_vis_rotary_cos_sin": (_I, [_P, _I64, _I, _D, _P, _P]),
             "orc_rms_norm": (_I, [_P, _I64, _I, _P, _D, _I, _P]),
+            "orc_rope_index": (_I, [_P, _P, _I, _I64, _P, _I, _P, _I, _I, _P, _P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -126,6 +127,28 @@ class Oracle:
         y = self.rms_norm(x, weight, eps, dtype)
         out = self.mrope_apply(y, positions, inv_freq, section, interleaved, with_mag)
         return (out[0], out[1], y) if with_mag else (out, y)
+
+    def rope_index(self, types, mask, image_grid_thw, video_grid_thw, merge):
+        """(position_ids [3, B, L], rope_deltas [B]) of a batch of mixed
+        sequences (types [B, L]; mask [B, L] or None; grids [n, 3] or None)."""
+        ty = np.ascontiguousarray(types, np.int64)
+        assert ty.ndim == 2
+        B, L = ty.shape
+        mk = None if mask is None else np.ascontiguousarray(mask, np.int64)
+        assert mk is None or mk.shape == ty.shape
+        ig = np.ascontiguousarray(np.zeros((0, 3)) if image_grid_thw is None else image_grid_thw, np.int64).reshape(-1, 3)
+        vg = np.ascontiguousarray(np.zeros((0, 3)) if video_grid_thw is None else video_grid_thw, np.int64).reshape(-1, 3)
+        pos = np.zeros((3, B, L), np.int64)
+        deltas = np.zeros(B, np.int64)
+        rc = self._lib.orc_rope_index(_ptr(ty), None if mk is None else _ptr(mk), B, L, _ptr(ig), ig.shape[0],
+                                      _ptr(vg), vg.shape[0], int(merge), _ptr(pos), _ptr(deltas))
+        if rc == -2:
+            raise ValueError("rope_index: a vision run found its grid iterator exhausted")
+        if rc == -3:
+            raise ValueError("rope_index: the joined table does not have one column per kept slot")
+        if rc:
+            raise ValueError("rope_index: bad arguments")
+        return pos, deltas
 
     # -------------------------------------------------------------- vision
     def grid_patches(self, grid_thw, merge):

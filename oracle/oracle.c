@@ -500,3 +500,151 @@ int orc_rms_norm(const double *x, int64_t R, int D, const double *weight, double
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Three-axis position table of a batch of mixed sequences, and the per-sample
+ * rope deltas.
+ * [IRPE] get_rope_index(): preparing the grids, filtering padding and
+ * splitting runs, advancing the position, flattening the vision grid,
+ * joining the sequence back, returning positions and deltas; and the worked
+ * single-batch table.  [IRPE] mm_tokens gives the type codes: 0 text (and
+ * message / media start-end markers), 1 image, 2 video, 3 audio.
+ *
+ * Steps, in the page's order:
+ *  1. every video grid row (t, h, w) becomes t rows (1, h, w), one per
+ *     temporal slice; image rows are used as they are;
+ *  2. one image iterator and one video iterator serve the whole batch, in
+ *     the order of samples and of appearance within a sample;
+ *  3. per sample: keep the slots whose mask is non-zero, split the kept
+ *     type sequence into runs of equal consecutive type;
+ *  4. current_pos starts at 0; a text run of n slots gets arange(n) +
+ *     current_pos on all three rows and advances current_pos by n; a vision
+ *     run takes the next grid of its kind, lays out llm_t = t, llm_h = h / m,
+ *     llm_w = w / m slots width-fastest with coordinates
+ *     (current_pos + tt, current_pos + row, current_pos + col) and advances
+ *     current_pos by max(h, w) / m (not by its slot count);
+ *  5. the runs are joined and written back to the kept slots; padded slots
+ *     stay 0; the delta is max(joined) + 1 - (number of kept slots).
+ * Readings: an audio run (type 3) is laid out like text -- the page on the
+ * Omni drills states that audio positions advance linearly in time, and the
+ * listing has no grid for it.  A sample with no kept slot gets delta 0 (the
+ * listing would take the maximum of an empty table).
+ *
+ * types, mask: [B][L] (mask may be NULL: every slot kept); img_grid: [n_img][3];
+ * vid_grid: [n_vid][3]; pos: [3][B][L]; deltas: [B].
+ * Returns 0; -1 on bad arguments; -2 when a vision run finds its iterator
+ * exhausted; -3 when the joined table of a sample does not have one column
+ * per kept slot.
+ * ---------------------------------------------------------------------- */
+int orc_rope_index(const int64_t *types, const int64_t *mask, int B, int64_t L, const int64_t *img_grid,
+                   int n_img, const int64_t *vid_grid, int n_vid, int m, int64_t *pos, int64_t *deltas)
+{
+    if (B < 0 || L < 0 || n_img < 0 || n_vid < 0 || m <= 0)
+        return -1;
+    /* 1. video grids repeated per temporal slice, t set to 1 */
+    int64_t n_slices = 0;
+    for (int v = 0; v < n_vid; ++v) {
+        if (vid_grid[3 * v] < 0)
+            return -1;
+        n_slices += vid_grid[3 * v];
+    }
+    int64_t *slices = malloc(sizeof(int64_t) * 3 * (size_t)(n_slices > 0 ? n_slices : 1));
+    int64_t *kept = malloc(sizeof(int64_t) * (size_t)(L > 0 ? L : 1));
+    int64_t *table = malloc(sizeof(int64_t) * 3 * (size_t)(L > 0 ? L : 1));
+    if (!slices || !kept || !table) {
+        free(slices);
+        free(kept);
+        free(table);
+        return -1;
+    }
+    int64_t s = 0;
+    for (int v = 0; v < n_vid; ++v)
+        for (int64_t r = 0; r < vid_grid[3 * v]; ++r, ++s) {
+            slices[3 * s] = 1;
+            slices[3 * s + 1] = vid_grid[3 * v + 1];
+            slices[3 * s + 2] = vid_grid[3 * v + 2];
+        }
+    for (int64_t i = 0; i < 3 * (int64_t)B * L; ++i)
+        pos[i] = 0;
+    /* 2. iterators shared by the batch */
+    int64_t next_img = 0, next_vid = 0;
+    int rc = 0;
+    for (int b = 0; b < B && rc == 0; ++b) {
+        /* 3. kept slots (their indices into the padded row) */
+        int64_t n = 0;
+        for (int64_t l = 0; l < L; ++l)
+            if (mask == NULL || mask[(int64_t)b * L + l] != 0)
+                kept[n++] = l;
+        /* 4. runs of equal type over the kept sequence, current_pos from 0 */
+        int64_t cur = 0, cols = 0;
+        int64_t start = 0;
+        while (start < n && rc == 0) {
+            int64_t key = types[(int64_t)b * L + kept[start]];
+            int64_t end = start + 1;
+            while (end < n && types[(int64_t)b * L + kept[end]] == key)
+                ++end;
+            if (key == 0 || key == 3) {
+                int64_t text_len = end - start;
+                for (int64_t i = 0; i < text_len; ++i) {
+                    if (cols >= n) {
+                        rc = -3;
+                        break;
+                    }
+                    for (int a = 0; a < 3; ++a)
+                        table[a * n + cols] = i + cur;
+                    ++cols;
+                }
+                cur += text_len;
+            } else if (key == 1 || key == 2) {
+                const int64_t *g;
+                if (key == 1) {
+                    if (next_img >= n_img) {
+                        rc = -2;
+                        break;
+                    }
+                    g = img_grid + 3 * next_img++;
+                } else {
+                    if (next_vid >= n_slices) {
+                        rc = -2;
+                        break;
+                    }
+                    g = slices + 3 * next_vid++;
+                }
+                int64_t lt = g[0], lh = g[1] / m, lw = g[2] / m;
+                for (int64_t tt = 0; tt < lt; ++tt)
+                    for (int64_t hh = 0; hh < lh; ++hh)
+                        for (int64_t ww = 0; ww < lw; ++ww) {
+                            if (cols >= n) {
+                                rc = -3;
+                                break;
+                            }
+                            table[0 * n + cols] = tt * 1 + cur;   /* time_interval 1 */
+                            table[1 * n + cols] = hh + cur;
+                            table[2 * n + cols] = ww + cur;
+                            ++cols;
+                        }
+                cur += (g[1] > g[2] ? g[1] : g[2]) / m;
+            } else {
+                rc = -1;
+            }
+            start = end;
+        }
+        if (rc == 0 && cols != n)
+            rc = -3;
+        if (rc != 0)
+            break;
+        /* 5. write back to kept slots; delta from the joined table */
+        int64_t mx = 0;
+        for (int64_t c = 0; c < n; ++c)
+            for (int a = 0; a < 3; ++a) {
+                pos[((int64_t)a * B + b) * L + kept[c]] = table[a * n + c];
+                if ((c == 0 && a == 0) || table[a * n + c] > mx)
+                    mx = table[a * n + c];
+            }
+        deltas[b] = n > 0 ? mx + 1 - n : 0;
+    }
+    free(slices);
+    free(kept);
+    free(table);
+    return rc;
+}

@@ -343,4 +343,130 @@ def pin_vision_rotation_complex(o):
     assert np.allclose(out[:, :, 36:], z.imag, rtol=0, atol=1e-12)
 
 
+# -------------------------------------------------------- position table
+
+
+def _l10_example():
+    # t0, S, six merged slots of a [1, 4, 6] image (m = 2), E, t1
+    return [0, 0, 1, 1, 1, 1, 1, 1, 0, 0], [[1, 4, 6]]
+
+
+def pin_rope_index_golden(o):
+    want = {k[0]: [int(v) for v in vals] for k, vals in golden("positions_l10.txt")}
+    types, grids = _l10_example()
+    pos, deltas = o.rope_index([types], None, grids, None, 2)
+    for a, key in enumerate("THW"):
+        assert pos[a, 0].tolist() == want[key], key
+    # the next rotary position (7) minus the 10 kept slots
+    assert deltas.tolist() == [-3]
+
+
+def pin_rope_index_padding(o):
+    # Padded slots (mask 0) are dropped before the runs are formed and keep
+    # position 0; a masked slot inside the image run does not split it.
+    types, grids = _l10_example()
+    want, wd = o.rope_index([types], None, grids, None, 2)
+    for left, right in [(3, 0), (0, 4), (2, 2)]:
+        L = left + len(types) + right
+        ty = [0] * left + types + [2] * right
+        mk = [0] * left + [1] * len(types) + [0] * right
+        pos, deltas = o.rope_index([ty], [mk], grids, None, 2)
+        assert (pos[:, 0, left:left + len(types)] == want[:, 0]).all()
+        assert not pos[:, 0, :left].any() and not pos[:, 0, left + len(types):].any()
+        assert deltas.tolist() == wd.tolist() and pos.shape == (3, 1, L)
+    ty = types[:5] + [0] + types[5:]
+    mk = [1] * 5 + [0] + [1] * 5
+    pos, _ = o.rope_index([ty], [mk], grids, None, 2)
+    assert (np.delete(pos[:, 0], 5, axis=1) == want[:, 0]).all() and not pos[:, 0, 5].any()
+
+
+def _random_batch(rng, B, merge=2):
+    """Types, mask and grids of B mixed sequences: text, images, video slices
+    each behind a timestamp token, audio; random left or right padding."""
+    seqs, img, vid = [], [], []
+    for _ in range(B):
+        ty = []
+        for _ in range(rng.integers(1, 6)):
+            ty += [0] * int(rng.integers(1, 4))
+            kind = rng.integers(0, 4)
+            if kind == 1:
+                t, h, w = int(rng.integers(1, 3)), 2 * int(rng.integers(1, 5)), 2 * int(rng.integers(1, 5))
+                img.append([t, h, w])
+                ty += [1] * (t * (h // merge) * (w // merge))
+            elif kind == 2:
+                t, h, w = int(rng.integers(1, 4)), 2 * int(rng.integers(1, 5)), 2 * int(rng.integers(1, 5))
+                vid.append([t, h, w])
+                for _ in range(t):
+                    ty += [0] * int(rng.integers(1, 3)) + [2] * ((h // merge) * (w // merge))
+            elif kind == 3:
+                ty += [3] * int(rng.integers(1, 5))
+        seqs.append(ty)
+    L = max(len(t) for t in seqs) + 3
+    types = np.zeros((B, L), np.int64)
+    mask = np.zeros((B, L), np.int64)
+    for b, ty in enumerate(seqs):
+        off = int(rng.integers(0, L - len(ty) + 1))
+        types[b, off:off + len(ty)] = ty
+        types[b, :off] = rng.integers(0, 3, off)
+        mask[b, off:off + len(ty)] = 1
+    return types, mask, np.array(img, np.int64).reshape(-1, 3), np.array(vid, np.int64).reshape(-1, 3)
+
+
+def _rope_index_prefix_form(types, mask, img, vid, m):
+    """The same table from running counts instead of runs: a text slot sits
+    at (kept text slots before it) + (advances of the vision runs before it);
+    a vision run starts there and lays its grid out width-fastest."""
+    slices = [(1, h, w) for t, h, w in vid for _ in range(t)]
+    grids = {1: iter([tuple(g) for g in img]), 2: iter(slices)}
+    B, L = types.shape
+    pos = np.zeros((3, B, L), np.int64)
+    deltas = np.zeros(B, np.int64)
+    for b in range(B):
+        text_before, vision_adv, prev, hi, n = 0, 0, None, None, 0
+        for l in range(L):
+            if not mask[b, l]:
+                continue
+            ty = int(types[b, l])
+            if ty in (0, 3):
+                pos[:, b, l] = text_before + vision_adv
+                text_before += 1
+            else:
+                if ty != prev:
+                    t, h, w = next(grids[ty])
+                    start, off, gh, gw = text_before + vision_adv, 0, h // m, w // m
+                    vision_adv += max(h, w) // m
+                tt, rem = divmod(off, gh * gw)
+                pos[:, b, l] = (start + tt, start + rem // gw, start + rem % gw)
+                off += 1
+            prev = ty
+            n += 1
+            hi = pos[:, b, l].max() if hi is None else max(hi, pos[:, b, l].max())
+        deltas[b] = 0 if n == 0 else hi + 1 - n
+    return pos, deltas
+
+
+def pin_rope_index_prefix_form(o):
+    rng = _rng(17)
+    for B in (1, 3, 6):
+        types, mask, img, vid = _random_batch(rng, B)
+        pos, deltas = o.rope_index(types, mask, img, vid, 2)
+        want, wd = _rope_index_prefix_form(types, mask, img, vid, 2)
+        assert (pos == want).all() and (deltas == wd).all()
+    # text only: arange on all three rows, delta 0
+    pos, deltas = o.rope_index(np.zeros((2, 7), np.int64), None, None, None, 2)
+    assert (pos == np.arange(7)[None, None, :]).all() and not deltas.any()
+
+
+def pin_rope_index_errors(o):
+    types, grids = _l10_example()
+    for args in [([types], None, None, None, 2),                      # no image grid left
+                 ([types], None, [[1, 4, 4]], None, 2),               # 4 slots for a 6-slot run
+                 ([[0, 2, 2, 0, 2, 2]], None, None, [[1, 2, 4]], 2)]:  # one slice, two runs
+        try:
+            o.rope_index(*args)
+        except ValueError:
+            continue
+        raise AssertionError(f"accepted {args}")
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -58,6 +58,20 @@ MUTANTS = {
     "rms_eps_outside": ("double inv = 1.0 / sqrt(ss / D + eps);", "double inv = 1.0 / (sqrt(ss / D) + eps);"),
     # RMSNorm: sum of squares instead of the mean
     "rms_sum_not_mean": ("double inv = 1.0 / sqrt(ss / D + eps);", "double inv = 1.0 / sqrt(ss + eps);"),
+    # position table: a vision run advances by its slot count instead of its longer side
+    "rope_advance_slots": ("cur += (g[1] > g[2] ? g[1] : g[2]) / m;", "cur += lt * lh * lw;"),
+    # position table: padding kept (the mask ignored)
+    "rope_mask_ignored": ("if (mask == NULL || mask[(int64_t)b * L + l] != 0)", "if (1)"),
+    # position table: video grids not split into temporal slices
+    "rope_video_slices": ("slices[3 * s] = 1;", "slices[3 * s] = vid_grid[3 * v];"),
+    # position table: one image iterator per sample instead of per batch
+    "rope_iter_per_sample": ("int64_t cur = 0, cols = 0;", "int64_t cur = 0, cols = 0;\n        next_img = 0;"),
+    # position table: height and width coordinates exchanged
+    "rope_hw_swap": ("table[1 * n + cols] = hh + cur;", "table[1 * n + cols] = ww + cur;"),
+    # position table: delta taken against the padded length
+    "rope_delta_padded": ("deltas[b] = n > 0 ? mx + 1 - n : 0;", "deltas[b] = n > 0 ? mx + 1 - L : 0;"),
+    # position table: image temporal index dropped
+    "rope_image_time": ("table[0 * n + cols] = tt * 1 + cur;", "table[0 * n + cols] = cur;"),
 }
 
 
