@@ -43,6 +43,7 @@
 #ifndef IPE_H
 #define IPE_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -64,6 +65,7 @@ typedef enum {
 #define IPE_MAX_IMAGES 1024     /* images per vision call                     */
 #define IPE_MAX_HALF 256        /* rot_dim / 2 of the text rotary             */
 #define IPE_MAX_POSITION 16777216 /* positions must lie in [0, 2^24): fl32(pos) is exact */
+#define IPE_MAX_GRIDS 16384     /* image grids, and video grids, per position-table call */
 
 /* Message for the last non-OK status returned on this thread ("" if none). */
 const char *ipe_last_error(void);
@@ -78,8 +80,9 @@ int ipe_version(void);
  * code in a device status word and lets the kernel return instead of spinning.
  * This call synchronises `stream`, reads and clears that word, and returns
  * IPE_OK, or IPE_EDEVICE with a message naming the wait that gave up (the
- * results of the failed launch are then incomplete).  Not part of any page:
- * failure reporting of this library.
+ * results of the failed launch are then incomplete).  ipe_mrope_rope_index
+ * reports inputs that only the device can see the same way (codes 16 .. 20,
+ * listed there).  Not part of any page: failure reporting of this library.
  * ------------------------------------------------------------------------- */
 int ipe_device_status(void *stream);
 
@@ -195,6 +198,56 @@ int ipe_qk_norm_mrope(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int 
                       const void *k_weight, float eps, const int32_t *positions,
                       const float *inv_freq_host, int rot_dim, const int32_t *section,
                       int interleaved, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * ipe_mrope_rope_index -- three-axis position table and rope deltas of a batch
+ * of B mixed sequences padded to L slots, on the device (no host sync).
+ * [IRPE] get_rope_index(): preparing the grids, filtering padding and
+ * splitting runs, advancing the position, flattening the vision grid, joining
+ * the sequence back, returning positions and deltas; the worked single-batch
+ * table; mm_tokens (type codes).  The rules:
+ *   - video grid rows (t, h, w) count as t grids (1, h, w), one per temporal
+ *     slice; image grids are used as given (llm_t = t);
+ *   - one image and one video grid sequence serve the whole batch, consumed
+ *     in the order of samples and, within a sample, of appearance;
+ *   - per sample the slots with mask 0 are dropped; the kept slots form runs
+ *     of equal type; a position starting at 0 walks the runs: a text run
+ *     (type 0, or 3 = audio, laid out like text) takes consecutive positions
+ *     on all three rows; a vision run (1 image, 2 video) takes the next grid
+ *     of its kind and gives its k-th slot, k = (tt*(h/m) + row)*(w/m) + col,
+ *     the coordinates (start + tt, start + row, start + col); the position
+ *     then moves on by max(h, w) / m;
+ *   - dropped slots get 0 on all rows; rope_deltas[b] = (largest coordinate
+ *     of the sample) + 1 - (its kept slots), 0 for a sample with none.
+ *   mm_token_type_ids  device [B, L] integers of id_bytes (4 or 8) each
+ *   attention_mask     device [B, L] of id_bytes, non-zero = kept; NULL keeps all
+ *   image_grid_thw     device [n_images, 3] integers of grid_bytes (4 or 8)
+ *   video_grid_thw     device [n_videos, 3] of grid_bytes; NULL iff n_videos == 0
+ *                      (likewise the image grids)
+ *   spatial_merge      m, 1 .. 64
+ *   position_ids       device int32 [3, B, L], written (rows t, h, w)
+ *   rope_deltas        device int32 [B], written
+ *   workspace          device scratch of at least
+ *                      ipe_mrope_rope_index_workspace(B, L, n_images, n_videos)
+ *                      bytes, 16-byte aligned; overwritten; no initial value
+ *                      needed.  Calls that share it must not overlap.
+ * Limits: B * L <= 2^31 - 1, L <= 2^30, n_images and n_videos <= IPE_MAX_GRIDS.
+ * What only the device sees is reported through ipe_device_status: 16 a
+ * vision run found no grid left; 17 a vision run's length differs from its
+ * grid's cell count (the pages' listing only fails when a sample's totals
+ * differ; here every run is checked); 18 a kept slot of a type other than
+ * 0 .. 3 (laid out as text); 19 a grid with t, h or w outside 1 .. 32768;
+ * 20 a coordinate beyond the int32 range.  The table is written regardless.
+ * Uses three kernel launches on `stream`.
+ * ------------------------------------------------------------------------- */
+int ipe_mrope_rope_index(const void *mm_token_type_ids, const void *attention_mask, int id_bytes,
+                         int64_t B, int64_t L, const void *image_grid_thw, int n_images,
+                         const void *video_grid_thw, int n_videos, int grid_bytes, int spatial_merge,
+                         int32_t *position_ids, int32_t *rope_deltas, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/* Workspace bytes ipe_mrope_rope_index needs for these sizes (0 on bad sizes). */
+size_t ipe_mrope_rope_index_workspace(int64_t B, int64_t L, int n_images, int n_videos);
 
 /* ---------------------------------------------------------------------------
  * Vision grids.  grid_thw_host is a host int32 [n_images, 3] array of

@@ -39,6 +39,8 @@ _SIGS = {
     "ipe_mrope_apply": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, _I, _P, _I, _P]),
     "ipe_qk_norm_mrope": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, ctypes.c_float, _P, _P, _I, _P, _I,
                                _P]),
+    "ipe_mrope_rope_index": (_I, [_P, _P, _I, _I64, _I64, _P, _I, _P, _I, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
+    "ipe_mrope_rope_index_workspace": (ctypes.c_size_t, [_I64, _I64, _I, _I]),
     "ipe_vis_interp_plan": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
     "ipe_vis_pos_interp": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P]),
     "ipe_vis_rope2d": (_I, [_P, _P, _I, _I64, _I, _I, _I64, _I64, _P, _I, _I, _D, _P]),
@@ -263,6 +265,66 @@ def qk_norm_mrope(q, k, q_weight, k_weight, positions, inv_freq, section, interl
                                   float(eps), _ptr(positions), inv, 2 * half, _i32_host(section, 3),
                                   int(bool(interleaved)), _stream(stream)))
     return q, k
+
+
+def rope_index_workspace_bytes(B, L, n_images=0, n_videos=0):
+    """Device scratch bytes mrope_rope_index needs for these sizes."""
+    n = _lib.ipe_mrope_rope_index_workspace(int(B), int(L), int(n_images), int(n_videos))
+    if n == 0 and B > 0:
+        raise ValueError(f"rope_index: sizes out of range (B={B}, L={L}, images={n_images}, videos={n_videos})")
+    return n
+
+
+def _int_tensor(t, name, shape=None):
+    _cuda(t, name)
+    if t.dtype not in (torch.int32, torch.int64) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous int32 or int64 tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    return t
+
+
+def mrope_rope_index(mm_token_type_ids, image_grid_thw=None, video_grid_thw=None, attention_mask=None,
+                     spatial_merge_size=2, position_ids=None, rope_deltas=None, workspace=None, stream=None):
+    """(position_ids int32 [3, B, L], rope_deltas int32 [B]) of a batch of
+    mixed sequences, computed on the device.  Types and mask are [B, L] int32
+    or int64 (the same dtype); grids [n, 3] int32 or int64 (the same dtype)."""
+    ty = _int_tensor(mm_token_type_ids, "mm_token_type_ids")
+    if ty.dim() != 2:
+        raise ValueError("mm_token_type_ids must be [B, L]")
+    B, L = ty.shape
+    if attention_mask is not None:
+        _int_tensor(attention_mask, "attention_mask", (B, L))
+        if attention_mask.dtype != ty.dtype:
+            raise ValueError("attention_mask must have the dtype of mm_token_type_ids")
+    grids = [g for g in (image_grid_thw, video_grid_thw) if g is not None]
+    for g, nm in zip(grids, ("grid",) * 2):
+        _int_tensor(g, nm)
+        if g.dim() != 2 or g.shape[1] != 3:
+            raise ValueError("grids must be [n, 3]")
+    if len(grids) == 2 and grids[0].dtype != grids[1].dtype:
+        raise ValueError("image_grid_thw and video_grid_thw must share a dtype")
+    gbytes = grids[0].element_size() if grids else 4
+    n_img = 0 if image_grid_thw is None else image_grid_thw.shape[0]
+    n_vid = 0 if video_grid_thw is None else video_grid_thw.shape[0]
+    dev = ty.device
+    if position_ids is None:
+        position_ids = torch.empty(3, B, L, dtype=torch.int32, device=dev)
+    if rope_deltas is None:
+        rope_deltas = torch.empty(B, dtype=torch.int32, device=dev)
+    for t, nm, shp in ((position_ids, "position_ids", (3, B, L)), (rope_deltas, "rope_deltas", (B,))):
+        _cuda(t, nm)
+        if t.dtype != torch.int32 or tuple(t.shape) != shp or not t.is_contiguous():
+            raise ValueError(f"{nm} must be a contiguous int32 {shp} tensor")
+    need = rope_index_workspace_bytes(B, L, n_img, n_vid) if B > 0 else 0
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _cuda(workspace, "workspace")
+    _check(_lib.ipe_mrope_rope_index(_ptr(ty), _ptr(attention_mask), ty.element_size(), B, L, _ptr(image_grid_thw),
+                                     n_img, _ptr(video_grid_thw), n_vid, gbytes, int(spatial_merge_size),
+                                     _ptr(position_ids), _ptr(rope_deltas), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)))
+    return position_ids, rope_deltas
 
 
 # ------------------------------------------------------------------- vision

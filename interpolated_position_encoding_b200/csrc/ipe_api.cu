@@ -342,6 +342,11 @@ int ipe_device_status(void *stream)
     const char *what = v == 1 ? "a consumer warp gave up waiting for a stage's data"
                      : v == 2 ? "the producer gave up waiting for a free stage"
                      : v == 3 ? "loads in flight did not land while a block shut down"
+                     : v == 16 ? "position table: a vision run found no grid left"
+                     : v == 17 ? "position table: a vision run's length differs from its grid's cell count"
+                     : v == 18 ? "position table: a kept slot has a type other than 0, 1, 2, 3"
+                     : v == 19 ? "position table: a grid has t, h or w outside 1 .. 32768"
+                     : v == 20 ? "position table: a coordinate beyond the int32 range"
                               : "unknown";
     return fail(IPE_EDEVICE, "device fault %u: %s", v, what);
 }
@@ -505,6 +510,83 @@ int ipe_qk_norm_mrope(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int 
     n.eps = eps;
     cudaError_t e = launch_qk_norm_mrope(dtype == IPE_BF16, n, a, (cudaStream_t)stream);
     return e == cudaSuccess ? ok() : cuda_fail(e, "qk_norm_mrope launch");
+}
+
+static int rope_index_sizes(int64_t B, int64_t L, int n_images, int n_videos)
+{
+    if (B < 0 || L < 0) return fail(IPE_EINVAL, "B %lld and L %lld must be >= 0", (long long)B, (long long)L);
+    if (L > (1LL << 30) || (L > 0 && B > ((1LL << 31) - 1) / L))
+        return fail(IPE_ELIMIT, "B * L must stay within 2^31 - 1 and L within 2^30");
+    if (n_images < 0 || n_videos < 0 || n_images > IPE_MAX_GRIDS || n_videos > IPE_MAX_GRIDS)
+        return fail(IPE_ELIMIT, "n_images %d and n_videos %d must lie in 0 .. %d", n_images, n_videos, IPE_MAX_GRIDS);
+    return IPE_OK;
+}
+
+size_t ipe_mrope_rope_index_workspace(int64_t B, int64_t L, int n_images, int n_videos)
+{
+    if (rope_index_sizes(B, L, n_images, n_videos) != IPE_OK) return 0;
+    return rope_index_layout(B, L, n_images, n_videos).total;
+}
+
+int ipe_mrope_rope_index(const void *mm_token_type_ids, const void *attention_mask, int id_bytes, int64_t B, int64_t L,
+                         const void *image_grid_thw, int n_images, const void *video_grid_thw, int n_videos,
+                         int grid_bytes, int spatial_merge, int32_t *position_ids, int32_t *rope_deltas,
+                         void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (int rc = rope_index_sizes(B, L, n_images, n_videos)) return rc;
+    if (id_bytes != 4 && id_bytes != 8) return fail(IPE_EINVAL, "id_bytes %d must be 4 or 8", id_bytes);
+    if (grid_bytes != 4 && grid_bytes != 8) return fail(IPE_EINVAL, "grid_bytes %d must be 4 or 8", grid_bytes);
+    if (spatial_merge < 1 || spatial_merge > 64) return fail(IPE_EINVAL, "spatial_merge %d must lie in 1 .. 64", spatial_merge);
+    if (B == 0) return ok();
+    const RopeIndexLayout lay = rope_index_layout(B, L, n_images, n_videos);
+    if (workspace_bytes < lay.total)
+        return fail(IPE_EINVAL, "workspace_bytes %zu below the %zu this call needs", workspace_bytes, lay.total);
+    if (!aligned(mm_token_type_ids, id_bytes) || !aligned(attention_mask, id_bytes) ||
+        !aligned(image_grid_thw, grid_bytes) || !aligned(video_grid_thw, grid_bytes) || !aligned(position_ids, 4) ||
+        !aligned(rope_deltas, 4) || !aligned(workspace, 16))
+        return fail(IPE_EALIGN, "ids, grids, outputs and workspace must be aligned to their element (workspace: 16 bytes)");
+    const size_t slots = (size_t)B * (size_t)L;
+    if (slots > 0) {
+        if (int rc = check_dev(mm_token_type_ids, slots * id_bytes, "mm_token_type_ids")) return rc;
+        if (attention_mask) {
+            if (int rc = check_dev(attention_mask, slots * id_bytes, "attention_mask")) return rc;
+        }
+        if (int rc = check_dev(position_ids, 3 * slots * 4, "position_ids")) return rc;
+    }
+    if (int rc = check_dev(rope_deltas, (size_t)B * 4, "rope_deltas")) return rc;
+    if (n_images > 0) {
+        if (int rc = check_dev(image_grid_thw, (size_t)n_images * 3 * grid_bytes, "image_grid_thw")) return rc;
+    }
+    if (n_videos > 0) {
+        if (int rc = check_dev(video_grid_thw, (size_t)n_videos * 3 * grid_bytes, "video_grid_thw")) return rc;
+    }
+    if (int rc = check_dev(workspace, lay.total, "workspace")) return rc;
+    char *w = static_cast<char *>(workspace);
+    RopeIndexArgs a{};
+    a.types = mm_token_type_ids;
+    a.mask = attention_mask;
+    a.img_grid = image_grid_thw;
+    a.vid_grid = video_grid_thw;
+    a.id_bytes = id_bytes;
+    a.grid_bytes = grid_bytes;
+    a.B = B;
+    a.L = L;
+    a.tiles_per_row = (int)((L + kRiTile - 1) / kRiTile);
+    a.n_img = n_images;
+    a.n_vid = n_videos;
+    a.merge = spatial_merge;
+    a.pos = position_ids;
+    a.deltas = rope_deltas;
+    a.agg = w;
+    a.carry = w + lay.agg;
+    a.sample = w + lay.agg + lay.carry;
+    a.img_adv = reinterpret_cast<long long *>(w + lay.agg + lay.carry + lay.sample);
+    a.vid_slices = reinterpret_cast<long long *>(w + lay.agg + lay.carry + lay.sample + lay.img_adv);
+    a.vid_adv = reinterpret_cast<long long *>(w + lay.agg + lay.carry + lay.sample + lay.img_adv + lay.vid_slices);
+    a.status = device_status_word();
+    if (!a.status) return fail(IPE_ECUDA, "device status word unavailable");
+    cudaError_t e = launch_rope_index(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "rope_index launch");
 }
 
 int ipe_vis_interp_plan(const int32_t *grid_thw_host, int n_images, int merge, int grid_side, int32_t *idx4,

@@ -110,6 +110,37 @@ struct QkNormArgs {
 
 cudaError_t launch_qk_norm_mrope(bool bf16, const QkNormArgs &n, const MropeAngles &a, cudaStream_t s);
 
+// ------------------------------------------------------- position table
+// Tile of the position-table kernels: 256 threads x 4 consecutive slots.
+constexpr int kRiThreads = 256;
+constexpr int kRiPer = 4;
+constexpr int kRiTile = kRiThreads * kRiPer;
+
+// One call of ipe_mrope_rope_index, validated on the host.  The workspace
+// carries the per-tile aggregates, the per-tile carries, one record per sample
+// and the grid prefix sums, each at a 256-byte aligned offset.
+struct RopeIndexArgs {
+    const void *types, *mask;          // [B, L] of id_bytes each; mask may be NULL
+    const void *img_grid, *vid_grid;   // [n, 3] of grid_bytes each
+    int id_bytes, grid_bytes;
+    long long B, L;
+    int tiles_per_row;                 // ceil(L / kRiTile)
+    int n_img, n_vid, merge;
+    int32_t *pos;                      // [3, B, L]
+    int32_t *deltas;                   // [B]
+    void *agg, *carry, *sample;        // workspace sections
+    long long *img_adv;                // [n_img + 1] prefix of the image advances
+    long long *vid_slices, *vid_adv;   // [n_vid + 1] prefixes of slices and of slice advances
+    unsigned *status;
+};
+
+// Bytes of each workspace section for a call; the sum is the workspace size.
+struct RopeIndexLayout {
+    size_t agg, carry, sample, img_adv, vid_slices, vid_adv, total;
+};
+RopeIndexLayout rope_index_layout(long long B, long long L, int n_img, int n_vid);
+cudaError_t launch_rope_index(const RopeIndexArgs &a, cudaStream_t s);
+
 // Test hooks and the device status word (ipe_api.cu).
 unsigned *device_status_word();
 long long debug_skip_tile();

@@ -1,0 +1,700 @@
+// Three-axis position table (position_ids [3, B, L]) and rope deltas of a
+// batch of mixed text / image / video sequences.
+//
+// "Interleaved Rotary Position Embedding" (taking-lying-flat.github.io),
+// get_rope_index(): video grids are split into one (1, h, w) grid per temporal
+// slice; one image and one video grid sequence serve the whole batch in order;
+// per sample the padded slots are dropped, the kept slots are split into runs
+// of equal type, and a running position walks the runs -- a text run takes
+// consecutive positions on all three rows, a vision run lays its merged grid
+// out width-fastest at (start + t, start + row, start + col) and moves the
+// position on by its longer merged side.  The delta of a sample is its
+// largest coordinate + 1 - its kept slot count.  Section "mm_tokens" gives the
+// type codes (0 text, 1 image, 2 video, 3 audio); audio follows the text rule.
+//
+// The pages walk the runs one after another.  Here every coordinate follows
+// from counts over the slots before it, which makes the table a scan:
+//   * a kept text slot sits at (kept text slots before it in the sample)
+//     + (advances of the sample's vision runs that start before it);
+//   * a vision run starts at that same value and its k-th slot is the k-th
+//     cell of its grid.
+// Three launches, all on the caller's stream:
+//   1. ri_tile_kernel   -- per tile of 1024 slots: kept / text counts, run
+//      starts by kind, and where the last run start lies;
+//   2. ri_carry_kernel  -- one block: the grid prefix sums, then per sample a
+//      scan over its tiles giving the state before each tile (counts, the
+//      summed advances, and the run still open at the tile's first slot);
+//   3. ri_write_kernel  -- per tile: every slot's coordinates, the tile's
+//      largest one, and in the last tile of a sample to finish, the delta.
+// Slots of a kind the method does not define, grids that run out, and vision
+// runs whose length differs from their grid's cell count are reported through
+// the device status word (ipe_device_status); the table is still written.
+#include <climits>
+
+#include "ipe_internal.h"
+#include "ipe_tma.cuh"
+
+namespace ipe {
+
+// Status codes of this kernel family (the word's first fault wins).
+constexpr unsigned kRiNoGrid = 16;      // a vision run found no grid left
+constexpr unsigned kRiRunLength = 17;   // a vision run's length differs from its grid's cell count
+constexpr unsigned kRiBadType = 18;     // a kept slot of a type other than 0, 1, 2, 3
+constexpr unsigned kRiBadGrid = 19;     // a grid with t, h or w outside 1 .. kRiMaxSide
+constexpr unsigned kRiOverflow = 20;    // a coordinate beyond the int32 range
+constexpr int kRiMaxSide = 1 << 15;
+
+struct RiTileAgg {
+    int kept, text;               // kept slots; kept text-like slots (type 0 or 3)
+    int first_cls, last_cls;      // class of the first / last kept slot (-1: none)
+    int img, vid;                 // image / video run starts, the first kept slot not counted
+    int ls_off;                   // kept offset in the tile of the last such start (-1: none)
+    int ls_text, ls_img, ls_vid;  // text slots and image / video starts of the tile before it
+    int ls_cls, pad;
+};
+
+struct RiCarry {
+    int k0, text0;                // kept and kept-text slots of the sample before the tile
+    int img0, vid0;               // image / video runs of the batch before the tile
+    long long vadv0;              // advances of the sample's vision runs started before the tile
+    int prev_cls;                 // class of the last kept slot before the tile (-1: none)
+    int open_k, open_grid;        // the run open at the tile's first slot: first kept index, grid
+    int pad;
+    long long open_start;         // ... and its start position
+};
+
+struct RiSample {
+    int kept;                     // kept slots of the sample
+    int img, vid;                 // image / video runs: of the sample, then (scanned) of the batch before it
+    int max_pos;                  // largest coordinate written
+    unsigned done;                // tiles finished
+    int pad[3];
+};
+
+RopeIndexLayout rope_index_layout(long long B, long long L, int n_img, int n_vid)
+{
+    auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
+    const long long tiles = B * ((L + kRiTile - 1) / kRiTile);
+    RopeIndexLayout l;
+    l.agg = up((size_t)tiles * sizeof(RiTileAgg));
+    l.carry = up((size_t)tiles * sizeof(RiCarry));
+    l.sample = up((size_t)B * sizeof(RiSample));
+    l.img_adv = up((size_t)(n_img + 1) * sizeof(long long));
+    l.vid_slices = up((size_t)(n_vid + 1) * sizeof(long long));
+    l.vid_adv = up((size_t)(n_vid + 1) * sizeof(long long));
+    l.total = l.agg + l.carry + l.sample + l.img_adv + l.vid_slices + l.vid_adv;
+    return l;
+}
+
+// ------------------------------------------------------------------ access
+
+__device__ __forceinline__ long long ld_int(const void *p, int bytes, long long i)
+{
+    return bytes == 8 ? static_cast<const long long *>(p)[i] : (long long)static_cast<const int *>(p)[i];
+}
+
+// Class of a slot: 0 text-like (types 0 and 3), 1 image, 2 video.  Types the
+// method does not define are reported and laid out as text.
+__device__ __forceinline__ void load_slots(const RopeIndexArgs &a, long long b, long long l0, int *cls, bool *kept,
+                                           bool report)
+{
+#pragma unroll
+    for (int i = 0; i < kRiPer; ++i) {
+        const long long l = l0 + i;
+        kept[i] = false;
+        cls[i] = 0;
+        if (l < a.L) {
+            const long long at = b * a.L + l;
+            kept[i] = a.mask == nullptr || ld_int(a.mask, a.id_bytes, at) != 0;
+            const long long t = ld_int(a.types, a.id_bytes, at);
+            if (t == 1 || t == 2) cls[i] = (int)t;
+            else if (kept[i] && t != 0 && t != 3 && report) record_fault(a.status, kRiBadType);
+        }
+    }
+}
+
+struct RiGrid {
+    int t, h, w;   // merged: t, h / merge, w / merge
+    int adv;       // max(h, w) / merge
+};
+
+__device__ __forceinline__ bool side_ok(long long v) { return v >= 1 && v <= kRiMaxSide; }
+
+// Grid row j of an image (t as given) or a video (t = 1 per slice).
+__device__ __forceinline__ RiGrid grid_row(const RopeIndexArgs &a, const void *g, int j, bool video)
+{
+    const long long t = ld_int(g, a.grid_bytes, 3LL * j), h = ld_int(g, a.grid_bytes, 3LL * j + 1),
+                    w = ld_int(g, a.grid_bytes, 3LL * j + 2);
+    RiGrid r{0, 0, 0, 0};
+    if (!side_ok(t) || !side_ok(h) || !side_ok(w)) return r;
+    r.t = video ? 1 : (int)t;
+    r.h = (int)h / a.merge;
+    r.w = (int)w / a.merge;
+    r.adv = (int)(h > w ? h : w) / a.merge;
+    return r;
+}
+
+// Video grid row holding slice v (v below the slice total).
+__device__ __forceinline__ int slice_row(const RopeIndexArgs &a, long long v)
+{
+    const long long *s = reinterpret_cast<const long long *>(a.vid_slices);
+    int lo = 0, hi = a.n_vid - 1;   // the largest j with s[j] <= v
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s[mid] <= v) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Summed advances of the image grids [0, i) and of the video slices [0, v).
+__device__ __forceinline__ long long img_adv_before(const RopeIndexArgs &a, long long i)
+{
+    return reinterpret_cast<const long long *>(a.img_adv)[i < a.n_img ? i : a.n_img];
+}
+__device__ __forceinline__ long long vid_adv_before(const RopeIndexArgs &a, long long v)
+{
+    const long long *s = reinterpret_cast<const long long *>(a.vid_slices);
+    const long long *p = reinterpret_cast<const long long *>(a.vid_adv);
+    if (a.n_vid == 0 || v >= s[a.n_vid]) return p[a.n_vid];
+    const int j = slice_row(a, v);
+    return p[j] + (v - s[j]) * (long long)grid_row(a, a.vid_grid, j, true).adv;
+}
+
+// Grid of vision run number g of class cls (false when the grids ran out).
+__device__ __forceinline__ bool run_grid(const RopeIndexArgs &a, int cls, long long g, RiGrid &r)
+{
+    if (cls == 1) {
+        if (g < 0 || g >= a.n_img) return false;
+        r = grid_row(a, a.img_grid, (int)g, false);
+        return true;
+    }
+    const long long *s = reinterpret_cast<const long long *>(a.vid_slices);
+    if (g < 0 || a.n_vid == 0 || g >= s[a.n_vid]) return false;
+    r = grid_row(a, a.vid_grid, slice_row(a, g), true);
+    return true;
+}
+
+// ------------------------------------------------------------ block scans
+
+// Four sums and a max (keys: 0 = none, larger = later).
+struct RiSums {
+    int kept, text, img, vid, last;
+};
+
+__device__ __forceinline__ RiSums ri_op(const RiSums &x, const RiSums &y)
+{
+    return {x.kept + y.kept, x.text + y.text, x.img + y.img, x.vid + y.vid, x.last > y.last ? x.last : y.last};
+}
+
+__device__ __forceinline__ RiSums ri_shfl_up(const RiSums &v, int d)
+{
+    return {__shfl_up_sync(0xffffffffu, v.kept, d), __shfl_up_sync(0xffffffffu, v.text, d),
+            __shfl_up_sync(0xffffffffu, v.img, d), __shfl_up_sync(0xffffffffu, v.vid, d),
+            __shfl_up_sync(0xffffffffu, v.last, d)};
+}
+
+// Exclusive scan over the block's threads in order; tot = the block total.
+__device__ RiSums ri_block_exclusive(const RiSums &v, RiSums *warp_tot, RiSums &tot)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    RiSums inc = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const RiSums o = ri_shfl_up(inc, d);
+        if (lane >= d) inc = ri_op(o, inc);
+    }
+    RiSums exc = ri_shfl_up(inc, 1);
+    if (lane == 0) exc = RiSums{0, 0, 0, 0, 0};
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    RiSums pre{0, 0, 0, 0, 0};
+    tot = pre;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+        if (w < warp) pre = ri_op(pre, warp_tot[w]);
+        tot = ri_op(tot, warp_tot[w]);
+    }
+    __syncthreads();
+    return ri_op(pre, exc);
+}
+
+// ------------------------------------------------------- 1. tile aggregates
+
+__global__ void __launch_bounds__(kRiThreads) ri_tile_kernel(const __grid_constant__ RopeIndexArgs a)
+{
+    __shared__ RiSums warp_tot[kRiThreads / 32];
+    __shared__ RiTileAgg s;
+    const long long tile = blockIdx.x;
+    const long long b = tile / a.tiles_per_row;
+    const int local0 = threadIdx.x * kRiPer;
+    const long long l0 = (tile % a.tiles_per_row) * kRiTile + local0;
+    int cls[kRiPer];
+    bool kept[kRiPer];
+    load_slots(a, b, l0, cls, kept, false);
+    if (threadIdx.x == 0) s = RiTileAgg{0, 0, -1, -1, 0, 0, -1, 0, 0, 0, -1, 0};
+
+    // class of the last kept slot before each thread's slots
+    RiSums v{0, 0, 0, 0, 0}, tot1, tot2;
+#pragma unroll
+    for (int i = 0; i < kRiPer; ++i)
+        if (kept[i]) v.last = (local0 + i + 1) * 4 + cls[i];
+    const RiSums ex1 = ri_block_exclusive(v, warp_tot, tot1);
+    int prev = ex1.last ? (ex1.last & 3) : -1;
+
+    // counts; run starts other than at the tile's first kept slot
+    RiSums c{0, 0, 0, 0, 0};
+    int ls_off = 0, ls_text = 0, ls_img = 0, ls_vid = 0, ls_cls = -1;
+#pragma unroll
+    for (int i = 0; i < kRiPer; ++i) {
+        if (!kept[i]) continue;
+        if (prev < 0) {
+            s.first_cls = cls[i];
+        } else if (cls[i] != prev) {
+            ls_off = c.kept;
+            ls_text = c.text;
+            ls_img = c.img;
+            ls_vid = c.vid;
+            ls_cls = cls[i];
+            c.last = local0 + i + 1;
+            c.img += cls[i] == 1;
+            c.vid += cls[i] == 2;
+        }
+        c.kept += 1;
+        c.text += cls[i] == 0;
+        prev = cls[i];
+    }
+    const RiSums ex2 = ri_block_exclusive(c, warp_tot, tot2);
+    if (c.last != 0 && c.last == tot2.last) {
+        s.ls_off = ex2.kept + ls_off;
+        s.ls_text = ex2.text + ls_text;
+        s.ls_img = ex2.img + ls_img;
+        s.ls_vid = ex2.vid + ls_vid;
+        s.ls_cls = ls_cls;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        RiTileAgg o = s;
+        o.kept = tot2.kept;
+        o.text = tot2.text;
+        o.img = tot2.img;
+        o.vid = tot2.vid;
+        o.last_cls = tot1.last ? (tot1.last & 3) : -1;
+        static_cast<RiTileAgg *>(a.agg)[tile] = o;
+    }
+}
+
+// --------------------------------------------------- 2. carries (one block)
+
+constexpr int kRiCarryThreads = 1024;
+
+// Exclusive block scan of long long pairs (1024 threads); tot = the total.
+__device__ longlong2 scan_pair(longlong2 v, longlong2 *warp_tot, longlong2 &tot)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    longlong2 inc = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const long long x = __shfl_up_sync(0xffffffffu, inc.x, d), y = __shfl_up_sync(0xffffffffu, inc.y, d);
+        if (lane >= d) {
+            inc.x += x;
+            inc.y += y;
+        }
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    longlong2 pre{0, 0};
+    tot = pre;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+        if (w < warp) {
+            pre.x += warp_tot[w].x;
+            pre.y += warp_tot[w].y;
+        }
+        tot.x += warp_tot[w].x;
+        tot.y += warp_tot[w].y;
+    }
+    __syncthreads();
+    return make_longlong2(pre.x + inc.x - v.x, pre.y + inc.y - v.y);
+}
+
+__device__ __forceinline__ int warp_incl_max(int v)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, d);
+        if (lane >= d && o > v) v = o;
+    }
+    return v;
+}
+
+__device__ __forceinline__ int warp_incl_sum(int v)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, d);
+        if (lane >= d) v += o;
+    }
+    return v;
+}
+
+// Per tile of one chunk of 32 (lane = tile): its aggregate, the class before
+// it, and whether its first kept slot starts a run.
+struct RiTileView {
+    RiTileAgg g;
+    int prev, first_start, img, vid;   // img / vid: run starts including the first kept slot
+};
+
+__device__ __forceinline__ RiTileView view_tile(const RopeIndexArgs &a, long long b, int t, int &carry_key)
+{
+    RiTileView r;
+    r.g = RiTileAgg{0, 0, -1, -1, 0, 0, -1, 0, 0, 0, -1, 0};
+    if (t < a.tiles_per_row) r.g = static_cast<const RiTileAgg *>(a.agg)[b * a.tiles_per_row + t];
+    const int key = r.g.kept > 0 ? (t + 1) * 4 + r.g.last_cls : 0;
+    const int inc = warp_incl_max(key);
+    int exc = __shfl_up_sync(0xffffffffu, inc, 1);
+    if ((threadIdx.x & 31) == 0) exc = 0;
+    if (carry_key > exc) exc = carry_key;
+    carry_key = max(carry_key, __shfl_sync(0xffffffffu, inc, 31));
+    r.prev = exc ? (exc & 3) : -1;
+    r.first_start = r.g.kept > 0 && r.g.first_cls != r.prev;
+    r.img = r.g.img + (r.first_start && r.g.first_cls == 1);
+    r.vid = r.g.vid + (r.first_start && r.g.first_cls == 2);
+    return r;
+}
+
+__global__ void __launch_bounds__(kRiCarryThreads) ri_carry_kernel(const __grid_constant__ RopeIndexArgs a)
+{
+    __shared__ longlong2 warp_tot[kRiCarryThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+    long long *img_adv = reinterpret_cast<long long *>(a.img_adv);
+    long long *vid_slices = reinterpret_cast<long long *>(a.vid_slices);
+    long long *vid_adv = reinterpret_cast<long long *>(a.vid_adv);
+    RiSample *smp = static_cast<RiSample *>(a.sample);
+
+    // grid prefix sums: image advances; video slices and slice advances
+    longlong2 run{0, 0}, tot;
+    for (int c0 = 0; c0 < a.n_img; c0 += blockDim.x) {
+        const int j = c0 + threadIdx.x;
+        long long adv = 0;
+        if (j < a.n_img) {
+            const long long t = ld_int(a.img_grid, a.grid_bytes, 3LL * j), h = ld_int(a.img_grid, a.grid_bytes, 3LL * j + 1),
+                            w = ld_int(a.img_grid, a.grid_bytes, 3LL * j + 2);
+            if (!side_ok(t) || !side_ok(h) || !side_ok(w)) record_fault(a.status, kRiBadGrid);
+            adv = grid_row(a, a.img_grid, j, false).adv;
+        }
+        const longlong2 ex = scan_pair(make_longlong2(adv, 0), warp_tot, tot);
+        if (j < a.n_img) img_adv[j] = run.x + ex.x;
+        run.x += tot.x;
+    }
+    if (threadIdx.x == 0) img_adv[a.n_img] = run.x;
+    run = make_longlong2(0, 0);
+    for (int c0 = 0; c0 < a.n_vid; c0 += blockDim.x) {
+        const int j = c0 + threadIdx.x;
+        longlong2 v{0, 0};
+        if (j < a.n_vid) {
+            const long long t = ld_int(a.vid_grid, a.grid_bytes, 3LL * j), h = ld_int(a.vid_grid, a.grid_bytes, 3LL * j + 1),
+                            w = ld_int(a.vid_grid, a.grid_bytes, 3LL * j + 2);
+            const bool good = side_ok(t) && side_ok(h) && side_ok(w);
+            if (!good) record_fault(a.status, kRiBadGrid);
+            v.x = good ? t : 0;
+            v.y = v.x * grid_row(a, a.vid_grid, j, true).adv;
+        }
+        const longlong2 ex = scan_pair(v, warp_tot, tot);
+        if (j < a.n_vid) {
+            vid_slices[j] = run.x + ex.x;
+            vid_adv[j] = run.y + ex.y;
+        }
+        run.x += tot.x;
+        run.y += tot.y;
+    }
+    if (threadIdx.x == 0) {
+        vid_slices[a.n_vid] = run.x;
+        vid_adv[a.n_vid] = run.y;
+    }
+
+    // image / video runs of every sample (one warp per sample)
+    for (long long b = warp; b < a.B; b += nwarp) {
+        int carry_key = 0, n_img = 0, n_vid = 0;
+        for (int c0 = 0; c0 < a.tiles_per_row; c0 += 32) {
+            const RiTileView r = view_tile(a, b, c0 + lane, carry_key);
+            n_img += __shfl_sync(0xffffffffu, warp_incl_sum(r.img), 31);
+            n_vid += __shfl_sync(0xffffffffu, warp_incl_sum(r.vid), 31);
+        }
+        if (lane == 0) {
+            smp[b].img = n_img;
+            smp[b].vid = n_vid;
+        }
+    }
+    __syncthreads();
+
+    // runs of the batch before each sample
+    run = make_longlong2(0, 0);
+    for (long long c0 = 0; c0 < a.B; c0 += blockDim.x) {
+        const long long b = c0 + threadIdx.x;
+        longlong2 v{0, 0};
+        if (b < a.B) v = make_longlong2(smp[b].img, smp[b].vid);
+        const longlong2 ex = scan_pair(v, warp_tot, tot);
+        if (b < a.B) {
+            smp[b].img = (int)(run.x + ex.x);
+            smp[b].vid = (int)(run.y + ex.y);
+        }
+        run.x += tot.x;
+        run.y += tot.y;
+    }
+    __syncthreads();
+
+    // the state before every tile (one warp per sample)
+    for (long long b = warp; b < a.B; b += nwarp) {
+        const int img_s = smp[b].img, vid_s = smp[b].vid;
+        const long long base_adv = img_adv_before(a, img_s) + vid_adv_before(a, vid_s);
+        int carry_key = 0, k_run = 0, text_run = 0, img_run = img_s, vid_run = vid_s;
+        // the last run start before the current chunk
+        int o_k = 0, o_grid = -1;
+        long long o_start = 0;
+        for (int c0 = 0; c0 < a.tiles_per_row; c0 += 32) {
+            const int t = c0 + lane;
+            const RiTileView r = view_tile(a, b, t, carry_key);
+            const int k_inc = warp_incl_sum(r.g.kept), text_inc = warp_incl_sum(r.g.text);
+            const int img_inc = warp_incl_sum(r.img), vid_inc = warp_incl_sum(r.vid);
+            const int k0 = k_run + k_inc - r.g.kept, text0 = text_run + text_inc - r.g.text;
+            const int img0 = img_run + img_inc - r.img, vid0 = vid_run + vid_inc - r.vid;
+            const long long vadv0 = img_adv_before(a, img0) + vid_adv_before(a, vid0) - base_adv;
+            // this tile's own last run start
+            const int has = r.g.ls_off >= 0 || r.first_start;
+            int my_k = 0, my_grid = -1;
+            long long my_start = 0;
+            if (has) {
+                const bool fs_img = r.first_start && r.g.first_cls == 1, fs_vid = r.first_start && r.g.first_cls == 2;
+                int off = 0, text_b = 0, ib = img0, vb = vid0, cls = r.g.first_cls;
+                if (r.g.ls_off >= 0) {
+                    off = r.g.ls_off;
+                    text_b = r.g.ls_text;
+                    ib = img0 + fs_img + r.g.ls_img;
+                    vb = vid0 + fs_vid + r.g.ls_vid;
+                    cls = r.g.ls_cls;
+                }
+                my_k = k0 + off;
+                my_start = text0 + text_b + img_adv_before(a, ib) + vid_adv_before(a, vb) - base_adv;
+                my_grid = cls == 1 ? ib : cls == 2 ? vb : -1;
+            }
+            // the last start in an earlier tile: exclusive "latest" scan over lanes
+            const int src_inc = warp_incl_max(has ? lane + 1 : 0);
+            int src = __shfl_up_sync(0xffffffffu, src_inc, 1);
+            if (lane == 0) src = 0;
+            const int sl = src > 0 ? src - 1 : 0;
+            const int s_k = __shfl_sync(0xffffffffu, my_k, sl), s_grid = __shfl_sync(0xffffffffu, my_grid, sl);
+            const long long s_start = __shfl_sync(0xffffffffu, my_start, sl);
+            if (t < a.tiles_per_row) {
+                RiCarry cr;
+                cr.k0 = k0;
+                cr.text0 = text0;
+                cr.img0 = img0;
+                cr.vid0 = vid0;
+                cr.vadv0 = vadv0;
+                cr.prev_cls = r.prev;
+                cr.open_k = src > 0 ? s_k : o_k;
+                cr.open_grid = src > 0 ? s_grid : o_grid;
+                cr.open_start = src > 0 ? s_start : o_start;
+                cr.pad = 0;
+                static_cast<RiCarry *>(a.carry)[b * a.tiles_per_row + t] = cr;
+            }
+            // carry to the next chunk
+            const int last_src = __shfl_sync(0xffffffffu, src_inc, 31);
+            if (last_src > 0) {
+                o_k = __shfl_sync(0xffffffffu, my_k, last_src - 1);
+                o_grid = __shfl_sync(0xffffffffu, my_grid, last_src - 1);
+                o_start = __shfl_sync(0xffffffffu, my_start, last_src - 1);
+            }
+            k_run += __shfl_sync(0xffffffffu, k_inc, 31);
+            text_run += __shfl_sync(0xffffffffu, text_inc, 31);
+            img_run += __shfl_sync(0xffffffffu, img_inc, 31);
+            vid_run += __shfl_sync(0xffffffffu, vid_inc, 31);
+        }
+        if (lane == 0) {
+            smp[b].kept = k_run;
+            smp[b].max_pos = -1;
+            smp[b].done = 0u;
+            if (a.tiles_per_row == 0) a.deltas[b] = 0;
+        }
+    }
+}
+
+// -------------------------------------------------------- 3. coordinates
+
+__global__ void __launch_bounds__(kRiThreads) ri_write_kernel(const __grid_constant__ RopeIndexArgs a)
+{
+    __shared__ RiSums warp_tot[kRiThreads / 32];
+    __shared__ int rec_k[kRiTile], rec_grid[kRiTile], rec_cls[kRiTile];
+    __shared__ long long rec_start[kRiTile];
+    __shared__ int warp_max[kRiThreads / 32];
+    const long long tile = blockIdx.x;
+    const long long b = tile / a.tiles_per_row;
+    const int local0 = threadIdx.x * kRiPer;
+    const long long l0 = (tile % a.tiles_per_row) * kRiTile + local0;
+    const RiCarry C = static_cast<const RiCarry *>(a.carry)[tile];
+    RiSample *smp = static_cast<RiSample *>(a.sample);
+    const int sample_kept = smp[b].kept;
+    const long long plane = a.B * a.L;
+    int cls[kRiPer];
+    bool kept[kRiPer];
+    load_slots(a, b, l0, cls, kept, true);
+
+    RiSums v{0, 0, 0, 0, 0}, tot;
+#pragma unroll
+    for (int i = 0; i < kRiPer; ++i)
+        if (kept[i]) v.last = (local0 + i + 1) * 4 + cls[i];
+    const RiSums ex1 = ri_block_exclusive(v, warp_tot, tot);
+    const int prev0 = ex1.last ? (ex1.last & 3) : C.prev_cls;
+
+    // counts and run starts, the tile's first kept slot included
+    RiSums c{0, 0, 0, 0, 0};
+    int prev = prev0;
+#pragma unroll
+    for (int i = 0; i < kRiPer; ++i) {
+        if (!kept[i]) continue;
+        if (cls[i] != prev) {
+            c.last = local0 + i + 1;
+            c.img += cls[i] == 1;
+            c.vid += cls[i] == 2;
+        }
+        c.kept += 1;
+        c.text += cls[i] == 0;
+        prev = cls[i];
+    }
+    const RiSums ex = ri_block_exclusive(c, warp_tot, tot);
+
+    // pass 1: records of the runs starting here; text slots
+    long long vadv = C.vadv0 + img_adv_before(a, C.img0 + ex.img) - img_adv_before(a, C.img0) +
+                     vid_adv_before(a, C.vid0 + ex.vid) - vid_adv_before(a, C.vid0);
+    int kept_b = ex.kept, text_b = ex.text, img_b = ex.img, vid_b = ex.vid;
+    long long mx = -1;
+    prev = prev0;
+#pragma unroll
+    for (int i = 0; i < kRiPer; ++i) {
+        const long long l = l0 + i;
+        if (l >= a.L) break;
+        const long long at = b * a.L + l;
+        if (!kept[i]) {
+            a.pos[at] = 0;
+            a.pos[plane + at] = 0;
+            a.pos[2 * plane + at] = 0;
+            continue;
+        }
+        const long long here = C.text0 + text_b + vadv;
+        if (cls[i] != prev) {
+            const int r = local0 + i;
+            rec_k[r] = C.k0 + kept_b;
+            rec_start[r] = here;
+            rec_cls[r] = cls[i];
+            rec_grid[r] = -1;
+            if (cls[i] != 0) {
+                const long long g = cls[i] == 1 ? (long long)C.img0 + img_b : (long long)C.vid0 + vid_b;
+                RiGrid gr;
+                rec_grid[r] = (int)g;
+                if (run_grid(a, cls[i], g, gr)) vadv += gr.adv;
+                img_b += cls[i] == 1;
+                vid_b += cls[i] == 2;
+            }
+        }
+        if (cls[i] == 0) {
+            if (here > INT_MAX) record_fault(a.status, kRiOverflow);
+            const int p = (int)min(here, (long long)INT_MAX);
+            a.pos[at] = p;
+            a.pos[plane + at] = p;
+            a.pos[2 * plane + at] = p;
+            mx = max(mx, (long long)p);
+            ++text_b;
+        }
+        ++kept_b;
+        prev = cls[i];
+    }
+    __syncthreads();
+
+    // pass 2: vision slots from their run's record
+    int rk = C.open_k, rgrid = C.open_grid, rcls = C.prev_cls > 0 ? C.prev_cls : 0;
+    long long rstart = C.open_start;
+    if (ex.last > 0) {
+        const int r = ex.last - 1;
+        rk = rec_k[r];
+        rgrid = rec_grid[r];
+        rcls = rec_cls[r];
+        rstart = rec_start[r];
+    }
+    RiGrid gr{0, 0, 0, 0};
+    bool have = rcls != 0 && run_grid(a, rcls, rgrid, gr);
+    kept_b = ex.kept;
+    prev = prev0;
+#pragma unroll
+    for (int i = 0; i < kRiPer; ++i) {
+        const long long l = l0 + i;
+        if (l >= a.L) break;
+        if (!kept[i]) continue;
+        const int k = C.k0 + kept_b;
+        if (cls[i] != prev) {
+            // the run that ends here must have filled its grid
+            if (rcls != 0 && (!have || (long long)(k - rk) != (long long)gr.t * gr.h * gr.w))
+                record_fault(a.status, kRiRunLength);
+            const int r = local0 + i;
+            rk = rec_k[r];
+            rgrid = rec_grid[r];
+            rcls = rec_cls[r];
+            rstart = rec_start[r];
+            have = rcls != 0 && run_grid(a, rcls, rgrid, gr);
+            if (rcls != 0 && !have) record_fault(a.status, kRiNoGrid);
+        }
+        if (cls[i] != 0) {
+            const long long at = b * a.L + l;
+            const long long off = k - rk;
+            const long long cells = (long long)gr.t * gr.h * gr.w;
+            long long tt = 0, row = 0, col = 0;
+            if (have && off < cells) {
+                const long long hw = (long long)gr.h * gr.w;
+                tt = off / hw;
+                const long long rem = off - tt * hw;
+                row = rem / gr.w;
+                col = rem - row * gr.w;
+            } else if (have) {
+                record_fault(a.status, kRiRunLength);
+            }
+            if (have && k == sample_kept - 1 && off + 1 != cells) record_fault(a.status, kRiRunLength);
+            const long long pt = rstart + tt, ph = rstart + row, pw = rstart + col;
+            const long long top = max(pt, max(ph, pw));
+            if (top > INT_MAX) record_fault(a.status, kRiOverflow);
+            a.pos[at] = (int)min(pt, (long long)INT_MAX);
+            a.pos[plane + at] = (int)min(ph, (long long)INT_MAX);
+            a.pos[2 * plane + at] = (int)min(pw, (long long)INT_MAX);
+            mx = max(mx, min(top, (long long)INT_MAX));
+        }
+        ++kept_b;
+        prev = cls[i];
+    }
+
+    // the tile's largest coordinate; the sample's last tile writes the delta
+    int m = (int)mx;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, d));
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kRiThreads / 32; ++w) m = max(m, warp_max[w]);
+        if (m >= 0) atomicMax(&smp[b].max_pos, m);
+        __threadfence();
+        if (atomicAdd(&smp[b].done, 1u) == (unsigned)a.tiles_per_row - 1) {
+            __threadfence();
+            const int top = atomicAdd(&smp[b].max_pos, 0);
+            a.deltas[b] = sample_kept > 0 ? top + 1 - sample_kept : 0;
+        }
+    }
+}
+
+cudaError_t launch_rope_index(const RopeIndexArgs &a, cudaStream_t s)
+{
+    const long long tiles = a.B * a.tiles_per_row;
+    if (tiles > 0) ri_tile_kernel<<<(unsigned)tiles, kRiThreads, 0, s>>>(a);
+    ri_carry_kernel<<<1, kRiCarryThreads, 0, s>>>(a);
+    if (tiles > 0) ri_write_kernel<<<(unsigned)tiles, kRiThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace ipe
