@@ -250,6 +250,30 @@ int ipe_mrope_rope_index(const void *mm_token_type_ids, const void *attention_ma
 size_t ipe_mrope_rope_index_workspace(int64_t B, int64_t L, int n_images, int n_videos);
 
 /* ---------------------------------------------------------------------------
+ * ipe_mrope_rope_index_static -- ipe_mrope_rope_index for callers that cannot
+ * supply device memory at call time (a serving loop that reserved all device
+ * memory up front and allows no allocation on its hot path, or a C host
+ * program without a device allocator).  No counterpart on the pages: this is
+ * an interface choice of this library, the computation is that of
+ * ipe_mrope_rope_index.
+ * Instead of a caller workspace it uses a scratch array of
+ * IPE_ROPE_INDEX_STATIC_BYTES compiled into the library, one per device; the
+ * call allocates no memory.  Sizes whose workspace
+ * (ipe_mrope_rope_index_workspace) exceeds that are rejected with IPE_ELIMIT.
+ * The first call on each device looks the array's address up (with that
+ * device current) and so does the set-up work: make it before any stream
+ * capture.  Nothing in the scratch needs clearing between calls.  All calls on
+ * one device share the array: calls whose kernels overlap in time (on other
+ * streams or from other host threads) race.  Arguments and results as
+ * ipe_mrope_rope_index without workspace / workspace_bytes.
+ * ------------------------------------------------------------------------- */
+#define IPE_ROPE_INDEX_STATIC_BYTES (4u << 20) /* 4 MiB: B * L up to about 40 million slots */
+int ipe_mrope_rope_index_static(const void *mm_token_type_ids, const void *attention_mask, int id_bytes,
+                                int64_t B, int64_t L, const void *image_grid_thw, int n_images,
+                                const void *video_grid_thw, int n_videos, int grid_bytes, int spatial_merge,
+                                int32_t *position_ids, int32_t *rope_deltas, void *stream);
+
+/* ---------------------------------------------------------------------------
  * Vision grids.  grid_thw_host is a host int32 [n_images, 3] array of
  * (t, h, w) patch grids BEFORE the spatial merge ([VLM] 1.1 Patch; [IRPE]
  * get_rope_index); h and w must be multiples of `merge` (spatial_merge_size,

@@ -41,6 +41,7 @@ _SIGS = {
                                _P]),
     "ipe_mrope_rope_index": (_I, [_P, _P, _I, _I64, _I64, _P, _I, _P, _I, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
     "ipe_mrope_rope_index_workspace": (ctypes.c_size_t, [_I64, _I64, _I, _I]),
+    "ipe_mrope_rope_index_static": (_I, [_P, _P, _I, _I64, _I64, _P, _I, _P, _I, _I, _I, _P, _P, _P]),
     "ipe_vis_interp_plan": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
     "ipe_vis_pos_interp": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P]),
     "ipe_vis_rope2d": (_I, [_P, _P, _I, _I64, _I, _I, _I64, _I64, _P, _I, _I, _D, _P]),
@@ -324,6 +325,41 @@ def mrope_rope_index(mm_token_type_ids, image_grid_thw=None, video_grid_thw=None
                                      n_img, _ptr(video_grid_thw), n_vid, gbytes, int(spatial_merge_size),
                                      _ptr(position_ids), _ptr(rope_deltas), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream)))
+    return position_ids, rope_deltas
+
+
+# Bytes of the library-owned scratch behind mrope_rope_index_static (per device).
+ROPE_INDEX_STATIC_BYTES = 4 << 20
+
+
+def mrope_rope_index_static(mm_token_type_ids, image_grid_thw, video_grid_thw, attention_mask, spatial_merge_size,
+                            position_ids, rope_deltas, stream=None):
+    """mrope_rope_index for callers that cannot allocate device memory at call
+    time: the outputs are the caller's, the scratch is a fixed buffer inside
+    the library (ROPE_INDEX_STATIC_BYTES per device), and nothing is allocated
+    here.  Calls on one device share that buffer, so calls that overlap in
+    time race; the first call on a device does a one-time set-up and should
+    come before any stream capture."""
+    ty = _int_tensor(mm_token_type_ids, "mm_token_type_ids")
+    if ty.dim() != 2:
+        raise ValueError("mm_token_type_ids must be [B, L]")
+    B, L = ty.shape
+    if attention_mask is not None:
+        _int_tensor(attention_mask, "attention_mask", (B, L))
+    grids = [g for g in (image_grid_thw, video_grid_thw) if g is not None]
+    for g in grids:
+        _int_tensor(g, "grid")
+    gbytes = grids[0].element_size() if grids else 4
+    n_img = 0 if image_grid_thw is None else image_grid_thw.shape[0]
+    n_vid = 0 if video_grid_thw is None else video_grid_thw.shape[0]
+    for t, nm, shp in ((position_ids, "position_ids", (3, B, L)), (rope_deltas, "rope_deltas", (B,))):
+        _cuda(t, nm)
+        if t.dtype != torch.int32 or tuple(t.shape) != shp or not t.is_contiguous():
+            raise ValueError(f"{nm} must be a contiguous int32 {shp} tensor")
+    _check(_lib.ipe_mrope_rope_index_static(_ptr(ty), _ptr(attention_mask), ty.element_size(), B, L,
+                                            _ptr(image_grid_thw), n_img, _ptr(video_grid_thw), n_vid, gbytes,
+                                            int(spatial_merge_size), _ptr(position_ids), _ptr(rope_deltas),
+                                            _stream(stream)))
     return position_ids, rope_deltas
 
 

@@ -322,6 +322,9 @@ bool tma_rot_args(const RotArgs &r, int eb, TmaRotArgs &t)
     return t.status != nullptr;
 }
 
+// Status and message for ipe_last_error, for entry points in other files.
+int set_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
 }  // namespace ipe
 
 extern "C" {
