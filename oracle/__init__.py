@@ -46,6 +46,7 @@ class Oracle:
             "orc_vis_rotary_cos_sin": (_I, [_P, _I64, _I, _D, _P, _P]),
             "orc_rms_norm": (_I, [_P, _I64, _I, _P, _D, _I, _P]),
             "orc_rope_index": (_I, [_P, _P, _I, _I64, _P, _I, _P, _I, _I, _P, _P]),
+            "orc_decode_positions": (_I, [_P, _I, _I64, _P, _I64, _P, _P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -149,6 +150,21 @@ class Oracle:
         if rc:
             raise ValueError("rope_index: bad arguments")
         return pos, deltas
+
+    def decode_positions(self, n_new, mask=None, cache_len=None, deltas=None):
+        """Positions [3, B, n_new] of the newest n_new tokens of each sample,
+        from the padding mask [B, S] (or the cache lengths [B]) and the rope
+        deltas [B]."""
+        mk = None if mask is None else np.ascontiguousarray(mask, np.int64)
+        cl = None if cache_len is None else np.ascontiguousarray(cache_len, np.int64)
+        B = mk.shape[0] if mk is not None else cl.shape[0]
+        S = mk.shape[1] if mk is not None else 0
+        dl = None if deltas is None else np.ascontiguousarray(deltas, np.int64)
+        pos = np.zeros((3, B, n_new), np.int64)
+        if self._lib.orc_decode_positions(None if mk is None else _ptr(mk), B, S, None if cl is None else _ptr(cl),
+                                          int(n_new), None if dl is None else _ptr(dl), _ptr(pos)):
+            raise ValueError("decode_positions: bad arguments")
+        return pos
 
     # -------------------------------------------------------------- vision
     def grid_patches(self, grid_thw, merge):

@@ -648,3 +648,39 @@ int orc_rope_index(const int64_t *types, const int64_t *mask, int B, int64_t L, 
     free(table);
     return rc;
 }
+
+/* ------------------------------------------------------------------------
+ * Positions of the tokens of a generation step, from the sequence index and
+ * the rope deltas saved at prefill.
+ * [IRPE] compute_3d_position_ids(), "recovering the positions": with a
+ * padding mask the sequence index is cumsum(mask, -1) - 1 with the padded
+ * slots set to 0; without one it is arange from the cache length.  The index
+ * is expanded to three rows and the sample's delta is added; all three axes
+ * then carry the same text position.
+ * mask: [B][S] over the whole sequence so far, the n_new new tokens last (or
+ * NULL: cache_len[b] + i); deltas: [B] (or NULL: 0); pos: [3][B][n_new].
+ * ---------------------------------------------------------------------- */
+int orc_decode_positions(const int64_t *mask, int B, int64_t S, const int64_t *cache_len, int64_t n_new,
+                         const int64_t *deltas, int64_t *pos)
+{
+    if (B < 0 || n_new < 0 || (mask != NULL && (S < n_new)) || (mask == NULL && cache_len == NULL))
+        return -1;
+    for (int b = 0; b < B; ++b) {
+        int64_t run = 0;   /* cumsum of the mask up to the current slot */
+        for (int64_t i = 0; i < (mask ? S : n_new); ++i) {
+            int64_t seq;
+            if (mask) {
+                run += mask[(int64_t)b * S + i];
+                seq = mask[(int64_t)b * S + i] == 0 ? 0 : run - 1;
+                if (i < S - n_new)
+                    continue;
+            } else {
+                seq = cache_len[b] + i;
+            }
+            int64_t col = mask ? i - (S - n_new) : i;
+            for (int a = 0; a < 3; ++a)
+                pos[((int64_t)a * B + b) * n_new + col] = seq + (deltas ? deltas[b] : 0);
+        }
+    }
+    return 0;
+}

@@ -469,4 +469,34 @@ def pin_rope_index_errors(o):
         raise AssertionError(f"accepted {args}")
 
 
+def pin_decode_continues_prefill(o):
+    # The delta saved at prefill is the next rotary position minus the kept
+    # length, so the first generated token lands one past the largest prefill
+    # coordinate on all three axes.
+    rng = _rng(23)
+    types, mask, img, vid = _random_batch(rng, 5)
+    pos, deltas = o.rope_index(types, mask, img, vid, 2)
+    grown = np.concatenate([mask, np.ones((mask.shape[0], 1), np.int64)], axis=1)
+    nxt = o.decode_positions(1, mask=grown, deltas=deltas)[:, :, 0]
+    for b in range(types.shape[0]):
+        top = pos[:, b][:, mask[b] == 1].max()
+        assert (nxt[:, b] == top + 1).all(), (b, nxt[:, b], top)
+    # the same from cache lengths (no padding): the kept length is the cache length
+    nxt2 = o.decode_positions(1, cache_len=mask.sum(1), deltas=deltas)[:, :, 0]
+    assert (nxt2 == nxt).all()
+
+
+def pin_decode_closed_forms(o):
+    # cache lengths: arange from the length, plus the delta, on all rows
+    got = o.decode_positions(3, cache_len=[5, 0], deltas=[-2, 7])
+    assert (got == np.array([[3, 4, 5], [7, 8, 9]])[None]).all()
+    # mask with left padding: the sequence index counts kept slots only
+    mask = [[0, 0, 1, 1, 1], [1, 1, 1, 1, 1]]
+    got = o.decode_positions(2, mask=mask, deltas=[0, 10])
+    assert (got == np.array([[1, 2], [13, 14]])[None]).all()
+    # a padded new slot sits at 0 before the delta
+    got = o.decode_positions(1, mask=[[1, 1, 0]], deltas=[4])
+    assert (got[:, 0, 0] == 4).all()
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

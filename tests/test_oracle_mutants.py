@@ -70,6 +70,11 @@ MUTANTS = {
     "rope_hw_swap": ("table[1 * n + cols] = hh + cur;", "table[1 * n + cols] = ww + cur;"),
     # position table: delta taken against the padded length
     "rope_delta_padded": ("deltas[b] = n > 0 ? mx + 1 - n : 0;", "deltas[b] = n > 0 ? mx + 1 - L : 0;"),
+    # decode positions: cumsum taken as the index (no - 1)
+    "decode_cumsum": ("seq = mask[(int64_t)b * S + i] == 0 ? 0 : run - 1;",
+                      "seq = mask[(int64_t)b * S + i] == 0 ? 0 : run;"),
+    # decode positions: the rope delta not added
+    "decode_no_delta": ("= seq + (deltas ? deltas[b] : 0);", "= seq;"),
     # position table: image temporal index dropped
     "rope_image_time": ("table[0 * n + cols] = tt * 1 + cur;", "table[0 * n + cols] = cur;"),
 }
