@@ -81,8 +81,9 @@ int ipe_version(void);
  * This call synchronises `stream`, reads and clears that word, and returns
  * IPE_OK, or IPE_EDEVICE with a message naming the wait that gave up (the
  * results of the failed launch are then incomplete).  ipe_mrope_rope_index
- * reports inputs that only the device can see the same way (codes 16 .. 20,
- * listed there).  Not part of any page: failure reporting of this library.
+ * and ipe_mrope_decode report inputs that only the device can see the same
+ * way (codes 16 .. 22, listed there).  Not part of any page: failure
+ * reporting of this library.
  * ------------------------------------------------------------------------- */
 int ipe_device_status(void *stream);
 
@@ -198,6 +199,42 @@ int ipe_qk_norm_mrope(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int 
                       const void *k_weight, float eps, const int32_t *positions,
                       const float *inv_freq_host, int rot_dim, const int32_t *section,
                       int interleaved, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * ipe_mrope_decode -- one generation step: for each of B sequences one new
+ * token, its position recovered from the sequence index and the rope delta,
+ * optional QK-RMSNorm, q and k rotated in place, and the rotated k and v
+ * written to their KV-cache slots, in one launch.
+ * [IRPE] compute_3d_position_ids() ("recovering the positions": sequence
+ * index, expanded to three rows, plus the sample's delta); [M01] follow-up
+ * questions (decode cos / sin of a single token):
+ *   p[b] = seq_pos[b] + rope_deltas[b]      the same on all three axes, so the
+ *                                           axis layout (section) plays no part
+ *   angle[j] = fl32(fl32(p) * inv_freq[j]); rotation as ipe_mrope_apply
+ * seq_pos is the new token's sequence index: cumsum(attention_mask)[-1] - 1
+ * with a padding mask, else the cache length before the token.
+ *   q, k        device, dtype, [B, hq, head_dim] / [B, hk, head_dim], token
+ *               strides q_tok_stride / k_tok_stride (elements), rewritten in place
+ *   v           device [B, hk, head_dim], token stride v_tok_stride; read only
+ *               when v_cache is given (else may be NULL)
+ *   seq_pos     device int32 [B]; rope_deltas device int32 [B] or NULL (0)
+ *   q_weight, k_weight  device [head_dim] of dtype, or both NULL: no norm;
+ *               with them every q / k row is RMS-normalised first, as
+ *               ipe_qk_norm_mrope (eps >= 0)
+ *   k_cache, v_cache  device rows of [hk, head_dim] at slot * cache_slot_stride
+ *               (elements), num_slots slots; v_cache may be NULL
+ *   slot_mapping  device int64 [B]: cache slot of each new token, < 0 = no
+ *               write (padding); NULL: no cache write (then both caches NULL)
+ * head_dim, rot_dim and alignment as ipe_qk_norm_mrope (q, k, v, caches,
+ * weights and all strides 16-byte aligned).  Reported through
+ * ipe_device_status: 21 a position outside [0, 2^24); 22 a slot at or beyond
+ * num_slots (that write is skipped).
+ * ------------------------------------------------------------------------- */
+int ipe_mrope_decode(void *q, void *k, const void *v, ipe_dtype dtype, int64_t B, int hq, int hk, int head_dim,
+                     int64_t q_tok_stride, int64_t k_tok_stride, int64_t v_tok_stride, const int32_t *seq_pos,
+                     const int32_t *rope_deltas, const void *q_weight, const void *k_weight, float eps,
+                     const float *inv_freq_host, int rot_dim, void *k_cache, void *v_cache,
+                     int64_t cache_slot_stride, int64_t num_slots, const int64_t *slot_mapping, void *stream);
 
 /* ---------------------------------------------------------------------------
  * ipe_mrope_rope_index -- three-axis position table and rope deltas of a batch

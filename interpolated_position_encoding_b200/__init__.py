@@ -39,6 +39,8 @@ _SIGS = {
     "ipe_mrope_apply": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, _I, _P, _I, _P]),
     "ipe_qk_norm_mrope": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, ctypes.c_float, _P, _P, _I, _P, _I,
                                _P]),
+    "ipe_mrope_decode": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _I64, _P, _P, _P, _P, ctypes.c_float, _P,
+                              _I, _P, _P, _I64, _I64, _P, _P]),
     "ipe_mrope_rope_index": (_I, [_P, _P, _I, _I64, _I64, _P, _I, _P, _I, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
     "ipe_mrope_rope_index_workspace": (ctypes.c_size_t, [_I64, _I64, _I, _I]),
     "ipe_mrope_rope_index_static": (_I, [_P, _P, _I, _I64, _I64, _P, _I, _P, _I, _I, _I, _P, _P, _P]),
@@ -265,6 +267,51 @@ def qk_norm_mrope(q, k, q_weight, k_weight, positions, inv_freq, section, interl
     _check(_lib.ipe_qk_norm_mrope(_ptr(q), _ptr(k), dt, T, hq, hk, D, qs, ks, _ptr(q_weight), _ptr(k_weight),
                                   float(eps), _ptr(positions), inv, 2 * half, _i32_host(section, 3),
                                   int(bool(interleaved)), _stream(stream)))
+    return q, k
+
+
+def mrope_decode(q, k, seq_pos, inv_freq, rope_deltas=None, v=None, q_weight=None, k_weight=None, eps=1e-6,
+                 k_cache=None, v_cache=None, slot_mapping=None, stream=None):
+    """One generation step, in place: q [B, hq, D] and k [B, hk, D] (any
+    token stride, contiguous heads) rotated at positions seq_pos + rope_deltas
+    (int32 [B] each), after an optional QK-RMSNorm (q_weight, k_weight); with
+    slot_mapping (int64 [B], < 0 = skip) the rotated k rows and the v rows are
+    written to k_cache / v_cache ([num_slots, hk, D] views, any slot stride)."""
+    dt, B, hq, hk, D, qs, ks = _qk_args(q, k)
+    for t, nm in ((seq_pos, "seq_pos"), (rope_deltas, "rope_deltas")):
+        if t is not None:
+            _cuda(t, nm)
+            if t.dtype != torch.int32 or tuple(t.shape) != (B,) or not t.is_contiguous():
+                raise ValueError(f"{nm} must be a contiguous int32 [{B}] tensor")
+    ref = q if q is not None else k
+    for w, nm in ((q_weight, "q_weight"), (k_weight, "k_weight")):
+        if w is not None:
+            _cuda(w, nm)
+            if w.dtype != ref.dtype or tuple(w.shape) != (D,) or not w.is_contiguous():
+                raise ValueError(f"{nm} must be a contiguous [{D}] tensor of the activation dtype")
+    vs = 0
+    if v is not None:
+        _cuda(v, "v")
+        vs = _row_stride(v, hk, D, "v")
+        if v.shape[0] != B or v.dtype != ref.dtype:
+            raise ValueError("v must be [B, hk, D] of the activation dtype")
+    cs, nslots = 0, 0
+    if k_cache is not None:
+        _cuda(k_cache, "k_cache")
+        cs = _row_stride(k_cache, hk, D, "k_cache")
+        nslots = k_cache.shape[0]
+        if v_cache is not None:
+            _cuda(v_cache, "v_cache")
+            if _row_stride(v_cache, hk, D, "v_cache") != cs or v_cache.shape[0] != nslots:
+                raise ValueError("v_cache must match k_cache in shape and slot stride")
+    if slot_mapping is not None:
+        _cuda(slot_mapping, "slot_mapping")
+        if slot_mapping.dtype != torch.int64 or tuple(slot_mapping.shape) != (B,) or not slot_mapping.is_contiguous():
+            raise ValueError(f"slot_mapping must be a contiguous int64 [{B}] tensor")
+    inv, half = _inv_host(inv_freq)
+    _check(_lib.ipe_mrope_decode(_ptr(q), _ptr(k), _ptr(v), dt, B, hq, hk, D, qs, ks, vs, _ptr(seq_pos),
+                                 _ptr(rope_deltas), _ptr(q_weight), _ptr(k_weight), float(eps), inv, 2 * half,
+                                 _ptr(k_cache), _ptr(v_cache), cs, nslots, _ptr(slot_mapping), _stream(stream)))
     return q, k
 
 

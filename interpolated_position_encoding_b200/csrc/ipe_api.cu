@@ -350,6 +350,8 @@ int ipe_device_status(void *stream)
                      : v == 18 ? "position table: a kept slot has a type other than 0, 1, 2, 3"
                      : v == 19 ? "position table: a grid has t, h or w outside 1 .. 32768"
                      : v == 20 ? "position table: a coordinate beyond the int32 range"
+                     : v == 21 ? "decode: seq_pos + rope delta outside [0, 2^24)"
+                     : v == 22 ? "decode: a cache slot at or beyond num_slots (that write was skipped)"
                               : "unknown";
     return fail(IPE_EDEVICE, "device fault %u: %s", v, what);
 }
@@ -513,6 +515,90 @@ int ipe_qk_norm_mrope(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int 
     n.eps = eps;
     cudaError_t e = launch_qk_norm_mrope(dtype == IPE_BF16, n, a, (cudaStream_t)stream);
     return e == cudaSuccess ? ok() : cuda_fail(e, "qk_norm_mrope launch");
+}
+
+int ipe_mrope_decode(void *q, void *k, const void *v, ipe_dtype dtype, int64_t B, int hq, int hk, int head_dim,
+                     int64_t q_tok_stride, int64_t k_tok_stride, int64_t v_tok_stride, const int32_t *seq_pos,
+                     const int32_t *rope_deltas, const void *q_weight, const void *k_weight, float eps,
+                     const float *inv_freq_host, int rot_dim, void *k_cache, void *v_cache, int64_t cache_slot_stride,
+                     int64_t num_slots, const int64_t *slot_mapping, void *stream)
+{
+    if (int rc = check_dtype(dtype)) return rc;
+    const int eb = elem_bytes(dtype), ec = 16 / eb;
+    if (head_dim <= 0 || head_dim % ec) return fail(IPE_EINVAL, "head_dim %d must be a multiple of %d", head_dim, ec);
+    const int lpr = head_dim / ec;
+    if (lpr < 2 || lpr > 32 || (lpr & (lpr - 1)))
+        return fail(IPE_ELIMIT, "head_dim %d: %d-element chunks per row must be a power of two in 2 .. 32", head_dim, ec);
+    if (rot_dim < 2 || rot_dim % 2 || rot_dim > head_dim)
+        return fail(IPE_EINVAL, "rot_dim %d must be even and in 2 .. head_dim", rot_dim);
+    if ((rot_dim / 2) % ec) return fail(IPE_EINVAL, "rot_dim / 2 = %d must be a multiple of %d", rot_dim / 2, ec);
+    if (int rc = check_half(rot_dim / 2)) return rc;
+    if (inv_freq_host == nullptr) return fail(IPE_EINVAL, "inv_freq_host is NULL");
+    MropeAngles a{};
+    for (int j = 0; j < rot_dim / 2; ++j) {
+        if (!std::isfinite(inv_freq_host[j])) return fail(IPE_EINVAL, "inv_freq[%d] is not finite", j);
+        a.inv[j] = inv_freq_host[j];
+    }
+    if ((q_weight == nullptr) != (k_weight == nullptr)) return fail(IPE_EINVAL, "give both norm weights or neither");
+    if (q_weight && (!(eps >= 0.f) || !std::isfinite(eps))) return fail(IPE_EINVAL, "eps must be finite and >= 0");
+    const bool cache = slot_mapping != nullptr;
+    if (!cache && (k_cache || v_cache)) return fail(IPE_EINVAL, "caches given without slot_mapping");
+    if (cache && hk > 0 && k_cache == nullptr) return fail(IPE_EINVAL, "slot_mapping given without k_cache");
+    if (v_cache && v == nullptr) return fail(IPE_EINVAL, "v_cache given without v");
+    if (cache && (num_slots < 0 || cache_slot_stride < (long long)hk * head_dim))
+        return fail(IPE_EINVAL, "num_slots must be >= 0 and cache_slot_stride >= hk * head_dim");
+    if (int rc = check_qk(q, k, dtype, B, hq, hk, head_dim, q_tok_stride, k_tok_stride, "q", "k")) return rc;
+    if (v_cache && hk > 0 && v_tok_stride < (long long)hk * head_dim)
+        return fail(IPE_EINVAL, "v row stride %lld < heads * head_dim", (long long)v_tok_stride);
+    if ((hq && (q_tok_stride % ec || !aligned(q, 16))) || (hk && (k_tok_stride % ec || !aligned(k, 16))) ||
+        (v_cache && (v_tok_stride % ec || !aligned(v, 16))) ||
+        (cache && (cache_slot_stride % ec || !aligned(k_cache, 16) || !aligned(v_cache, 16))) ||
+        !aligned(q_weight, 16) || !aligned(k_weight, 16) || !aligned(seq_pos, 4) || !aligned(rope_deltas, 4) ||
+        !aligned(slot_mapping, 8))
+        return fail(IPE_EALIGN, "q, k, v, caches, weights and their strides must be 16-byte aligned");
+    if (B == 0 || hq + hk == 0) return ok();
+    if (int rc = check_dev(seq_pos, (size_t)B * 4, "seq_pos")) return rc;
+    if (rope_deltas) {
+        if (int rc = check_dev(rope_deltas, (size_t)B * 4, "rope_deltas")) return rc;
+    }
+    if (q_weight) {
+        if (int rc = check_dev(q_weight, (size_t)head_dim * eb, "q_weight")) return rc;
+        if (int rc = check_dev(k_weight, (size_t)head_dim * eb, "k_weight")) return rc;
+    }
+    if (cache && hk > 0) {
+        if (int rc = check_dev(slot_mapping, (size_t)B * 8, "slot_mapping")) return rc;
+        const size_t span = num_slots > 0 ? ((size_t)(num_slots - 1) * cache_slot_stride + (size_t)hk * head_dim) * eb : 0;
+        if (int rc = check_dev(k_cache, span, "k_cache")) return rc;
+        if (v_cache) {
+            if (int rc = check_dev(v_cache, span, "v_cache")) return rc;
+            if (int rc = check_dev(v, ((size_t)(B - 1) * v_tok_stride + (size_t)hk * head_dim) * eb, "v")) return rc;
+        }
+    }
+    DecodeArgs d{};
+    d.q = hq ? q : nullptr;
+    d.k = hk ? k : nullptr;
+    d.v = (v_cache && hk) ? v : nullptr;
+    d.k_cache = (cache && hk) ? k_cache : nullptr;
+    d.v_cache = (cache && hk) ? v_cache : nullptr;
+    d.slots = (cache && hk) ? slot_mapping : nullptr;
+    d.seq_pos = seq_pos;
+    d.deltas = rope_deltas;
+    d.q_weight = q_weight;
+    d.k_weight = k_weight;
+    d.B = B;
+    d.q_stride = q_tok_stride;
+    d.k_stride = k_tok_stride;
+    d.v_stride = v_tok_stride;
+    d.cache_stride = cache_slot_stride;
+    d.hq = hq;
+    d.hk = hk;
+    d.head_dim = head_dim;
+    d.half = rot_dim / 2;
+    d.eps = eps;
+    d.status = device_status_word();
+    if (!d.status) return fail(IPE_ECUDA, "device status word unavailable");
+    cudaError_t e = launch_mrope_decode(dtype == IPE_BF16, d, a, num_slots, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "mrope_decode launch");
 }
 
 static int rope_index_sizes(int64_t B, int64_t L, int n_images, int n_videos)

@@ -110,6 +110,27 @@ struct QkNormArgs {
 
 cudaError_t launch_qk_norm_mrope(bool bf16, const QkNormArgs &n, const MropeAngles &a, cudaStream_t s);
 
+// One generation step (ipe_mrope_decode): per sequence one new token whose
+// position is seq_pos + delta on all three axes; optional QK-RMSNorm; q and k
+// rotated in place; k (rotated) and v written to their cache slots.
+struct DecodeArgs {
+    void *q, *k;                      // [B, hq, D], [B, hk, D], rewritten in place
+    const void *v;                    // [B, hk, D] or NULL
+    void *k_cache, *v_cache;          // rows of [hk, D] at slot * cache_stride, or NULL
+    const int64_t *slots;             // [B] cache slot of each new token (< 0: none) or NULL
+    const int32_t *seq_pos;           // [B] sequence index of the new token
+    const int32_t *deltas;            // [B] rope deltas or NULL
+    const void *q_weight, *k_weight;  // [D] norm weights, or both NULL (no norm)
+    long long B;
+    long long q_stride, k_stride, v_stride, cache_stride;   // elements
+    int hq, hk, head_dim, half;
+    float eps;
+    unsigned *status;
+};
+
+cudaError_t launch_mrope_decode(bool bf16, const DecodeArgs &d, const MropeAngles &a, long long num_slots,
+                                cudaStream_t s);
+
 // ------------------------------------------------------- position table
 // Tile of the position-table kernels: 256 threads x 4 consecutive slots.
 constexpr int kRiThreads = 256;

@@ -12,7 +12,7 @@
 // (EC elements = 16 bytes per lane), its sum of squares reduced with
 // shuffles inside those lanes, and the rotary partner of a chunk fetched from
 // the lane half a rotary slice away.  All D channels are written back.
-#include "ipe_rotary_tma.cuh"
+#include "ipe_chunk.cuh"
 
 namespace ipe {
 
@@ -25,59 +25,10 @@ namespace ipe {
 constexpr int kQkWarps = 8;
 constexpr int kQkUnroll = IPE_QK_UNROLL;     // head rows per lane in flight
 
-template <typename T> struct QkElem;
-template <> struct QkElem<__nv_bfloat16> {
-    static constexpr int EC = 8;
-};
-template <> struct QkElem<float> {
-    static constexpr int EC = 4;
-};
-
-// A 16-byte chunk (4 words) as EC/2 fp32 pairs, and back (one rounding to
-// the dtype per element).
-template <typename T> __device__ __forceinline__ void chunk_to_pairs(const uint32_t *w, float2 *p);
-template <> __device__ __forceinline__ void chunk_to_pairs<__nv_bfloat16>(const uint32_t *w, float2 *p)
-{
-#pragma unroll
-    for (int i = 0; i < 4; ++i) p[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
-}
-template <> __device__ __forceinline__ void chunk_to_pairs<float>(const uint32_t *w, float2 *p)
-{
-#pragma unroll
-    for (int i = 0; i < 2; ++i) p[i] = make_float2(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]));
-}
-template <typename T> __device__ __forceinline__ void pairs_to_chunk(const float2 *p, uint32_t *w);
-template <> __device__ __forceinline__ void pairs_to_chunk<__nv_bfloat16>(const float2 *p, uint32_t *w)
-{
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 b = __floats2bfloat162_rn(p[i].x, p[i].y);
-        w[i] = *reinterpret_cast<const uint32_t *>(&b);
-    }
-}
-template <> __device__ __forceinline__ void pairs_to_chunk<float>(const float2 *p, uint32_t *w)
-{
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        w[2 * i] = __float_as_uint(p[i].x);
-        w[2 * i + 1] = __float_as_uint(p[i].y);
-    }
-}
-
-// Product of two bf16 pairs rounded once to bf16 (the exact product of two
-// bf16 values fits in fp32, so this equals rounding the fp32 product).
-__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b)
-{
-    uint32_t d;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
 template <typename T, int LPR>
 __global__ void __launch_bounds__(32 * kQkWarps, IPE_QK_MIN_BLOCKS)
     qk_norm_mrope_kernel(const __grid_constant__ QkNormArgs n, const __grid_constant__ MropeAngles a)
 {
-    constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr int EC = QkElem<T>::EC;
     constexpr int NP = EC / 2;                        // fp32 pairs of a 16-byte chunk
     constexpr int RPW = 32 / LPR;                     // head rows per warp access
@@ -147,41 +98,12 @@ __global__ void __launch_bounds__(32 * kQkWarps, IPE_QK_MIN_BLOCKS)
                 // every lane of the warp takes part in the shuffles, rows past
                 // H included (zeros; never stored)
                 const int h = h0 + u * RPW + sub;
-                float2 xv[NP];
-                chunk_to_pairs<T>(x[u].v, xv);
-                float2 acc = mul2(xv[0], xv[0]);
-#pragma unroll
-                for (int i = 1; i < NP; ++i) acc = fma2(xv[i], xv[i], acc);
-                float ss = __fadd_rn(acc.x, acc.y);
-#pragma unroll
-                for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off, LPR);
-                const float r = __frsqrt_rn(__fadd_rn(__fmul_rn(ss, inv_d), n.eps));
                 const bool is_q = h < n.hq;
-                // y = dtype(dtype(x r) * w): cast back first, then the weight
-                const float2 r2 = make_float2(r, r);
+                uint32_t w[4];
 #pragma unroll
-                for (int i = 0; i < NP; ++i) xv[i] = mul2(xv[i], r2);
-                Pack<uint32_t, 4> y;
-                pairs_to_chunk<T>(xv, y.v);
-                if constexpr (BF16) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) y.v[i] = mul_bf16x2(y.v[i], is_q ? wq.v[i] : wk.v[i]);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        y.v[i] = __float_as_uint(__fmul_rn(__uint_as_float(y.v[i]), __uint_as_float(is_q ? wq.v[i] : wk.v[i])));
-                }
-                Pack<uint32_t, 4> yp;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) yp.v[i] = __shfl_sync(0xffffffffu, y.v[i], partner);
-                // y[j] cos - y[j+h] sin ; y[j+h] cos + y[j] sin, the sign in si
-                float2 yv[NP], pv[NP];
-                chunk_to_pairs<T>(y.v, yv);
-                chunk_to_pairs<T>(yp.v, pv);
-#pragma unroll
-                for (int i = 0; i < NP; ++i) yv[i] = fma2(yv[i], co[i], mul2(pv[i], si[i]));
-                Pack<uint32_t, 4> o;
-                pairs_to_chunk<T>(yv, o.v);
+                for (int i = 0; i < 4; ++i) w[i] = is_q ? wq.v[i] : wk.v[i];
+                const Pack<uint32_t, 4> y = rms_norm_chunk<T, LPR>(x[u], w, inv_d, n.eps);
+                const Pack<uint32_t, 4> o = rotate_row_chunk<T>(y, co, si, partner);
                 if (h < H) st_pack<uint32_t, 4>(chunk_ptr(h), o);
             }
         }
