@@ -49,6 +49,11 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-variant side measurements")
     ap.add_argument("--extras-reps", type=int, default=20, help="timed repetitions of each side measurement")
+    ap.add_argument("--scale-down", type=int, default=1, choices=[1, 2, 4, 8, 16],
+                    help="run the step on 1/K of the tokens and video frames (profiling captures; implies "
+                         "--no-e2e --no-cpu-baseline --no-extras)")
+    ap.add_argument("--case", choices=sorted(CASES),
+                    help="time one kernel on its own case instead of the step (profiling captures)")
     return ap.parse_args()
 
 
@@ -283,6 +288,81 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------ single-kernel cases
+
+CASES = {
+    "qk_norm_mrope": "fused QK-RMSNorm + MRoPE on text_t32768_omni (Q [32768, 32, 128], K [32768, 4, 128] bf16)",
+    "rope_index": "device position table of the large-prefill request (B = 1, L = 131072, 16 video slices)",
+    "mrope_decode": "decode step, B = 256, Q [256, 24, 256], K / V [256, 4, 256] bf16, norm + KV-cache write",
+}
+
+
+def run_case(args):
+    """--case NAME: `--warmup` untimed and `--steps` timed launches of one
+    kernel on its case (inputs resident, no L2 flush); one JSON line."""
+    import numpy as np
+    import torch
+    import interpolated_position_encoding_b200 as ipe
+    import workloads as wl
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    name = args.case
+    if name == "qk_norm_mrope":
+        w = wl.WORKLOADS["text_t32768_omni"]
+        t = w.text
+        tin = wl.text_inputs(w)
+        Q = torch.from_numpy(tin["q"].view(np.int16)).view(torch.bfloat16).to(dev)
+        K = torch.from_numpy(tin["k"].view(np.int16)).view(torch.bfloat16).to(dev)
+        pos = torch.from_numpy(tin["positions"]).to(dev)
+        wq = torch.ones(t.head_dim, dtype=torch.bfloat16, device=dev)
+        inv = ipe.rope_inv_freq(t.rot_dim, t.theta)
+        fn = lambda: ipe.qk_norm_mrope(Q, K, wq, wq, pos, inv, t.section, True, stream=stream)  # noqa: E731
+        nbytes = (t.hq + t.hk) * t.T * t.head_dim * 2 * 2 + 3 * t.T * 4
+    elif name == "rope_index":
+        t = wl.WORKLOADS[WORKLOAD].text
+        types, vid = _segment_types(t.segments, t.merge)
+        gty, gvg = torch.from_numpy(types).to(dev), torch.from_numpy(vid).to(dev)
+        B, L = types.shape
+        posb = torch.empty(3, B, L, dtype=torch.int32, device=dev)
+        dl = torch.empty(B, dtype=torch.int32, device=dev)
+        ws = torch.empty(ipe.rope_index_workspace_bytes(B, L, 0, vid.shape[0]), dtype=torch.uint8, device=dev)
+        fn = lambda: ipe.mrope_rope_index(gty, None, gvg, None, t.merge, posb, dl, ws, stream=stream)  # noqa: E731
+        nbytes = B * L * 16 + B * 4
+    else:
+        t = wl.WORKLOADS[WORKLOAD].text
+        B, D = 256, t.head_dim
+        g = torch.Generator(device=dev).manual_seed(B)
+        q = torch.randn(B, t.hq, D, device=dev, generator=g).to(torch.bfloat16)
+        k = torch.randn(B, t.hk, D, device=dev, generator=g).to(torch.bfloat16)
+        v = torch.randn(B, t.hk, D, device=dev, generator=g).to(torch.bfloat16)
+        wq = torch.ones(D, dtype=torch.bfloat16, device=dev)
+        kc = torch.zeros(B * 1024, t.hk, D, dtype=torch.bfloat16, device=dev)
+        vc = torch.zeros_like(kc)
+        seq = torch.randint(2000, 100000, (B,), dtype=torch.int32, device=dev, generator=g)
+        dl = torch.randint(-2000, 0, (B,), dtype=torch.int32, device=dev, generator=g)
+        sm = torch.arange(B, device=dev, dtype=torch.int64) * 1024 + seq.long() % 1024
+        inv = ipe.rope_inv_freq(t.rot_dim, t.theta)
+        fn = lambda: ipe.mrope_decode(q, k, seq, inv, dl, v=v, q_weight=wq, k_weight=wq, k_cache=kc,  # noqa: E731
+                                      v_cache=vc, slot_mapping=sm, stream=stream)
+        nbytes = B * (t.hq + t.hk) * D * 2 * 2 + B * t.hk * D * 2 * 3 + B * 16 + 2 * D * 2
+    for _ in range(max(args.warmup, 0)):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ipe.device_status(stream)
+    ms = a.elapsed_time(b) / max(args.steps, 1)
+    peak, _ = measured_peaks()
+    print(json.dumps({"case": name, "what": CASES[name], "steps": args.steps, "warmup": args.warmup, "ms": ms,
+                      "alg_bytes": nbytes, "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / peak,
+                      "l2": "not flushed (inputs stay resident between launches)"}), flush=True)
+
+
 # ---------------------------------------------------------------- the GPU
 
 
@@ -290,6 +370,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return reference_arm(args)
+    if args.case:
+        return run_case(args)
 
     import numpy as np
     import torch
@@ -310,11 +392,24 @@ def main():
 
     w = wl.WORKLOADS[WORKLOAD]
     t, v = w.text, w.vision
-    N = wl.n_patches(v)
 
     # ---- inputs (host, seeded; rank r > 0 shifts the stream by r)
     tin = wl.text_inputs(w)
     vin = wl.vision_inputs(w)
+    if args.scale_down > 1:
+        # the first 1/K of the request: its tokens and its first video frames
+        import dataclasses
+        f = args.scale_down
+        Tn = t.T // f
+        frames, gh, gw = v.grid_thw[0]
+        Nn = frames // f * gh * gw
+        tin = {"positions": np.ascontiguousarray(tin["positions"][:, :Tn]), "q": tin["q"][:Tn], "k": tin["k"][:Tn]}
+        vin = dict(vin, q=vin["q"][:Nn], k=vin["k"][:Nn])
+        t = dataclasses.replace(t, T=Tn)
+        v = dataclasses.replace(v, grid_thw=[(frames // f, gh, gw)])
+        w = dataclasses.replace(w, text=t, vision=v)
+        args.no_e2e = args.no_cpu_baseline = args.no_extras = True
+    N = wl.n_patches(v)
     if rank:
         rng = np.random.default_rng(rank)
         tin["q"] = np.roll(tin["q"], int(rng.integers(1, 1000)), axis=0)
@@ -387,7 +482,8 @@ def main():
                    "frac": alg[n] / kernel_ms[n] / 1e6 / peak} for n in names}
     dom = max(names, key=lambda n: kernel_ms[n])
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak, "unit": "GB/s",
-                "frac": kernels[dom]["frac"], "traffic": dram_traffic(dom), "alg_bytes": alg[dom],
+                "frac": kernels[dom]["frac"], "traffic": dram_traffic(dom) if args.scale_down == 1 else None,
+                "alg_bytes": alg[dom],
                 "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured" else
                 "fallback 6650 GB/s"}
 
@@ -397,6 +493,7 @@ def main():
         extras = side_measurements(ipe, w, dev, stream, Q, K, pos, inv, table, qv, kv, out, alg, peak,
                                    args.extras_reps)
         extras["workloads"] = per_workload(ipe, dev, stream, peak, args.extras_reps)
+        extras["next"] = next_rows(ipe, dev, stream, peak, args.extras_reps)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -411,7 +508,8 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "tokens_per_step": t.T, "patches_per_step": N,
+        "config": {"workload": WORKLOAD if args.scale_down == 1 else f"{WORKLOAD} at 1/{args.scale_down}",
+                   "tokens_per_step": t.T, "patches_per_step": N,
                    "text": f"Q [{t.T},{t.hq},{t.head_dim}] K [{t.T},{t.hk},{t.head_dim}] bf16, rot {t.rot_dim}, "
                            f"theta {t.theta:g}, section {list(t.section)} interleaved, fused mrope_apply",
                    "vision": f"grid_thw {grid}, table [{v.grid_side ** 2},{v.hidden}] bf16, q/k [{N},{v.heads},"
@@ -555,6 +653,83 @@ def per_workload(ipe, dev, stream, peak, reps):
         res[name] = r
         torch.cuda.empty_cache()
     ipe.device_status(stream)
+    return res
+
+
+def _segment_types(segments, merge):
+    """Token types and video-slice grids of one sample laid out from the
+    workload's segments (text 0, audio 3, each vision segment a video slice)."""
+    import numpy as np
+    types, vid = [], []
+    for kind, arg in segments:
+        if kind in ("text", "audio"):
+            types.append(np.full(int(arg), 0 if kind == "text" else 3, np.int32))
+        else:
+            t, h, w = arg
+            types.append(np.full(t * (h // merge) * (w // merge), 2, np.int32))
+            vid.append([t, h, w])
+    return np.concatenate(types)[None], np.array(vid, np.int32).reshape(-1, 3)
+
+
+def next_rows(ipe, dev, stream, peak, reps):
+    """The rows beyond the path: the device position table (get_rope_index)
+    and the decode step, L2 flushed between timed calls."""
+    import numpy as np
+    import torch
+    import workloads as wl
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+
+    def entry(ms, nbytes, **kw):
+        return {"ms": ms, "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / peak, **kw}
+
+    # position table: the prefill request (B = 1) and a padded batch of 16
+    t = wl.WORKLOADS[WORKLOAD].text
+    types, vid = _segment_types(t.segments, t.merge)
+    small = wl.WORKLOADS["text_t4096_qwen35"].text
+    one, vid1 = _segment_types(small.segments, small.merge)
+    B, L = 16, one.shape[1] + 300
+    bt = np.zeros((B, L), np.int32)
+    bm = np.zeros((B, L), np.int32)
+    for b in range(B):
+        bt[b, 20 * b:20 * b + one.shape[1]] = one[0]
+        bm[b, 20 * b:20 * b + one.shape[1]] = 1
+    for name, ty, mk, vg in (("prefill_t131072", types, None, vid), ("batch16_l4396_padded", bt, bm, np.concatenate([vid1] * B))):
+        gty = torch.from_numpy(ty).to(dev)
+        gmk = None if mk is None else torch.from_numpy(mk).to(dev)
+        gvg = torch.from_numpy(vg).to(dev)
+        Bn, Ln = ty.shape
+        posb = torch.empty(3, Bn, Ln, dtype=torch.int32, device=dev)
+        dl = torch.empty(Bn, dtype=torch.int32, device=dev)
+        ws = torch.empty(ipe.rope_index_workspace_bytes(Bn, Ln, 0, vg.shape[0]), dtype=torch.uint8, device=dev)
+        nbytes = Bn * Ln * 4 * (1 + (mk is not None) + 3) + Bn * 4
+        ms = _time_flushed(torch, stream, lambda: ipe.mrope_rope_index(gty, None, gvg, gmk, t.merge, posb, dl, ws,
+                                                                       stream=stream), reps, flush)
+        res[f"rope_index/{name}"] = entry(ms, nbytes, slots=Bn * Ln, launches=3)
+
+    # decode step with the prefill model's heads: norm, rotation, cache write
+    D, hq, hk, rot = t.head_dim, t.hq, t.hk, t.rot_dim
+    inv = ipe.rope_inv_freq(rot, t.theta)
+    for B in (64, 256):
+        g = torch.Generator(device=dev).manual_seed(B)
+        q = torch.randn(B, hq, D, device=dev, generator=g).to(torch.bfloat16)
+        k = torch.randn(B, hk, D, device=dev, generator=g).to(torch.bfloat16)
+        v = torch.randn(B, hk, D, device=dev, generator=g).to(torch.bfloat16)
+        wq = torch.ones(D, dtype=torch.bfloat16, device=dev)
+        slots_n = B * 1024
+        kc = torch.zeros(slots_n, hk, D, dtype=torch.bfloat16, device=dev)
+        vc = torch.zeros_like(kc)
+        seq = torch.randint(2000, 100000, (B,), dtype=torch.int32, device=dev, generator=g)
+        dl = torch.randint(-2000, 0, (B,), dtype=torch.int32, device=dev, generator=g)
+        sm = (torch.arange(B, device=dev, dtype=torch.int64) * 1024 + seq.long() % 1024).contiguous()
+        nbytes = B * (hq + hk) * D * 2 * 2 + B * hk * D * 2 * 3 + B * 16 + 2 * D * 2
+        ms = _time_flushed(torch, stream, lambda: ipe.mrope_decode(q, k, seq, inv, dl, v=v, q_weight=wq, k_weight=wq,
+                                                                   k_cache=kc, v_cache=vc, slot_mapping=sm,
+                                                                   stream=stream), reps, flush)
+        res[f"mrope_decode/b{B}_norm_cache"] = entry(ms, nbytes, tokens=B, launches=1)
+        del kc, vc
+    ipe.device_status(stream)
+    torch.cuda.empty_cache()
     return res
 
 
