@@ -47,6 +47,8 @@ class Oracle:
             "orc_rms_norm": (_I, [_P, _I64, _I, _P, _D, _I, _P]),
             "orc_rope_index": (_I, [_P, _P, _I, _I64, _P, _I, _P, _I, _I, _P, _P]),
             "orc_decode_positions": (_I, [_P, _I, _I64, _P, _I64, _P, _P]),
+            "orc_vis_pos_interp_hf": (_I, [_P, _I, _I, _P, _I, _I, _P, _P, _I, _P]),
+            "orc_apply_rotary_hf": (_I, [_P, _I64, _I, _I, _P, _P, _I, _I, _P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -165,6 +167,54 @@ class Oracle:
                                           int(n_new), None if dl is None else _ptr(dl), _ptr(pos)):
             raise ValueError("decode_positions: bad arguments")
         return pos
+
+    # ------------------------------------------------------ HF rounding
+    def apply_rotary_hf(self, x, cos32, sin32, dtype):
+        """x [T, H, D] (values of `dtype`), cos / sin fp32 [T, rot]: the
+        rotation with every product and sum rounded to `dtype`."""
+        x = np.ascontiguousarray(x, np.float64)
+        c = np.ascontiguousarray(cos32, np.float32)
+        s_ = np.ascontiguousarray(sin32, np.float32)
+        T, H, D = x.shape
+        out = np.zeros_like(x)
+        if self._lib.orc_apply_rotary_hf(_ptr(x), T, H, D, _ptr(c), _ptr(s_), c.shape[1], {"f32": 0, "bf16": 1}[dtype],
+                                         _ptr(out)):
+            raise ValueError("apply_rotary_hf: bad arguments")
+        return out
+
+    def mrope_cos_sin_f32(self, positions, inv_freq, section, interleaved):
+        """The fp32 cos / sin tables: the double results rounded once."""
+        cos, sin = self.mrope_cos_sin(positions, inv_freq, section, interleaved)
+        return cos.astype(np.float32), sin.astype(np.float32)
+
+    def mrope_apply_hf(self, x, positions, inv_freq, section, interleaved, dtype):
+        cos, sin = self.mrope_cos_sin_f32(positions, inv_freq, section, interleaved)
+        return self.apply_rotary_hf(x, cos, sin, dtype)
+
+    @staticmethod
+    def linspace_f32(G, n):
+        """torch.linspace(0, G - 1, n) in fp32 (CPU), the listing's sample points."""
+        import torch
+        return torch.linspace(0, G - 1, n).numpy().astype(np.float32)
+
+    def vis_pos_interp_hf(self, table, grid_thw, merge, dtype):
+        """table [G*G, C] (values of `dtype`) -> [N, C] with the listing's
+        rounding points (fp32 linspace, weights and products in the dtype,
+        left-to-right sums)."""
+        tab = np.ascontiguousarray(table, np.float64)
+        GG, C = tab.shape
+        G = int(round(GG ** 0.5))
+        g = np.ascontiguousarray(grid_thw, np.int32).reshape(-1, 3)
+        N = self.grid_patches(g, merge)
+        ys = np.ascontiguousarray(np.concatenate([self.linspace_f32(G, int(h)) for _, h, _ in g] or [np.zeros(0)]),
+                                  np.float32)
+        xs = np.ascontiguousarray(np.concatenate([self.linspace_f32(G, int(w)) for _, _, w in g] or [np.zeros(0)]),
+                                  np.float32)
+        out = np.zeros((N, C), np.float64)
+        if self._lib.orc_vis_pos_interp_hf(_ptr(tab), G, C, _ptr(g), g.shape[0], int(merge), _ptr(ys), _ptr(xs),
+                                           {"f32": 0, "bf16": 1}[dtype], _ptr(out)):
+            raise ValueError("vis_pos_interp_hf: bad arguments")
+        return out
 
     # -------------------------------------------------------------- vision
     def grid_patches(self, grid_thw, merge):

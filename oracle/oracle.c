@@ -684,3 +684,100 @@ int orc_decode_positions(const int64_t *mask, int B, int64_t S, const int64_t *c
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * HF rounding mode (the rounding points of the listings run as written in
+ * the activation dtype), for users who must match those checkpoints bit
+ * for bit.
+ *
+ * Interpolation.  [QVL] fast_pos_embed_interpolate: the sample coordinates
+ * are an fp32 linspace (passed in: ys[h], xs[w] per image, concatenated);
+ * floor by truncation, ceiling min(floor + 1, G - 1); dh = y - floor in fp32;
+ * the four weights (1-dh)(1-dw), (1-dh)dw, dh(1-dw), dh dw are fp32 products
+ * and are then stored in the table's dtype; each corner row times its weight
+ * is one dtype product, and the four products are summed left to right, each
+ * sum rounded to the dtype (the dtype's arithmetic evaluates in fp32 and
+ * rounds back); frames repeat, then the 6-D merge permute.
+ * table: [G*G][C] values of the dtype; dtype 0 fp32, 1 bf16; out: [N][C].
+ * ---------------------------------------------------------------------- */
+int orc_vis_pos_interp_hf(const double *table, int G, int C, const int *grid_thw, int n_images, int m,
+                          const float *ys, const float *xs, int dtype, double *out)
+{
+    int64_t total;
+    if (G < 1 || C < 1 || (dtype != 0 && dtype != 1) || check_grid(grid_thw, n_images, m, &total))
+        return -1;
+    int64_t row0 = 0, yoff = 0, xoff = 0;
+    for (int i = 0; i < n_images; ++i) {
+        const int t = grid_thw[3 * i], h = grid_thw[3 * i + 1], w = grid_thw[3 * i + 2];
+        const int64_t hw = (int64_t)h * w;
+        double *frame = malloc(sizeof(double) * (size_t)(hw > 0 ? hw : 1) * C);
+        int64_t *src = malloc(sizeof(int64_t) * (size_t)(hw > 0 ? hw : 1) * t);
+        if (!frame || !src) {
+            free(frame);
+            free(src);
+            return -1;
+        }
+        for (int r = 0; r < h; ++r)
+            for (int c = 0; c < w; ++c) {
+                const float y = ys[yoff + r], x = xs[xoff + c];
+                const int y0 = (int)y, x0 = (int)x;               /* .int(): truncation */
+                const int y1 = y0 + 1 < G - 1 ? y0 + 1 : G - 1;   /* .clip(max=G-1) */
+                const int x1 = x0 + 1 < G - 1 ? x0 + 1 : G - 1;
+                const float dh = y - (float)y0, dw = x - (float)x0;
+                const float one_h = 1.0f - dh, one_w = 1.0f - dw;
+                float wt[4] = {one_h * one_w, one_h * dw, dh * one_w, dh * dw};
+                const int64_t idx[4] = {(int64_t)y0 * G + x0, (int64_t)y0 * G + x1, (int64_t)y1 * G + x0,
+                                        (int64_t)y1 * G + x1};
+                for (int q = 0; q < 4; ++q)
+                    wt[q] = (float)round_to(wt[q], dtype);       /* weights in the table dtype */
+                for (int ch = 0; ch < C; ++ch) {
+                    double s = 0.0;
+                    for (int q = 0; q < 4; ++q) {
+                        const double p = round_to(table[idx[q] * C + ch] * (double)wt[q], dtype);
+                        s = q == 0 ? p : round_to((double)((float)s + (float)p), dtype);
+                    }
+                    frame[((int64_t)r * w + c) * C + ch] = s;
+                }
+            }
+        /* frames repeat frame 0, then the merge permute */
+        merge_permute_rows(t, h, w, m, src);
+        for (int64_t k = 0; k < (int64_t)t * hw; ++k)
+            memcpy(out + (row0 + k) * C, frame + (src[k] % hw) * C, sizeof(double) * C);
+        free(frame);
+        free(src);
+        row0 += (int64_t)t * hw;
+        yoff += h;
+        xoff += w;
+    }
+    (void)total;
+    return 0;
+}
+
+/* Rotation.  [QVL] Qwen3VLTextRotaryEmbedding.forward returns cos and sin
+ * cast to the activation dtype; [IRPE] apply_rotary_pos_emb computes
+ * (q_rot * cos) + (rotate_half(q_rot) * sin) in that dtype; [M01] hints: for
+ * bf16 inputs cos / sin are cast first, then multiplied.  Each product and
+ * the sum are rounded to the dtype (the sum evaluated in fp32 first).
+ * x: [T][H][D] values of the dtype; cos_v, sin_v: [T][rot] fp32 values. */
+int orc_apply_rotary_hf(const double *x, int64_t T, int H, int D, const float *cos_v, const float *sin_v, int rot,
+                        int dtype, double *out)
+{
+    if (T < 0 || H < 0 || rot < 2 || rot % 2 || rot > D || (dtype != 0 && dtype != 1))
+        return -1;
+    const int h = rot / 2;
+    for (int64_t t = 0; t < T; ++t)
+        for (int hd = 0; hd < H; ++hd) {
+            const double *xr = x + (t * H + hd) * D;
+            double *o = out + (t * H + hd) * D;
+            for (int j = 0; j < rot; ++j) {
+                const double c = round_to(cos_v[t * rot + j], dtype);
+                const double s = round_to(sin_v[t * rot + j], dtype);
+                const double rh = j < h ? -xr[j + h] : xr[j - h];      /* rotate_half */
+                const double a = round_to(xr[j] * c, dtype);
+                const double b = round_to(rh * s, dtype);
+                o[j] = round_to((double)((float)a + (float)b), dtype);
+            }
+            memcpy(o + rot, xr + rot, sizeof(double) * (size_t)(D - rot));    /* pass-through */
+        }
+    return 0;
+}

@@ -499,4 +499,76 @@ def pin_decode_closed_forms(o):
     assert (got[:, 0, 0] == 4).all()
 
 
+# ------------------------------------------------------------ HF rounding
+
+
+def _torch_listing_interp(table, grids, m):
+    """The interpolation listing's steps evaluated by torch on the CPU in the
+    table's dtype (torch's bf16 arithmetic computes in fp32 and rounds back)."""
+    import torch
+    G = int(round(table.shape[0] ** 0.5))
+    outs = []
+    for t, h, w in grids:
+        ys, xs = torch.linspace(0, G - 1, h), torch.linspace(0, G - 1, w)
+        y0, x0 = ys.int(), xs.int()
+        y1, x1 = (y0 + 1).clip(max=G - 1), (x0 + 1).clip(max=G - 1)
+        dy, dx = ys - y0, xs - x0
+        corners = torch.stack([(y0[:, None] * G + x0[None]), (y0[:, None] * G + x1[None]),
+                               (y1[:, None] * G + x0[None]), (y1[:, None] * G + x1[None])]).reshape(4, -1)
+        wts = torch.stack([torch.outer(1 - dy, 1 - dx), torch.outer(1 - dy, dx), torch.outer(dy, 1 - dx),
+                           torch.outer(dy, dx)]).reshape(4, -1).to(table.dtype)
+        prod = table[corners.long()] * wts[:, :, None]
+        frame = ((prod[0] + prod[1]) + prod[2]) + prod[3]
+        merged = frame.repeat(t, 1).view(t, h // m, m, w // m, m, -1).permute(0, 1, 3, 2, 4, 5).reshape(t * h * w, -1)
+        outs.append(merged)
+    return torch.cat(outs)
+
+
+def pin_interp_hf_matches_torch_listing(o):
+    import torch
+    rng = _rng(29)
+    cases = [([(1, 4, 6), (2, 6, 4), (1, 48, 48), (1, 10, 14)], 2), ([(1, 5, 7), (3, 1, 9)], 1)]
+    for dt, tdt in (("bf16", torch.bfloat16), ("f32", torch.float32)):
+        table = torch.from_numpy(rng.standard_normal((48 * 48, 24)).astype(np.float32)).to(tdt)
+        vals = table.float().numpy().astype(np.float64)
+        for grids, m in cases:
+            want = _torch_listing_interp(table, grids, m).float().numpy().astype(np.float64)
+            got = o.vis_pos_interp_hf(vals, grids, m, dt)
+            assert got.shape == want.shape and (got == want).all(), (dt, grids)
+
+
+def pin_rotary_hf_matches_torch(o):
+    import torch
+    rng = _rng(31)
+    T, H, D, rot = 9, 3, 16, 8
+    pos = rng.integers(0, 5000, (3, T))
+    inv = o.rope_inv_freq(rot, 1e4)
+    cos, sin = o.mrope_cos_sin_f32(pos, inv, (2, 1, 1), True)
+    for dt, tdt in (("bf16", torch.bfloat16), ("f32", torch.float32)):
+        x = torch.from_numpy(rng.standard_normal((T, H, D)).astype(np.float32)).to(tdt)
+        c = torch.from_numpy(cos).to(tdt)[:, None, :]
+        s_ = torch.from_numpy(sin).to(tdt)[:, None, :]
+        xr, xp = x[..., :rot], x[..., rot:]
+        rh = torch.cat([-xr[..., rot // 2:], xr[..., :rot // 2]], dim=-1)
+        want = torch.cat([xr * c + rh * s_, xp], dim=-1).float().numpy().astype(np.float64)
+        got = o.apply_rotary_hf(x.float().numpy().astype(np.float64), cos, sin, dt)
+        assert (got == want).all(), dt
+
+
+def pin_hf_rounding_close_to_exact(o):
+    # a handful of dtype roundings away from the exact definitions
+    rng = _rng(37)
+    table = rng.standard_normal((48 * 48, 16)).astype(np.float32).astype(np.float64)
+    grids = [(1, 6, 10), (2, 4, 4)]
+    exact = o.vis_pos_embed_interpolate(table, grids, 2)
+    hf = o.vis_pos_interp_hf(table, grids, 2, "f32")
+    assert np.abs(hf - exact).max() <= 1e-5 * (1 + np.abs(exact).max())
+    x = rng.standard_normal((5, 2, 12))
+    pos = rng.integers(0, 100, (3, 5))
+    inv = o.rope_inv_freq(12, 1e4)
+    exact = o.mrope_apply(x.astype(np.float32).astype(np.float64), pos, inv, (2, 2, 2), False)
+    hf = o.mrope_apply_hf(x.astype(np.float32).astype(np.float64), pos, inv, (2, 2, 2), False, "f32")
+    assert np.abs(hf - exact).max() <= 1e-5 * (1 + np.abs(exact).max())
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -75,6 +75,17 @@ MUTANTS = {
                       "seq = mask[(int64_t)b * S + i] == 0 ? 0 : run;"),
     # decode positions: the rope delta not added
     "decode_no_delta": ("= seq + (deltas ? deltas[b] : 0);", "= seq;"),
+    # HF interpolation: top-right and bottom-left weights exchanged
+    "hf_weight_swap": ("float wt[4] = {one_h * one_w, one_h * dw, dh * one_w, dh * dw};",
+                       "float wt[4] = {one_h * one_w, dh * one_w, one_h * dw, dh * dw};"),
+    # HF interpolation: the running sum kept in double
+    "hf_sum_unrounded": ("s = q == 0 ? p : round_to((double)((float)s + (float)p), dtype);",
+                         "s = q == 0 ? p : s + p;"),
+    # HF rotation: cos not cast to the activation dtype
+    "hf_cos_unrounded": ("const double c = round_to(cos_v[t * rot + j], dtype);",
+                         "const double c = cos_v[t * rot + j];"),
+    # HF rotation: the product x cos not rounded
+    "hf_product_unrounded": ("const double a = round_to(xr[j] * c, dtype);", "const double a = xr[j] * c;"),
     # position table: image temporal index dropped
     "rope_image_time": ("table[0 * n + cols] = tt * 1 + cur;", "table[0 * n + cols] = cur;"),
 }
