@@ -179,6 +179,28 @@ int ipe_mrope_apply(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk
                     int interleaved, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * HF rounding mode of the text rotation: ipe_apply_rotary_partial_hf and
+ * ipe_mrope_apply_hf take the same arguments as the calls without the
+ * suffix and round where the reference listings round, so that results
+ * match those checkpoints' own code bit for bit:
+ * [QVL] Qwen3VLTextRotaryEmbedding.forward returns cos / sin cast to the
+ * activation dtype; [IRPE] apply_rotary_pos_emb computes
+ * (q_rot * cos) + (rotate_half(q_rot) * sin) in that dtype; [M01] hints
+ * (cos / sin cast first, then multiplied):
+ *   c = dtype(cos), s = dtype(sin)          (fp32 cos / sin as in the default mode)
+ *   out = dtype(fl32(dtype(x c) + dtype(rotate_half(x) s)))
+ * For fp32 activations every product and the sum are separate fp32
+ * roundings (no fused multiply-add).  Pass-through channels are untouched.
+ * ------------------------------------------------------------------------- */
+int ipe_apply_rotary_partial_hf(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk,
+                                int head_dim, int64_t q_tok_stride, int64_t k_tok_stride,
+                                const float *cos, const float *sin, int rot_dim, void *stream);
+int ipe_mrope_apply_hf(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
+                       int64_t q_tok_stride, int64_t k_tok_stride, const int32_t *positions,
+                       const float *inv_freq_host, int rot_dim, const int32_t *section,
+                       int interleaved, void *stream);
+
+/* ---------------------------------------------------------------------------
  * ipe_qk_norm_mrope -- RMSNorm of every head row of Q and K followed by the
  * multimodal rotation of ipe_mrope_apply, in one pass, in place.
  * [M01] problem summary and hints (rms_norm; the vllm-omni note on fusing it
@@ -350,6 +372,24 @@ int ipe_vis_interp_plan(const int32_t *grid_thw_host, int n_images, int merge, i
 int ipe_vis_pos_interp(const void *table, ipe_dtype dtype, int grid_side, int hidden,
                        const int32_t *grid_thw_host, int n_images, int merge, void *out,
                        void *stream);
+
+/* ---------------------------------------------------------------------------
+ * ipe_vis_pos_interp_hf -- ipe_vis_pos_interp with the rounding points of
+ * the [QVL] fast_pos_embed_interpolate listing, run as written in the
+ * table's dtype (same arguments):
+ *   sample points torch.linspace(0, G-1, n) in fp32: step fl32((G-1)/(n-1)),
+ *     point i = fl32(i step) for i < n/2, else fl32((G-1) - (n-1-i) step);
+ *   y0 = trunc(y), y1 = min(y0 + 1, G-1), dy = y - y0 (fp32), likewise x;
+ *   weights ((1-dy)(1-dx), (1-dy)dx, dy(1-dx), dy dx) as fp32 products, then
+ *     rounded to the dtype;
+ *   out = dtype(dtype(dtype(p0 + p1) + p2) + p3), p_c = dtype(T[idx_c] w_c),
+ *     each sum taken in fp32 first.
+ * hidden a multiple of 8 (bf16) or 4 (fp32); table and out 16-byte aligned
+ * (IPE_EALIGN otherwise).
+ * ------------------------------------------------------------------------- */
+int ipe_vis_pos_interp_hf(const void *table, ipe_dtype dtype, int grid_side, int hidden,
+                          const int32_t *grid_thw_host, int n_images, int merge, void *out,
+                          void *stream);
 
 /* ---------------------------------------------------------------------------
  * ipe_vis_rope2d -- vision 2-D rotary over the whole head, in place on q and k.

@@ -39,6 +39,9 @@ _SIGS = {
     "ipe_mrope_apply": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, _I, _P, _I, _P]),
     "ipe_qk_norm_mrope": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, ctypes.c_float, _P, _P, _I, _P, _I,
                                _P]),
+    "ipe_apply_rotary_partial_hf": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, _I, _P]),
+    "ipe_mrope_apply_hf": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, _I, _P, _I, _P]),
+    "ipe_vis_pos_interp_hf": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P]),
     "ipe_mrope_decode": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _I64, _P, _P, _P, _P, ctypes.c_float, _P,
                               _I, _P, _P, _I64, _I64, _P, _P]),
     "ipe_mrope_rope_index": (_I, [_P, _P, _I, _I64, _I64, _P, _I, _P, _I, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -227,27 +230,35 @@ def _qk_args(q, k):
     return _dtype_code(ref), T, hq, hk, head_dim, qs, ks
 
 
-def apply_rotary_partial(q, k, cos, sin, stream=None):
+def _rounding(rounding):
+    if rounding not in ("fp32", "hf"):
+        raise ValueError('rounding must be "fp32" (one rounding at the end) or "hf" (the reference listings\' '
+                         'rounding points)')
+    return rounding == "hf"
+
+
+def apply_rotary_partial(q, k, cos, sin, stream=None, rounding="fp32"):
     """In place: rotate_half rotation of the first cos.shape[1] channels of q [T, hq, D], k [T, hk, D]."""
     dt, T, hq, hk, D, qs, ks = _qk_args(q, k)
     for t, n in ((cos, "cos"), (sin, "sin")):
         _cuda(t, n)
         if t.dtype != torch.float32 or t.dim() != 2 or t.shape[0] != T or not t.is_contiguous():
             raise ValueError(f"{n} must be a contiguous float32 [T, rot_dim] tensor")
-    _check(_lib.ipe_apply_rotary_partial(_ptr(q), _ptr(k), dt, T, hq, hk, D, qs, ks, _ptr(cos), _ptr(sin),
-                                         cos.shape[1], _stream(stream)))
+    fn = _lib.ipe_apply_rotary_partial_hf if _rounding(rounding) else _lib.ipe_apply_rotary_partial
+    _check(fn(_ptr(q), _ptr(k), dt, T, hq, hk, D, qs, ks, _ptr(cos), _ptr(sin), cos.shape[1], _stream(stream)))
     return q, k
 
 
-def mrope_apply(q, k, positions, inv_freq, section, interleaved=True, stream=None):
+def mrope_apply(q, k, positions, inv_freq, section, interleaved=True, stream=None, rounding="fp32"):
     """In place: fused multimodal RoPE of q [T, hq, D] and k [T, hk, D] (cos / sin stay in registers)."""
     dt, T, hq, hk, D, qs, ks = _qk_args(q, k)
     _cuda(positions, "positions")
     if positions.dtype != torch.int32 or tuple(positions.shape) != (3, T) or not positions.is_contiguous():
         raise ValueError("positions must be a contiguous int32 [3, T] tensor")
     inv, half = _inv_host(inv_freq)
-    _check(_lib.ipe_mrope_apply(_ptr(q), _ptr(k), dt, T, hq, hk, D, qs, ks, _ptr(positions), inv, 2 * half,
-                                _i32_host(section, 3), int(bool(interleaved)), _stream(stream)))
+    fn = _lib.ipe_mrope_apply_hf if _rounding(rounding) else _lib.ipe_mrope_apply
+    _check(fn(_ptr(q), _ptr(k), dt, T, hq, hk, D, qs, ks, _ptr(positions), inv, 2 * half, _i32_host(section, 3),
+              int(bool(interleaved)), _stream(stream)))
     return q, k
 
 
@@ -435,7 +446,7 @@ def _table_args(table):
     return G, table.shape[1]
 
 
-def vis_pos_interp(table, grid_thw, merge=2, out=None, stream=None):
+def vis_pos_interp(table, grid_thw, merge=2, out=None, stream=None, rounding="fp32"):
     """[N, hidden] interpolated position embeddings in merge order, dtype of the table."""
     G, C = _table_args(table)
     g, n = _grid_host(grid_thw)
@@ -445,8 +456,8 @@ def vis_pos_interp(table, grid_thw, merge=2, out=None, stream=None):
     _cuda(out, "out")
     if out.dtype != table.dtype or tuple(out.shape) != (N, C) or not out.is_contiguous():
         raise ValueError(f"out must be a contiguous [{N}, {C}] tensor of the table's dtype")
-    _check(_lib.ipe_vis_pos_interp(_ptr(table), _dtype_code(table), G, C, g, n, int(merge), _ptr(out),
-                                   _stream(stream)))
+    fn = _lib.ipe_vis_pos_interp_hf if _rounding(rounding) else _lib.ipe_vis_pos_interp
+    _check(fn(_ptr(table), _dtype_code(table), G, C, g, n, int(merge), _ptr(out), _stream(stream)))
     return out
 
 

@@ -420,9 +420,9 @@ int ipe_mrope_cos_sin(const int32_t *positions, int64_t T, const float *inv_freq
     return e == cudaSuccess ? ok() : cuda_fail(e, "mrope_cos_sin launch");
 }
 
-int ipe_apply_rotary_partial(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
-                             int64_t q_tok_stride, int64_t k_tok_stride, const float *cos, const float *sin,
-                             int rot_dim, void *stream)
+static int apply_rotary_partial_impl(bool hf, void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk,
+                                     int head_dim, int64_t q_tok_stride, int64_t k_tok_stride, const float *cos,
+                                     const float *sin, int rot_dim, void *stream)
 {
     if (int rc = check_dtype(dtype)) return rc;
     if (rot_dim < 2 || rot_dim % 2) return fail(IPE_EINVAL, "rot_dim %d must be even and >= 2", rot_dim);
@@ -444,13 +444,30 @@ int ipe_apply_rotary_partial(void *q, void *k, ipe_dtype dtype, int64_t T, int h
     r.head_dim = head_dim;
     r.half = rot_dim / 2;
     TableAngles a{cos, sin};
-    cudaError_t e = launch_rotary_table(dtype == IPE_BF16, r, a, (cudaStream_t)stream);
+    cudaError_t e = launch_rotary_table(dtype == IPE_BF16, r, a, (cudaStream_t)stream, hf);
     return e == cudaSuccess ? ok() : cuda_fail(e, "apply_rotary_partial launch");
 }
 
-int ipe_mrope_apply(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
-                    int64_t q_tok_stride, int64_t k_tok_stride, const int32_t *positions, const float *inv_freq_host,
-                    int rot_dim, const int32_t *section, int interleaved, void *stream)
+int ipe_apply_rotary_partial(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
+                             int64_t q_tok_stride, int64_t k_tok_stride, const float *cos, const float *sin,
+                             int rot_dim, void *stream)
+{
+    return apply_rotary_partial_impl(false, q, k, dtype, T, hq, hk, head_dim, q_tok_stride, k_tok_stride, cos, sin,
+                                     rot_dim, stream);
+}
+
+int ipe_apply_rotary_partial_hf(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
+                                int64_t q_tok_stride, int64_t k_tok_stride, const float *cos, const float *sin,
+                                int rot_dim, void *stream)
+{
+    return apply_rotary_partial_impl(true, q, k, dtype, T, hq, hk, head_dim, q_tok_stride, k_tok_stride, cos, sin,
+                                     rot_dim, stream);
+}
+
+static int mrope_apply_impl(bool hf, void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
+                            int64_t q_tok_stride, int64_t k_tok_stride, const int32_t *positions,
+                            const float *inv_freq_host, int rot_dim, const int32_t *section, int interleaved,
+                            void *stream)
 {
     if (int rc = check_dtype(dtype)) return rc;
     if (rot_dim < 2 || rot_dim % 2) return fail(IPE_EINVAL, "rot_dim %d must be even and >= 2", rot_dim);
@@ -470,8 +487,24 @@ int ipe_mrope_apply(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk
     r.hk = hk;
     r.head_dim = head_dim;
     r.half = rot_dim / 2;
-    cudaError_t e = launch_rotary_mrope(dtype == IPE_BF16, r, a, (cudaStream_t)stream);
+    cudaError_t e = launch_rotary_mrope(dtype == IPE_BF16, r, a, (cudaStream_t)stream, hf);
     return e == cudaSuccess ? ok() : cuda_fail(e, "mrope_apply launch");
+}
+
+int ipe_mrope_apply(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
+                    int64_t q_tok_stride, int64_t k_tok_stride, const int32_t *positions, const float *inv_freq_host,
+                    int rot_dim, const int32_t *section, int interleaved, void *stream)
+{
+    return mrope_apply_impl(false, q, k, dtype, T, hq, hk, head_dim, q_tok_stride, k_tok_stride, positions,
+                            inv_freq_host, rot_dim, section, interleaved, stream);
+}
+
+int ipe_mrope_apply_hf(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
+                       int64_t q_tok_stride, int64_t k_tok_stride, const int32_t *positions,
+                       const float *inv_freq_host, int rot_dim, const int32_t *section, int interleaved, void *stream)
+{
+    return mrope_apply_impl(true, q, k, dtype, T, hq, hk, head_dim, q_tok_stride, k_tok_stride, positions,
+                            inv_freq_host, rot_dim, section, interleaved, stream);
 }
 
 int ipe_qk_norm_mrope(void *q, void *k, ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim, int64_t q_tok_stride,
@@ -732,6 +765,22 @@ int ipe_vis_pos_interp(const void *table, ipe_dtype dtype, int grid_side, int hi
     if (int rc = interp_args(table, dtype, grid_side, hidden, out, d, ia)) return rc;
     cudaError_t e = launch_vis_interp(dtype == IPE_BF16, d, ia, (cudaStream_t)stream);
     return e == cudaSuccess ? ok() : cuda_fail(e, "vis_pos_interp launch");
+}
+
+int ipe_vis_pos_interp_hf(const void *table, ipe_dtype dtype, int grid_side, int hidden, const int32_t *grid_thw_host,
+                          int n_images, int merge, void *out, void *stream)
+{
+    VisDesc<1024> &d = *desc_buffer();
+    if (int rc = build_vis_desc(grid_thw_host, n_images, merge, grid_side, d)) return rc;
+    if (d.n_patch == 0) return check_dtype(dtype) ? IPE_EINVAL : ok();
+    if (int rc = check_dtype(dtype)) return rc;
+    const int ec = 16 / elem_bytes(dtype);
+    if (hidden <= 0 || hidden % ec) return fail(IPE_EINVAL, "hidden %d must be a positive multiple of %d", hidden, ec);
+    if (!aligned(table, 16) || !aligned(out, 16)) return fail(IPE_EALIGN, "table / out must be 16-byte aligned");
+    InterpArgs ia;
+    if (int rc = interp_args(table, dtype, grid_side, hidden, out, d, ia)) return rc;
+    cudaError_t e = launch_vis_interp_hf(dtype == IPE_BF16, d, ia, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "vis_pos_interp_hf launch");
 }
 
 static int vis_rot_args(void *q, void *k, ipe_dtype dtype, int64_t n_patch, int heads, int head_dim,

@@ -22,6 +22,9 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(v);
 }
 
+// v rounded to the dtype T and back to fp32 (round to nearest even; exact for fp32).
+template <typename T> __device__ __forceinline__ float round_to_dtype(float v) { return to_f32(from_f32<T>(v)); }
+
 // N contiguous elements moved as one aligned access (N * sizeof(T) <= 16).
 template <typename T, int N>
 struct __align__(sizeof(T) * N) Pack {

@@ -182,12 +182,15 @@ cudaError_t launch_mrope_cos_sin(const MropeAngles &a, int half, float *cos_out,
                                  cudaStream_t s);
 cudaError_t launch_mrope_axis_map(int half, const int *section, int interleaved, int8_t *axis,
                                   cudaStream_t s);
-cudaError_t launch_rotary_mrope(bool bf16, const RotArgs &r, const MropeAngles &a, cudaStream_t s);
-cudaError_t launch_rotary_table(bool bf16, const RotArgs &r, const TableAngles &a, cudaStream_t s);
+cudaError_t launch_rotary_mrope(bool bf16, const RotArgs &r, const MropeAngles &a, cudaStream_t s,
+                                bool hf = false);
+cudaError_t launch_rotary_table(bool bf16, const RotArgs &r, const TableAngles &a, cudaStream_t s,
+                                bool hf = false);
 
 cudaError_t launch_vis_plan(const VisDesc<1024> &d, int32_t *idx4, float *w4, int32_t *rowcol,
                             cudaStream_t s);
 cudaError_t launch_vis_interp(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, cudaStream_t s);
+cudaError_t launch_vis_interp_hf(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, cudaStream_t s);
 cudaError_t launch_vis_rope(bool bf16, const VisDesc<1024> &d, const RotArgs &r,
                             const VisAngleFreqs &f, cudaStream_t s);
 cudaError_t launch_vis_fused(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, const RotArgs &r,

@@ -7,6 +7,8 @@
 // apply_rotary_pos_emb; "M01 RMSNorm and multimodal RoPE" (kuanzhou.online).
 #include <algorithm>
 
+#include <type_traits>
+
 #include "ipe_rotary_tma.cuh"
 
 namespace ipe {
@@ -123,27 +125,46 @@ static cudaError_t dispatch_tma(const TmaRotArgs &t, const RotArgs &r, const Src
     return launch_rotary_tma_vec<T, 2, Src>(t, src, s);
 }
 
-cudaError_t launch_rotary_mrope(bool bf16, const RotArgs &r, const MropeAngles &a, cudaStream_t s)
+// HF rounding mode (hf): the same engines with cos / sin cast to the
+// activation dtype and each product and sum rounded to it.
+template <typename T, bool HF>
+using MropeTmaOf = std::conditional_t<HF, HfTmaSrc<MropeTmaSrc, T>, MropeTmaSrc>;
+template <typename T, bool HF>
+using TableTmaOf = std::conditional_t<HF, HfTmaSrc<TableTmaSrc, T>, TableTmaSrc>;
+template <typename T, bool HF>
+using MropeVecOf = std::conditional_t<HF, HfVecSrc<MropeSrc, T>, MropeSrc>;
+template <typename T, bool HF>
+using TableVecOf = std::conditional_t<HF, HfVecSrc<TableSrc, T>, TableSrc>;
+
+template <typename T, bool HF>
+static cudaError_t rotary_mrope(const RotArgs &r, const MropeAngles &a, cudaStream_t s)
 {
     TmaRotArgs t;
-    if (tma_rot_args(r, bf16 ? 2 : 4, t)) {
+    if (tma_rot_args(r, sizeof(T), t)) {
         // positions [3, T] as a {T, 3} tensor: rows must be 16-byte multiples
         const uint64_t dims[2] = {(uint64_t)a.T, 3};
         const uint64_t str[1] = {(uint64_t)a.T * 4};
         const uint32_t box[2] = {(uint32_t)t.P, 3};
         t.aux_tma = a.T % 4 == 0 && encode_tmap(&t.taux0, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, a.positions, dims, str, box);
         t.aux_bytes = (unsigned)t.P * 3 * 4;
-        MropeTmaSrc src{a};
-        return bf16 ? dispatch_tma<__nv_bfloat16>(t, r, src, s) : dispatch_tma<float>(t, r, src, s);
+        MropeTmaOf<T, HF> src{MropeTmaSrc{a}};
+        return dispatch_tma<T>(t, r, src, s);
     }
-    MropeSrc src{a};
-    return bf16 ? dispatch_vec<__nv_bfloat16>(r, src, s) : dispatch_vec<float>(r, src, s);
+    MropeVecOf<T, HF> src{MropeSrc{a}};
+    return dispatch_vec<T>(r, src, s);
 }
 
-cudaError_t launch_rotary_table(bool bf16, const RotArgs &r, const TableAngles &a, cudaStream_t s)
+cudaError_t launch_rotary_mrope(bool bf16, const RotArgs &r, const MropeAngles &a, cudaStream_t s, bool hf)
+{
+    if (hf) return bf16 ? rotary_mrope<__nv_bfloat16, true>(r, a, s) : rotary_mrope<float, true>(r, a, s);
+    return bf16 ? rotary_mrope<__nv_bfloat16, false>(r, a, s) : rotary_mrope<float, false>(r, a, s);
+}
+
+template <typename T, bool HF>
+static cudaError_t rotary_table(const RotArgs &r, const TableAngles &a, cudaStream_t s)
 {
     TmaRotArgs t;
-    if (tma_rot_args(r, bf16 ? 2 : 4, t)) {
+    if (tma_rot_args(r, sizeof(T), t)) {
         const int rot = 2 * r.half;
         const uint64_t dims[2] = {(uint64_t)rot, (uint64_t)r.rows};
         const uint64_t str[1] = {(uint64_t)rot * 4};
@@ -151,11 +172,17 @@ cudaError_t launch_rotary_table(bool bf16, const RotArgs &r, const TableAngles &
         t.aux_tma = encode_tmap(&t.taux0, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a.cos, dims, str, box) &&
                     encode_tmap(&t.taux1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a.sin, dims, str, box);
         t.aux_bytes = 2u * t.P * rot * 4;
-        TableTmaSrc src{a};
-        return bf16 ? dispatch_tma<__nv_bfloat16>(t, r, src, s) : dispatch_tma<float>(t, r, src, s);
+        TableTmaOf<T, HF> src{TableTmaSrc{a}};
+        return dispatch_tma<T>(t, r, src, s);
     }
-    TableSrc src{a};
-    return bf16 ? dispatch_vec<__nv_bfloat16>(r, src, s) : dispatch_vec<float>(r, src, s);
+    TableVecOf<T, HF> src{TableSrc{a}};
+    return dispatch_vec<T>(r, src, s);
+}
+
+cudaError_t launch_rotary_table(bool bf16, const RotArgs &r, const TableAngles &a, cudaStream_t s, bool hf)
+{
+    if (hf) return bf16 ? rotary_table<__nv_bfloat16, true>(r, a, s) : rotary_table<float, true>(r, a, s);
+    return bf16 ? rotary_table<__nv_bfloat16, false>(r, a, s) : rotary_table<float, false>(r, a, s);
 }
 
 }  // namespace ipe

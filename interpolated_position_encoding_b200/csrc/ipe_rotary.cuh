@@ -25,6 +25,7 @@ constexpr int kRotBatch = 4;       // independent head-row chunks in flight per 
 
 struct MropeSrc {
     static constexpr bool kHi = false;
+    static constexpr bool kHf = false;
     MropeAngles a;
     __device__ __forceinline__ void prepare(long long r0, int rows, int half, float2 *lo, float2 *,
                                             int *) const
@@ -44,6 +45,7 @@ struct MropeSrc {
 
 struct TableSrc {
     static constexpr bool kHi = true;
+    static constexpr bool kHf = false;
     TableAngles a;
     __device__ __forceinline__ void prepare(long long r0, int rows, int half, float2 *lo, float2 *hi,
                                             int *) const
@@ -61,6 +63,7 @@ struct TableSrc {
 template <int MAXIMG>
 struct VisSrc {
     static constexpr bool kHi = false;
+    static constexpr bool kHf = false;
     VisDesc<MAXIMG> d;
     VisAngleFreqs f;
     // aux: (row, col) of each tile row.
@@ -84,6 +87,21 @@ struct VisSrc {
             float s, c;
             sincosf(angle, &s, &c);
             lo[i] = make_float2(c, s);
+        }
+    }
+};
+
+// HF rounding mode of a source: cos / sin cast to the activation dtype T
+// (each thread rounds the entries it wrote in prepare()).
+template <class Base, typename T>
+struct HfVecSrc : Base {
+    static constexpr bool kHf = true;
+    __device__ __forceinline__ void prepare(long long r0, int rows, int half, float2 *lo, float2 *hi, int *aux) const
+    {
+        Base::prepare(r0, rows, half, lo, hi, aux);
+        for (int i = threadIdx.x; i < rows * half; i += blockDim.x) {
+            lo[i] = make_float2(round_to_dtype<T>(lo[i].x), round_to_dtype<T>(lo[i].y));
+            if constexpr (Base::kHi) hi[i] = make_float2(round_to_dtype<T>(hi[i].x), round_to_dtype<T>(hi[i].y));
         }
     }
 };
@@ -153,8 +171,16 @@ __device__ __forceinline__ void rotary_tiles(const RotArgs &r, const Src &src, l
                     const float a = to_f32(xa[b].v[e]);
                     const float bb = to_f32(xb[b].v[e]);
                     // x[j] cos - x[j+h] sin ; x[j+h] cos + x[j] sin
-                    ya.v[e] = from_f32<T>(__fmaf_rn(a, cl.x, -__fmul_rn(bb, cl.y)));
-                    yb.v[e] = from_f32<T>(__fmaf_rn(bb, ch.x, __fmul_rn(a, ch.y)));
+                    if constexpr (Src::kHf) {
+                        // each product rounded to T, the sum in fp32, then to T
+                        ya.v[e] = from_f32<T>(__fadd_rn(round_to_dtype<T>(__fmul_rn(a, cl.x)),
+                                                        round_to_dtype<T>(-__fmul_rn(bb, cl.y))));
+                        yb.v[e] = from_f32<T>(__fadd_rn(round_to_dtype<T>(__fmul_rn(bb, ch.x)),
+                                                        round_to_dtype<T>(__fmul_rn(a, ch.y))));
+                    } else {
+                        ya.v[e] = from_f32<T>(__fmaf_rn(a, cl.x, -__fmul_rn(bb, cl.y)));
+                        yb.v[e] = from_f32<T>(__fmaf_rn(bb, ch.x, __fmul_rn(a, ch.y)));
+                    }
                 }
                 st_pack<T, VEC>(ptr[b], ya);
                 st_pack<T, VEC>(ptr[b] + half, yb);

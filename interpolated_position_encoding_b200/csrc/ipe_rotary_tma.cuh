@@ -111,6 +111,7 @@ __device__ __forceinline__ void load_coef(const float *p, float2 *v)
 
 struct MropeTmaSrc {
     static constexpr bool kHi = false;
+    static constexpr bool kHf = false;
     MropeAngles a;
     __device__ __forceinline__ void issue_aux(const TmaRotArgs &r, uint32_t stage, int r0, uint32_t bar) const
     {
@@ -136,6 +137,7 @@ struct MropeTmaSrc {
 
 struct TableTmaSrc {
     static constexpr bool kHi = true;
+    static constexpr bool kHf = false;
     TableAngles a;
     __device__ __forceinline__ void issue_aux(const TmaRotArgs &r, uint32_t stage, int r0, uint32_t bar) const
     {
@@ -163,6 +165,7 @@ struct TableTmaSrc {
 template <int MAXIMG>
 struct VisTmaSrc {
     static constexpr bool kHi = false;
+    static constexpr bool kHf = false;
     VisDesc<MAXIMG> d;
     VisAngleFreqs f;
     __device__ __forceinline__ void issue_aux(const TmaRotArgs &, uint32_t, int, uint32_t) const {}
@@ -185,6 +188,38 @@ struct VisTmaSrc {
     }
 };
 
+// HF rounding mode of a source: its cos / sin cast to the activation dtype T
+// before they are used (each lane rounds the entries it wrote).
+template <class Base, typename T>
+struct HfTmaSrc : Base {
+    static constexpr bool kHf = true;
+    __device__ __forceinline__ void angles(const TmaRotArgs &r, const unsigned char *stage, int c, long long row,
+                                           int lane, const CsSlot &cs) const
+    {
+        Base::angles(r, stage, c, row, lane, cs);
+        for (int j = lane; j < r.half; j += 32) {
+            const float sn = round_to_dtype<T>(cs.s[j]);
+            cs.c[j] = round_to_dtype<T>(cs.c[j]);
+            cs.s[j] = sn;
+            cs.ns[j] = -sn;
+            if constexpr (Base::kHi) {
+                cs.ch[j] = round_to_dtype<T>(cs.ch[j]);
+                cs.sh[j] = round_to_dtype<T>(cs.sh[j]);
+            }
+        }
+    }
+};
+
+// HF combine of a pair: each product rounded to T, their sum evaluated in
+// fp32 (the caller's store rounds it to T).
+template <typename T>
+__device__ __forceinline__ float2 hf_pair(float2 a, float2 b)
+{
+    a = make_float2(round_to_dtype<T>(a.x), round_to_dtype<T>(a.y));
+    b = make_float2(round_to_dtype<T>(b.x), round_to_dtype<T>(b.y));
+    return make_float2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y));
+}
+
 // One chunk: elements [u VEC, u VEC + VEC) of the first half of head row `p`
 // and the matching chunk of the second half, rotated in place.  With `swap`
 // the lane reads (and writes) the second half first, which spreads
@@ -193,7 +228,7 @@ struct VisTmaSrc {
 //   x'[j + h] = x[j + h] cos_{j+h} + x[j] sin_{j+h}
 // written as  w1 = v1 C1 + v2 S1,  w2 = v2 C2 + v1 S2  on the values v1, v2
 // at the first and second address, with C / S chosen (not computed) per lane.
-template <typename T, int VEC, bool HI>
+template <typename T, int VEC, bool HI, bool HF>
 __device__ __forceinline__ void rotate_chunk(T *p, int half, int u, bool swap, const CsSlot &cs)
 {
     static_assert(VEC >= 2, "pairs");
@@ -213,15 +248,20 @@ __device__ __forceinline__ void rotate_chunk(T *p, int half, int u, bool swap, c
     if constexpr (HI) load_coef<VEC>(C2, c2);
 #pragma unroll
     for (int i = 0; i < VEC / 2; ++i) {
-        w1[i] = fma2(v1[i], c1[i], mul2(v2[i], s1[i]));
-        w2[i] = fma2(v2[i], HI ? c2[i] : c1[i], mul2(v1[i], s2[i]));
+        if constexpr (HF) {
+            w1[i] = hf_pair<T>(mul2(v1[i], c1[i]), mul2(v2[i], s1[i]));
+            w2[i] = hf_pair<T>(mul2(v2[i], HI ? c2[i] : c1[i]), mul2(v1[i], s2[i]));
+        } else {
+            w1[i] = fma2(v1[i], c1[i], mul2(v2[i], s1[i]));
+            w2[i] = fma2(v2[i], HI ? c2[i] : c1[i], mul2(v1[i], s2[i]));
+        }
     }
     store_pairs<T, VEC>(p1, w1);
     store_pairs<T, VEC>(p2, w2);
 }
 
 // Rotate the head rows of one tile row (q slot then k slot) in shared memory.
-template <typename T, int VEC, bool HI>
+template <typename T, int VEC, bool HI, bool HF>
 __device__ __forceinline__ void rotate_slots(const TmaRotArgs &a, unsigned char *sq, unsigned char *sk, int lane,
                                              const CsSlot &cs)
 {
@@ -233,7 +273,7 @@ __device__ __forceinline__ void rotate_slots(const TmaRotArgs &a, unsigned char 
         if (lane < H) {
             T *p = lane < a.hq ? q + lane * rot : k + (lane - a.hq) * rot;
             const bool swap = (lane >> a.swap_shift) & 1;
-            for (int u = 0; u < nvec; ++u) rotate_chunk<T, VEC, HI>(p, half, u, swap, cs);
+            for (int u = 0; u < nvec; ++u) rotate_chunk<T, VEC, HI, HF>(p, half, u, swap, cs);
         }
     } else {
         // lanes sweep (head, chunk) with the chunk fastest; odd heads swap
@@ -241,7 +281,7 @@ __device__ __forceinline__ void rotate_slots(const TmaRotArgs &a, unsigned char 
         const int dh = 32 / nvec, du = 32 - dh * nvec;
         while (h < H) {
             T *p = h < a.hq ? q + h * rot : k + (h - a.hq) * rot;
-            rotate_chunk<T, VEC, HI>(p, half, u, h & 1, cs);
+            rotate_chunk<T, VEC, HI, HF>(p, half, u, h & 1, cs);
             u += du;
             h += dh;
             if (u >= nvec) {
@@ -366,7 +406,7 @@ __device__ __forceinline__ void rotary_tma_block(const TmaRotArgs &a, const Src 
             unsigned char *sk = stage + a.off_k + (size_t)c * a.slot_k;
             src.angles(a, stage, c, row, lane, cs);
             __syncwarp();
-            rotate_slots<T, VEC, Src::kHi>(a, sq, sk, lane, cs);
+            rotate_slots<T, VEC, Src::kHi, Src::kHf>(a, sq, sk, lane, cs);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {

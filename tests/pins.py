@@ -503,8 +503,9 @@ def pin_decode_closed_forms(o):
 
 
 def _torch_listing_interp(table, grids, m):
-    """The interpolation listing's steps evaluated by torch on the CPU in the
-    table's dtype (torch's bf16 arithmetic computes in fp32 and rounds back)."""
+    """The interpolation listing's steps evaluated by torch in the table's
+    dtype on the table's device (torch's bf16 arithmetic computes in fp32 and
+    rounds back); the sample points come from torch.linspace on the CPU."""
     import torch
     G = int(round(table.shape[0] ** 0.5))
     outs = []
@@ -516,8 +517,8 @@ def _torch_listing_interp(table, grids, m):
         corners = torch.stack([(y0[:, None] * G + x0[None]), (y0[:, None] * G + x1[None]),
                                (y1[:, None] * G + x0[None]), (y1[:, None] * G + x1[None])]).reshape(4, -1)
         wts = torch.stack([torch.outer(1 - dy, 1 - dx), torch.outer(1 - dy, dx), torch.outer(dy, 1 - dx),
-                           torch.outer(dy, dx)]).reshape(4, -1).to(table.dtype)
-        prod = table[corners.long()] * wts[:, :, None]
+                           torch.outer(dy, dx)]).reshape(4, -1).to(table.dtype).to(table.device)
+        prod = table[corners.long().to(table.device)] * wts[:, :, None]
         frame = ((prod[0] + prod[1]) + prod[2]) + prod[3]
         merged = frame.repeat(t, 1).view(t, h // m, m, w // m, m, -1).permute(0, 1, 3, 2, 4, 5).reshape(t * h * w, -1)
         outs.append(merged)
