@@ -728,6 +728,27 @@ def next_rows(ipe, dev, stream, peak, reps):
                                                                    stream=stream), reps, flush)
         res[f"mrope_decode/b{B}_norm_cache"] = entry(ms, nbytes, tokens=B, launches=1)
         del kc, vc
+    # HF rounding mode: interpolation (four-corner sum) and the fused MRoPE
+    for name in ("prefill_t131072_video", "vision_batch8_bf16"):
+        w = wl.WORKLOADS[name]
+        v = w.vision
+        vin = wl.vision_inputs(w)
+        table = torch.from_numpy(vin["table"].view(np.int16)).view(torch.bfloat16).to(dev)
+        out = torch.empty(wl.n_patches(v), v.hidden, dtype=torch.bfloat16, device=dev)
+        ms = _time_flushed(torch, stream, lambda: ipe.vis_pos_interp(table, v.grid_thw, v.merge, out=out, stream=stream,
+                                                                     rounding="hf"), reps, flush)
+        res[f"vis_pos_interp_hf/{name}"] = entry(ms, algorithmic_bytes_vision(v))
+        del out
+    w = wl.WORKLOADS[WORKLOAD]
+    tin = wl.text_inputs(w)
+    Q = torch.from_numpy(tin["q"].view(np.int16)).view(torch.bfloat16).to(dev)
+    K = torch.from_numpy(tin["k"].view(np.int16)).view(torch.bfloat16).to(dev)
+    pos = torch.from_numpy(tin["positions"]).to(dev)
+    inv = ipe.rope_inv_freq(t.rot_dim, t.theta)
+    ms = _time_flushed(torch, stream, lambda: ipe.mrope_apply(Q, K, pos, inv, t.section, True, stream=stream,
+                                                              rounding="hf"), reps, flush)
+    res[f"mrope_apply_hf/{WORKLOAD}"] = entry(ms, (t.hq + t.hk) * t.T * t.rot_dim * 2 * 2 + 3 * t.T * 4)
+    del Q, K
     ipe.device_status(stream)
     torch.cuda.empty_cache()
     return res
