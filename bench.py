@@ -298,8 +298,9 @@ CASES = {
 
 
 def run_case(args):
-    """--case NAME: `--warmup` untimed and `--steps` timed launches of one
-    kernel on its case (inputs resident, no L2 flush); one JSON line."""
+    """--case NAME: `--warmup` untimed and `--steps` timed calls of one
+    kernel on its case (inputs resident, no L2 flush), each timed alone
+    after a short GPU sleep; one JSON line."""
     import numpy as np
     import torch
     import interpolated_position_encoding_b200 as ipe
@@ -349,14 +350,19 @@ def run_case(args):
     for _ in range(max(args.warmup, 0)):
         fn()
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
+    total = 0.0
     for _ in range(args.steps):
+        # a short GPU sleep first, so the call is queued before its start
+        # event fires and the events time the device, not the host
+        torch.cuda._sleep(200_000)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
         fn()
-    b.record(stream)
-    torch.cuda.synchronize()
+        b.record(stream)
+        torch.cuda.synchronize()
+        total += a.elapsed_time(b)
     ipe.device_status(stream)
-    ms = a.elapsed_time(b) / max(args.steps, 1)
+    ms = total / max(args.steps, 1)
     peak, _ = measured_peaks()
     print(json.dumps({"case": name, "what": CASES[name], "steps": args.steps, "warmup": args.warmup, "ms": ms,
                       "alg_bytes": nbytes, "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / peak,

@@ -59,16 +59,18 @@ struct RiCarry {
     long long vadv0;              // advances of the sample's vision runs started before the tile
     int prev_cls;                 // class of the last kept slot before the tile (-1: none)
     int open_k, open_grid;        // the run open at the tile's first slot: first kept index, grid
+    int own_k, own_grid;          // the tile's own last run start (read by later tiles)
     int pad;
-    long long open_start;         // ... and its start position
+    long long open_start, own_start;
 };
 
 struct RiSample {
     int kept;                     // kept slots of the sample
-    int img, vid;                 // image / video runs: of the sample, then (scanned) of the batch before it
+    int img, vid;                 // image / video runs of the batch before the sample
     int max_pos;                  // largest coordinate written
     unsigned done;                // tiles finished
-    int pad[3];
+    int k_base, text_base;        // kept / kept-text slots of the batch before the sample
+    int pad;
 };
 
 RopeIndexLayout rope_index_layout(long long B, long long L, int n_img, int n_vid)
@@ -316,61 +318,27 @@ __device__ longlong2 scan_pair(longlong2 v, longlong2 *warp_tot, longlong2 &tot)
     return make_longlong2(pre.x + inc.x - v.x, pre.y + inc.y - v.y);
 }
 
-__device__ __forceinline__ int warp_incl_max(int v)
-{
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, v, d);
-        if (lane >= d && o > v) v = o;
-    }
-    return v;
-}
-
-__device__ __forceinline__ int warp_incl_sum(int v)
-{
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, v, d);
-        if (lane >= d) v += o;
-    }
-    return v;
-}
-
-// Per tile of one chunk of 32 (lane = tile): its aggregate, the class before
-// it, and whether its first kept slot starts a run.
-struct RiTileView {
-    RiTileAgg g;
-    int prev, first_start, img, vid;   // img / vid: run starts including the first kept slot
-};
-
-__device__ __forceinline__ RiTileView view_tile(const RopeIndexArgs &a, long long b, int t, int &carry_key)
-{
-    RiTileView r;
-    r.g = RiTileAgg{0, 0, -1, -1, 0, 0, -1, 0, 0, 0, -1, 0};
-    if (t < a.tiles_per_row) r.g = static_cast<const RiTileAgg *>(a.agg)[b * a.tiles_per_row + t];
-    const int key = r.g.kept > 0 ? (t + 1) * 4 + r.g.last_cls : 0;
-    const int inc = warp_incl_max(key);
-    int exc = __shfl_up_sync(0xffffffffu, inc, 1);
-    if ((threadIdx.x & 31) == 0) exc = 0;
-    if (carry_key > exc) exc = carry_key;
-    carry_key = max(carry_key, __shfl_sync(0xffffffffu, inc, 31));
-    r.prev = exc ? (exc & 3) : -1;
-    r.first_start = r.g.kept > 0 && r.g.first_cls != r.prev;
-    r.img = r.g.img + (r.first_start && r.g.first_cls == 1);
-    r.vid = r.g.vid + (r.first_start && r.g.first_cls == 2);
-    return r;
-}
-
+// One thread per tile of the whole batch (in chunks of the block size), two
+// block scans per chunk carried across chunks:
+//   1. the latest tile with a kept slot (key (g + 1) * 4 + class, max):
+//      the class before each tile, and whether its first kept slot starts a
+//      run (the same sample only: the key's tile must not precede the
+//      sample's first tile);
+//   2. kept, text, image-run and video-run counts (sums over the batch) and
+//      the latest tile with a run start (max).  Image / video runs of the
+//      batch are plain prefix sums (the grid sequences serve the batch in
+//      order); kept and text counts are taken relative to the sample's first
+//      tile.
 __global__ void __launch_bounds__(kRiCarryThreads) ri_carry_kernel(const __grid_constant__ RopeIndexArgs a)
 {
-    __shared__ longlong2 warp_tot[kRiCarryThreads / 32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+    __shared__ longlong2 warp_tot2[kRiCarryThreads / 32];
+    __shared__ RiSums warp_tot[kRiCarryThreads / 32];
     long long *img_adv = reinterpret_cast<long long *>(a.img_adv);
     long long *vid_slices = reinterpret_cast<long long *>(a.vid_slices);
     long long *vid_adv = reinterpret_cast<long long *>(a.vid_adv);
     RiSample *smp = static_cast<RiSample *>(a.sample);
+    RiCarry *carry = static_cast<RiCarry *>(a.carry);
+    const RiTileAgg *agg = static_cast<const RiTileAgg *>(a.agg);
 
     // grid prefix sums: image advances; video slices and slice advances
     longlong2 run{0, 0}, tot;
@@ -383,7 +351,7 @@ __global__ void __launch_bounds__(kRiCarryThreads) ri_carry_kernel(const __grid_
             if (!side_ok(t) || !side_ok(h) || !side_ok(w)) record_fault(a.status, kRiBadGrid);
             adv = grid_row(a, a.img_grid, j, false).adv;
         }
-        const longlong2 ex = scan_pair(make_longlong2(adv, 0), warp_tot, tot);
+        const longlong2 ex = scan_pair(make_longlong2(adv, 0), warp_tot2, tot);
         if (j < a.n_img) img_adv[j] = run.x + ex.x;
         run.x += tot.x;
     }
@@ -400,7 +368,7 @@ __global__ void __launch_bounds__(kRiCarryThreads) ri_carry_kernel(const __grid_
             v.x = good ? t : 0;
             v.y = v.x * grid_row(a, a.vid_grid, j, true).adv;
         }
-        const longlong2 ex = scan_pair(v, warp_tot, tot);
+        const longlong2 ex = scan_pair(v, warp_tot2, tot);
         if (j < a.n_vid) {
             vid_slices[j] = run.x + ex.x;
             vid_adv[j] = run.y + ex.y;
@@ -412,110 +380,94 @@ __global__ void __launch_bounds__(kRiCarryThreads) ri_carry_kernel(const __grid_
         vid_slices[a.n_vid] = run.x;
         vid_adv[a.n_vid] = run.y;
     }
-
-    // image / video runs of every sample (one warp per sample)
-    for (long long b = warp; b < a.B; b += nwarp) {
-        int carry_key = 0, n_img = 0, n_vid = 0;
-        for (int c0 = 0; c0 < a.tiles_per_row; c0 += 32) {
-            const RiTileView r = view_tile(a, b, c0 + lane, carry_key);
-            n_img += __shfl_sync(0xffffffffu, warp_incl_sum(r.img), 31);
-            n_vid += __shfl_sync(0xffffffffu, warp_incl_sum(r.vid), 31);
-        }
-        if (lane == 0) {
-            smp[b].img = n_img;
-            smp[b].vid = n_vid;
-        }
+    if (a.tiles_per_row == 0) {          // L = 0: no tiles, every delta is 0
+        for (long long b = threadIdx.x; b < a.B; b += blockDim.x) a.deltas[b] = 0;
+        return;
     }
     __syncthreads();
 
-    // runs of the batch before each sample
-    run = make_longlong2(0, 0);
-    for (long long c0 = 0; c0 < a.B; c0 += blockDim.x) {
-        const long long b = c0 + threadIdx.x;
-        longlong2 v{0, 0};
-        if (b < a.B) v = make_longlong2(smp[b].img, smp[b].vid);
-        const longlong2 ex = scan_pair(v, warp_tot, tot);
-        if (b < a.B) {
-            smp[b].img = (int)(run.x + ex.x);
-            smp[b].vid = (int)(run.y + ex.y);
-        }
-        run.x += tot.x;
-        run.y += tot.y;
-    }
-    __syncthreads();
+    const long long tiles = a.B * a.tiles_per_row;
+    int run_last_kept = 0;
+    RiSums run2{0, 0, 0, 0, 0};
+    for (long long c0 = 0; c0 < tiles; c0 += blockDim.x) {
+        const long long g = c0 + threadIdx.x;
+        const bool valid = g < tiles;
+        RiTileAgg r = RiTileAgg{0, 0, -1, -1, 0, 0, -1, 0, 0, 0, -1, 0};
+        if (valid) r = agg[g];
+        const long long b = valid ? g / a.tiles_per_row : 0;
+        const long long g0 = b * a.tiles_per_row;
+        const int t = (int)(g - g0);
 
-    // the state before every tile (one warp per sample)
-    for (long long b = warp; b < a.B; b += nwarp) {
-        const int img_s = smp[b].img, vid_s = smp[b].vid;
-        const long long base_adv = img_adv_before(a, img_s) + vid_adv_before(a, vid_s);
-        int carry_key = 0, k_run = 0, text_run = 0, img_run = img_s, vid_run = vid_s;
-        // the last run start before the current chunk
-        int o_k = 0, o_grid = -1;
-        long long o_start = 0;
-        for (int c0 = 0; c0 < a.tiles_per_row; c0 += 32) {
-            const int t = c0 + lane;
-            const RiTileView r = view_tile(a, b, t, carry_key);
-            const int k_inc = warp_incl_sum(r.g.kept), text_inc = warp_incl_sum(r.g.text);
-            const int img_inc = warp_incl_sum(r.img), vid_inc = warp_incl_sum(r.vid);
-            const int k0 = k_run + k_inc - r.g.kept, text0 = text_run + text_inc - r.g.text;
-            const int img0 = img_run + img_inc - r.img, vid0 = vid_run + vid_inc - r.vid;
-            const long long vadv0 = img_adv_before(a, img0) + vid_adv_before(a, vid0) - base_adv;
+        // 1. class of the last kept slot before the tile, within the sample
+        RiSums v1{0, 0, 0, 0, r.kept > 0 ? (int)((g + 1) * 4 + r.last_cls) : 0}, tot1;
+        RiSums ex1 = ri_block_exclusive(v1, warp_tot, tot1);
+        const int key = max(ex1.last, run_last_kept);
+        run_last_kept = max(run_last_kept, tot1.last);
+        const int prev = (key > 0 && (key >> 2) - 1 >= g0) ? (key & 3) : -1;
+        const bool fs = r.kept > 0 && r.first_cls != prev;
+        const int img_t = r.img + (fs && r.first_cls == 1), vid_t = r.vid + (fs && r.first_cls == 2);
+        const bool has = r.ls_off >= 0 || fs;
+
+        // 2. counts over the batch and the latest tile with a run start
+        RiSums v2{r.kept, r.text, img_t, vid_t, has ? (int)(g + 1) : 0}, tot2;
+        const RiSums ex2 = ri_op(run2, ri_block_exclusive(v2, warp_tot, tot2));
+        run2 = ri_op(run2, tot2);
+        if (valid && t == 0) {
+            smp[b].k_base = ex2.kept;
+            smp[b].text_base = ex2.text;
+            smp[b].img = ex2.img;
+            smp[b].vid = ex2.vid;
+        }
+        __syncthreads();
+
+        int k0 = 0, text0 = 0;
+        long long base_adv = 0;
+        if (valid) {
+            const RiSample sm = smp[b];
+            k0 = ex2.kept - sm.k_base;
+            text0 = ex2.text - sm.text_base;
+            base_adv = img_adv_before(a, sm.img) + vid_adv_before(a, sm.vid);
             // this tile's own last run start
-            const int has = r.g.ls_off >= 0 || r.first_start;
-            int my_k = 0, my_grid = -1;
-            long long my_start = 0;
+            int own_k = 0, own_grid = -1;
+            long long own_start = 0;
             if (has) {
-                const bool fs_img = r.first_start && r.g.first_cls == 1, fs_vid = r.first_start && r.g.first_cls == 2;
-                int off = 0, text_b = 0, ib = img0, vb = vid0, cls = r.g.first_cls;
-                if (r.g.ls_off >= 0) {
-                    off = r.g.ls_off;
-                    text_b = r.g.ls_text;
-                    ib = img0 + fs_img + r.g.ls_img;
-                    vb = vid0 + fs_vid + r.g.ls_vid;
-                    cls = r.g.ls_cls;
+                const bool fs_img = fs && r.first_cls == 1, fs_vid = fs && r.first_cls == 2;
+                int off = 0, text_b = 0, ib = ex2.img, vb = ex2.vid, cls = r.first_cls;
+                if (r.ls_off >= 0) {
+                    off = r.ls_off;
+                    text_b = r.ls_text;
+                    ib = ex2.img + fs_img + r.ls_img;
+                    vb = ex2.vid + fs_vid + r.ls_vid;
+                    cls = r.ls_cls;
                 }
-                my_k = k0 + off;
-                my_start = text0 + text_b + img_adv_before(a, ib) + vid_adv_before(a, vb) - base_adv;
-                my_grid = cls == 1 ? ib : cls == 2 ? vb : -1;
+                own_k = k0 + off;
+                own_start = text0 + text_b + img_adv_before(a, ib) + vid_adv_before(a, vb) - base_adv;
+                own_grid = cls == 1 ? ib : cls == 2 ? vb : -1;
             }
-            // the last start in an earlier tile: exclusive "latest" scan over lanes
-            const int src_inc = warp_incl_max(has ? lane + 1 : 0);
-            int src = __shfl_up_sync(0xffffffffu, src_inc, 1);
-            if (lane == 0) src = 0;
-            const int sl = src > 0 ? src - 1 : 0;
-            const int s_k = __shfl_sync(0xffffffffu, my_k, sl), s_grid = __shfl_sync(0xffffffffu, my_grid, sl);
-            const long long s_start = __shfl_sync(0xffffffffu, my_start, sl);
-            if (t < a.tiles_per_row) {
-                RiCarry cr;
-                cr.k0 = k0;
-                cr.text0 = text0;
-                cr.img0 = img0;
-                cr.vid0 = vid0;
-                cr.vadv0 = vadv0;
-                cr.prev_cls = r.prev;
-                cr.open_k = src > 0 ? s_k : o_k;
-                cr.open_grid = src > 0 ? s_grid : o_grid;
-                cr.open_start = src > 0 ? s_start : o_start;
-                cr.pad = 0;
-                static_cast<RiCarry *>(a.carry)[b * a.tiles_per_row + t] = cr;
-            }
-            // carry to the next chunk
-            const int last_src = __shfl_sync(0xffffffffu, src_inc, 31);
-            if (last_src > 0) {
-                o_k = __shfl_sync(0xffffffffu, my_k, last_src - 1);
-                o_grid = __shfl_sync(0xffffffffu, my_grid, last_src - 1);
-                o_start = __shfl_sync(0xffffffffu, my_start, last_src - 1);
-            }
-            k_run += __shfl_sync(0xffffffffu, k_inc, 31);
-            text_run += __shfl_sync(0xffffffffu, text_inc, 31);
-            img_run += __shfl_sync(0xffffffffu, img_inc, 31);
-            vid_run += __shfl_sync(0xffffffffu, vid_inc, 31);
+            carry[g].own_k = own_k;
+            carry[g].own_grid = own_grid;
+            carry[g].own_start = own_start;
         }
-        if (lane == 0) {
-            smp[b].kept = k_run;
-            smp[b].max_pos = -1;
-            smp[b].done = 0u;
-            if (a.tiles_per_row == 0) a.deltas[b] = 0;
+        __syncthreads();
+        if (valid) {
+            // the run open at the tile's first slot: the latest start before it, same sample
+            const long long src = (long long)ex2.last - 1;
+            const bool open = src >= g0;
+            RiCarry &cr = carry[g];
+            cr.k0 = k0;
+            cr.text0 = text0;
+            cr.img0 = ex2.img;
+            cr.vid0 = ex2.vid;
+            cr.vadv0 = img_adv_before(a, ex2.img) + vid_adv_before(a, ex2.vid) - base_adv;
+            cr.prev_cls = prev;
+            cr.open_k = open ? carry[src].own_k : 0;
+            cr.open_grid = open ? carry[src].own_grid : -1;
+            cr.open_start = open ? carry[src].own_start : 0;
+            if (t == a.tiles_per_row - 1) {
+                smp[b].kept = k0 + r.kept;
+                smp[b].max_pos = -1;
+                smp[b].done = 0u;
+            }
         }
     }
 }
