@@ -761,8 +761,9 @@ def next_rows(ipe, dev, stream, peak, reps):
 
 
 def end_to_end(ipe, torch, w, dev, stream, vin, tin, inv, steps, max_over_ranks, barrier):
-    """Same step with host inputs: H2D of every input from pinned memory and
-    D2H of every result inside the timed region."""
+    """Same step through the C ABI's host-buffer entry points: every input
+    copied in from pinned memory and every result copied back inside the
+    timed region."""
     t, v = w.text, w.vision
     N = v and sum(a * b * c for a, b, c in v.grid_thw)
 
@@ -781,14 +782,15 @@ def end_to_end(ipe, torch, w, dev, stream, vin, tin, inv, steps, max_over_ranks,
     bo = sum(x.numel() * x.element_size() for x in h_out.values())
 
     def step():
-        for k, x in h_in.items():
-            d[k].copy_(x, non_blocking=True)
-        ipe.vis_pos_interp(d["table"], v.grid_thw, v.merge, out=out, stream=stream)
-        ipe.vis_rope2d(d["qv"], d["kv"], v.grid_thw, v.merge, v.theta, stream=stream)
-        ipe.mrope_apply(d["Q"], d["K"], d["pos"], inv, t.section, True, stream=stream)
-        h_out["out"].copy_(out, non_blocking=True)
-        for k in ("qv", "kv", "Q", "K"):
-            h_out[k].copy_(d[k], non_blocking=True)
+        # the library's host-buffer entry points: chunks move in, through the
+        # kernels and back, both copy directions overlapping; the last call
+        # joins `stream`, so the step ends when every result is in host memory
+        ipe.vis_pos_interp_host(h_in["table"], v.grid_thw, h_out["out"], d["table"], out, v.merge,
+                                chunk_rows=16384, join=False, stream=stream)
+        ipe.vis_rope2d_host(h_in["qv"], h_in["kv"], v.grid_thw, d["qv"], d["kv"], v.merge, v.theta, h_out["qv"],
+                            h_out["kv"], chunk_rows=8192, join=False, stream=stream)
+        ipe.mrope_apply_host(h_in["Q"], h_in["K"], h_in["pos"], inv, t.section, True, d["Q"], d["K"], d["pos"],
+                             h_out["Q"], h_out["K"], chunk_tokens=4096, join=True, stream=stream)
 
     step()
     torch.cuda.synchronize()

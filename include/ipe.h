@@ -420,6 +420,61 @@ int ipe_vis_pos_interp_rope2d(const void *table, int grid_side, int hidden, void
                               double theta, ipe_dtype dtype, const int32_t *grid_thw_host,
                               int n_images, int merge, void *stream);
 
+/* ---------------------------------------------------------------------------
+ * Host-buffer entry points.  Not part of any page: the streaming runtime of
+ * this library around the same kernels.  The data moves host -> device,
+ * through the kernel and back in chunks, so that both copy directions and
+ * the kernels overlap:
+ *   copies in   on a library copy stream (one per device),
+ *   the kernel  on `stream`, after its chunk's copies in,
+ *   copies out  on a second library copy stream, after the kernel.
+ * Consecutive calls share the copy streams, so one call's copies also
+ * overlap the next call's.  Results are exactly those of the device entry
+ * points (the same kernels on each chunk).
+ *   *_host      host buffers; page-locked memory gives the overlap
+ *               (pageable memory works without it).  The out buffers may be
+ *               the in buffers.
+ *   *_dev       device staging buffers of the full size, caller-owned.  The
+ *               library remembers, per staging buffer, where the last
+ *               copies out of it end; a later call waits for them before
+ *               copying in again.
+ *   join        non-zero: `stream` waits for every copy out enqueued so far
+ *               on the device, so its completion means the results are in
+ *               host memory; zero: use ipe_host_join or a later call with
+ *               join set.
+ * The first call on a device creates its two copy streams and their events.
+ * Argument checks of the device calls apply to every chunk; a failed chunk
+ * stops the call with its status (earlier chunks stay enqueued).
+ * ------------------------------------------------------------------------- */
+
+/* `stream` waits for every copy out enqueued so far on the current device. */
+int ipe_host_join(void *stream);
+
+/* ipe_mrope_apply on host q [T, hq, head_dim] / k [T, hk, head_dim]
+ * (contiguous) and host positions [3, T], chunk_tokens tokens at a time;
+ * q_dev / k_dev: [T, hq / hk, head_dim]; positions_dev: 3 T int32 (each
+ * chunk's positions stored as [3, n] at offset 3 t0). */
+int ipe_mrope_apply_host(const void *q_host, const void *k_host, void *q_out_host, void *k_out_host,
+                         ipe_dtype dtype, int64_t T, int hq, int hk, int head_dim,
+                         const int32_t *positions_host, const float *inv_freq_host, int rot_dim,
+                         const int32_t *section, int interleaved, void *q_dev, void *k_dev,
+                         int32_t *positions_dev, int64_t chunk_tokens, int join, void *stream);
+
+/* ipe_vis_rope2d on host q / k [N, heads, head_dim] (contiguous); chunks of
+ * whole images up to chunk_rows patches, an image above that split into
+ * frame ranges.  k_host / k_out_host / k_dev may be NULL together. */
+int ipe_vis_rope2d_host(const void *q_host, const void *k_host, void *q_out_host, void *k_out_host,
+                        ipe_dtype dtype, int heads, int head_dim, const int32_t *grid_thw_host,
+                        int n_images, int merge, double theta, void *q_dev, void *k_dev,
+                        int64_t chunk_rows, int join, void *stream);
+
+/* ipe_vis_pos_interp from a host table [G*G, hidden] to host out [N, hidden];
+ * the table moves in once, the output comes back in chunks as for
+ * ipe_vis_rope2d_host. */
+int ipe_vis_pos_interp_host(const void *table_host, ipe_dtype dtype, int grid_side, int hidden,
+                            const int32_t *grid_thw_host, int n_images, int merge, void *out_host,
+                            void *table_dev, void *out_dev, int64_t chunk_rows, int join, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

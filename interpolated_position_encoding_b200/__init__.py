@@ -42,6 +42,10 @@ _SIGS = {
     "ipe_apply_rotary_partial_hf": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, _I, _P]),
     "ipe_mrope_apply_hf": (_I, [_P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _P, _P, _I, _P, _I, _P]),
     "ipe_vis_pos_interp_hf": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P]),
+    "ipe_host_join": (_I, [_P]),
+    "ipe_mrope_apply_host": (_I, [_P, _P, _P, _P, _I, _I64, _I, _I, _I, _P, _P, _I, _P, _I, _P, _P, _P, _I64, _I, _P]),
+    "ipe_vis_rope2d_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _I, _I, _D, _P, _P, _I64, _I, _P]),
+    "ipe_vis_pos_interp_host": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P, _P, _I64, _I, _P]),
     "ipe_mrope_decode": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _I64, _I64, _I64, _P, _P, _P, _P, ctypes.c_float, _P,
                               _I, _P, _P, _I64, _I64, _P, _P]),
     "ipe_mrope_rope_index": (_I, [_P, _P, _I, _I64, _I64, _P, _I, _P, _I, _I, _I, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -419,6 +423,78 @@ def mrope_rope_index_static(mm_token_type_ids, image_grid_thw, video_grid_thw, a
                                             int(spatial_merge_size), _ptr(position_ids), _ptr(rope_deltas),
                                             _stream(stream)))
     return position_ids, rope_deltas
+
+
+# ------------------------------------------------------ host buffers
+
+
+def _host(t, name):
+    if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous host tensor (page-locked for overlap)")
+    return t
+
+
+def _dev_like(t, host, name):
+    _cuda(t, name)
+    if t.numel() * t.element_size() < host.numel() * host.element_size() or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous device tensor at least the size of its host buffer")
+    return t
+
+
+def host_join(stream=None):
+    """The stream waits for every copy back to the host enqueued so far."""
+    _check(_lib.ipe_host_join(_stream(stream)))
+
+
+def mrope_apply_host(q, k, positions, inv_freq, section, interleaved, q_dev, k_dev, positions_dev, q_out=None,
+                     k_out=None, chunk_tokens=8192, join=True, stream=None):
+    """mrope_apply on host tensors q [T, hq, D], k [T, hk, D], positions [3, T]
+    (int32), streamed through the device buffers in chunks; results land in
+    q_out / k_out (default: in place)."""
+    _host(q, "q"), _host(k, "k"), _host(positions, "positions")
+    q_out = q if q_out is None else _host(q_out, "q_out")
+    k_out = k if k_out is None else _host(k_out, "k_out")
+    T, hq, D = q.shape
+    hk = k.shape[1]
+    _dev_like(q_dev, q, "q_dev"), _dev_like(k_dev, k, "k_dev"), _dev_like(positions_dev, positions, "positions_dev")
+    inv, half = _inv_host(inv_freq)
+    _check(_lib.ipe_mrope_apply_host(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _dtype_code(q), T, hq, hk, D,
+                                     _ptr(positions), inv, 2 * half, _i32_host(section, 3), int(bool(interleaved)),
+                                     _ptr(q_dev), _ptr(k_dev), _ptr(positions_dev), int(chunk_tokens), int(bool(join)),
+                                     _stream(stream)))
+    return q_out, k_out
+
+
+def vis_rope2d_host(q, k, grid_thw, q_dev, k_dev, merge=2, theta=1e4, q_out=None, k_out=None, chunk_rows=16384,
+                    join=True, stream=None):
+    """vis_rope2d on host tensors q / k [N, heads, head_dim], streamed in chunks."""
+    _host(q, "q")
+    q_out = q if q_out is None else _host(q_out, "q_out")
+    if k is not None:
+        _host(k, "k")
+        k_out = k if k_out is None else _host(k_out, "k_out")
+    g, n = _grid_host(grid_thw)
+    _, heads, hd = q.shape
+    _dev_like(q_dev, q, "q_dev")
+    if k is not None:
+        _dev_like(k_dev, k, "k_dev")
+    _check(_lib.ipe_vis_rope2d_host(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _dtype_code(q), heads, hd, g, n,
+                                    int(merge), float(theta), _ptr(q_dev), _ptr(k_dev) if k is not None else None,
+                                    int(chunk_rows), int(bool(join)), _stream(stream)))
+    return q_out, k_out
+
+
+def vis_pos_interp_host(table, grid_thw, out, table_dev, out_dev, merge=2, chunk_rows=16384, join=True,
+                        stream=None):
+    """vis_pos_interp from a host table to a host output, streamed in chunks."""
+    _host(table, "table"), _host(out, "out")
+    g, n = _grid_host(grid_thw)
+    G = int(round(table.shape[0] ** 0.5))
+    _dev_like(table_dev, table, "table_dev"), _dev_like(out_dev, out, "out_dev")
+    _check(_lib.ipe_vis_pos_interp_host(_ptr(table), _dtype_code(table), G, table.shape[1], g, n, int(merge),
+                                        _ptr(out), _ptr(table_dev), _ptr(out_dev), int(chunk_rows), int(bool(join)),
+                                        _stream(stream)))
+    return out
 
 
 # ------------------------------------------------------------------- vision
