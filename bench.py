@@ -776,10 +776,12 @@ def end_to_end(ipe, torch, w, dev, stream, vin, tin, inv, steps, max_over_ranks,
     d = {k: torch.empty_like(x, device=dev) for k, x in h_in.items()}
     out = torch.empty(N, v.hidden, dtype=torch.bfloat16, device=dev)
     h_out = {"out": torch.empty(N, v.hidden, dtype=torch.bfloat16).pin_memory(),
-             "qv": torch.empty_like(h_in["qv"]).pin_memory(), "kv": torch.empty_like(h_in["kv"]).pin_memory(),
-             "Q": torch.empty_like(h_in["Q"]).pin_memory(), "K": torch.empty_like(h_in["K"]).pin_memory()}
-    bi = sum(x.numel() * x.element_size() for x in h_in.values())
-    bo = sum(x.numel() * x.element_size() for x in h_out.values())
+             "qv": torch.empty_like(h_in["qv"]).pin_memory(), "kv": torch.empty_like(h_in["kv"]).pin_memory()}
+    # bytes that cross the link per step: the vision tensors whole, the text
+    # Q / K rotary slices only (rotated in place on the host), positions in
+    text_slices = t.T * (t.hq + t.hk) * t.rot_dim * 2
+    bi = sum(h_in[k].numel() * h_in[k].element_size() for k in ("table", "qv", "kv", "pos")) + text_slices
+    bo = sum(x.numel() * x.element_size() for x in h_out.values()) + text_slices
 
     def step():
         # the library's host-buffer entry points: chunks move in, through the
@@ -789,8 +791,9 @@ def end_to_end(ipe, torch, w, dev, stream, vin, tin, inv, steps, max_over_ranks,
                                 chunk_rows=16384, join=False, stream=stream)
         ipe.vis_rope2d_host(h_in["qv"], h_in["kv"], v.grid_thw, d["qv"], d["kv"], v.merge, v.theta, h_out["qv"],
                             h_out["kv"], chunk_rows=8192, join=False, stream=stream)
+        # in place on the host Q / K: only the rotary slices cross the link
         ipe.mrope_apply_host(h_in["Q"], h_in["K"], h_in["pos"], inv, t.section, True, d["Q"], d["K"], d["pos"],
-                             h_out["Q"], h_out["K"], chunk_tokens=4096, join=True, stream=stream)
+                             chunk_tokens=4096, join=True, stream=stream)
 
     step()
     torch.cuda.synchronize()

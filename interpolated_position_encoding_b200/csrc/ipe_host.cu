@@ -262,20 +262,27 @@ int ipe_mrope_apply_host(const void *q_host, const void *k_host, void *q_out_hos
         return ipe::set_error(IPE_EINVAL, "a buffer is NULL");
     const size_t eb = elem_size(dtype);
     const size_t qrow = (size_t)hq * head_dim * eb, krow = (size_t)hk * head_dim * eb;
+    // In place (out == in), channels past rot_dim never change: only the
+    // rotary slice of each head row crosses the link, as a strided copy
+    // (rows of rot_dim elements, pitch head_dim), into the same place of the
+    // staging buffer.  Otherwise whole token rows move.
+    const bool slices = q_out_host == q_host && k_out_host == k_host && rot_dim > 0 && rot_dim < head_dim;
+    const size_t hrow = (size_t)head_dim * eb, srow = slices ? (size_t)rot_dim * eb : hrow;
     cudaStream_t s = (cudaStream_t)stream;
     return pipelined({q_dev, k_dev, positions_dev}, join, s, [&](Pipe &p) -> int {
         for (long long t0 = 0; t0 < T; t0 += chunk_tokens) {
             const long long n = T - t0 < chunk_tokens ? T - t0 : chunk_tokens;
             char *dq = static_cast<char *>(q_dev) + t0 * qrow, *dk = static_cast<char *>(k_dev) + t0 * krow;
             int32_t *dpos = positions_dev + 3 * t0;   // this chunk's positions, [3, n]
+            const size_t nq = hq ? (size_t)n * hq : 0, nk = hk ? (size_t)n * hk : 0;   // head rows
             std::vector<Copy> in = {
-                {dq, qrow, static_cast<const char *>(q_host) + t0 * qrow, qrow, qrow, (size_t)(hq ? n : 0)},
-                {dk, krow, static_cast<const char *>(k_host) + t0 * krow, krow, krow, (size_t)(hk ? n : 0)},
+                {dq, hrow, static_cast<const char *>(q_host) + t0 * qrow, hrow, srow, nq},
+                {dk, hrow, static_cast<const char *>(k_host) + t0 * krow, hrow, srow, nk},
                 {dpos, (size_t)n * 4, positions_host + t0, (size_t)T * 4, (size_t)n * 4, 3},
             };
             std::vector<Copy> out = {
-                {static_cast<char *>(q_out_host) + t0 * qrow, qrow, dq, qrow, qrow, (size_t)(hq ? n : 0)},
-                {static_cast<char *>(k_out_host) + t0 * krow, krow, dk, krow, krow, (size_t)(hk ? n : 0)},
+                {static_cast<char *>(q_out_host) + t0 * qrow, hrow, dq, hrow, srow, nq},
+                {static_cast<char *>(k_out_host) + t0 * krow, hrow, dk, hrow, srow, nk},
             };
             int rc = run_chunk(p, s, in, [&]() {
                 return ipe_mrope_apply(hq ? dq : nullptr, hk ? dk : nullptr, dtype, n, hq, hk, head_dim,

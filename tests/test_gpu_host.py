@@ -41,6 +41,25 @@ def test_mrope_apply_host_matches_device(T, chunk):
         assert torch.equal(q_out, want_q.cpu()) and torch.equal(k_out, want_k.cpu())
 
 
+@pytest.mark.parametrize("rot", [64, 128])
+def test_mrope_apply_host_in_place(rot):
+    # in place only the rotary slices cross the link; the rest stays as it was
+    rng = np.random.default_rng([rot, 9])
+    T, hq, hk, D = 3000, 4, 2, 128
+    inv = ipe.rope_inv_freq(rot, 1e6)
+    sec = (rot // 2 - 2 * (rot // 6), rot // 6, rot // 6)
+    q, k = _bf16(rng, (T, hq, D)).pin_memory(), _bf16(rng, (T, hk, D)).pin_memory()
+    pos = torch.from_numpy(rng.integers(0, 50000, (3, T)).astype(np.int32)).pin_memory()
+    want_q, want_k = q.cuda(), k.cuda()
+    ipe.mrope_apply(want_q, want_k, pos.cuda(), inv, sec, True)
+    q_dev, k_dev = torch.empty_like(want_q), torch.empty_like(want_k)
+    p_dev = torch.empty(3, T, dtype=torch.int32, device="cuda")
+    ipe.mrope_apply_host(q, k, pos, inv, sec, True, q_dev, k_dev, p_dev, chunk_tokens=1000)
+    torch.cuda.synchronize()
+    ipe.device_status()
+    assert torch.equal(q, want_q.cpu()) and torch.equal(k, want_k.cpu())
+
+
 def test_vis_rope2d_host_groups_and_splits():
     # small images grouped into chunks, a video split into frame ranges
     grid = [(1, 16, 16), (1, 8, 12), (6, 16, 20), (1, 4, 4), (2, 10, 10)]
