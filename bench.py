@@ -294,6 +294,8 @@ CASES = {
     "qk_norm_mrope": "fused QK-RMSNorm + MRoPE on text_t32768_omni (Q [32768, 32, 128], K [32768, 4, 128] bf16)",
     "rope_index": "device position table of the large-prefill request (B = 1, L = 131072, 16 video slices)",
     "mrope_decode": "decode step, B = 256, Q [256, 24, 256], K / V [256, 4, 256] bf16, norm + KV-cache write",
+    "mrope_cos_sin": "cos / sin tables of the large-prefill request (T = 131072, rot 64, interleaved)",
+    "vis_pos_interp_batch8": "interpolation of the batch of 8 single images (bf16 table, N = 26528)",
 }
 
 
@@ -330,6 +332,22 @@ def run_case(args):
         ws = torch.empty(ipe.rope_index_workspace_bytes(B, L, 0, vid.shape[0]), dtype=torch.uint8, device=dev)
         fn = lambda: ipe.mrope_rope_index(gty, None, gvg, None, t.merge, posb, dl, ws, stream=stream)  # noqa: E731
         nbytes = B * L * 16 + B * 4
+    elif name == "mrope_cos_sin":
+        w = wl.WORKLOADS[WORKLOAD]
+        t = w.text
+        pos = torch.from_numpy(wl.text_inputs(w, with_qk=False)["positions"]).to(dev)
+        inv = ipe.rope_inv_freq(t.rot_dim, t.theta)
+        cos = torch.empty(t.T, t.rot_dim, dtype=torch.float32, device=dev)
+        sin = torch.empty_like(cos)
+        fn = lambda: ipe.mrope_cos_sin(pos, inv, t.section, True, cos, sin, stream=stream)  # noqa: E731
+        nbytes = 3 * t.T * 4 + 2 * t.T * t.rot_dim * 4
+    elif name == "vis_pos_interp_batch8":
+        w = wl.WORKLOADS["vision_batch8_bf16"]
+        v = w.vision
+        table = torch.from_numpy(wl.vision_inputs(w)["table"].view(np.int16)).view(torch.bfloat16).to(dev)
+        out = torch.empty(wl.n_patches(v), v.hidden, dtype=torch.bfloat16, device=dev)
+        fn = lambda: ipe.vis_pos_interp(table, v.grid_thw, v.merge, out=out, stream=stream)  # noqa: E731
+        nbytes = algorithmic_bytes_vision(v)
     else:
         t = wl.WORKLOADS[WORKLOAD].text
         B, D = 256, t.head_dim

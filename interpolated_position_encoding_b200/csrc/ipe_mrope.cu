@@ -34,11 +34,17 @@ cudaError_t launch_mrope_axis_map(int half, const int *section, int interleaved,
 // takes U tokens per pass (their position loads in flight together) and
 // writes both halves of cat(f, f) for cos and sin with V-wide stores.
 template <int V>
-__global__ void __launch_bounds__(256) mrope_cos_sin_kernel(const __grid_constant__ MropeAngles a, int half,
-                                                             float *__restrict__ cos_out,
-                                                             float *__restrict__ sin_out)
+#ifndef IPE_CS_MIN_BLOCKS
+#define IPE_CS_MIN_BLOCKS 6
+#endif
+#ifndef IPE_CS_TOKENS
+#define IPE_CS_TOKENS 1
+#endif
+__global__ void __launch_bounds__(256, IPE_CS_MIN_BLOCKS) mrope_cos_sin_kernel(const __grid_constant__ MropeAngles a,
+                                                                               int half, float *__restrict__ cos_out,
+                                                                               float *__restrict__ sin_out)
 {
-    constexpr int U = 2;
+    constexpr int U = IPE_CS_TOKENS;
     const int j0 = threadIdx.x * V;
     int ax[V];
     float inv[V];
@@ -85,7 +91,7 @@ static cudaError_t cos_sin_vec(const MropeAngles &a, int half, float *cos_out, f
 {
     const int gx = half / V;
     const int gy = std::max(1, 256 / gx);
-    const long long need = (a.T + 2LL * gy - 1) / (2LL * gy);     // 2 tokens per thread and pass
+    const long long need = (a.T + (long long)IPE_CS_TOKENS * gy - 1) / ((long long)IPE_CS_TOKENS * gy);
     const int blocks = (int)std::max<long long>(1, std::min(need, (long long)sm_count() * 8));
     mrope_cos_sin_kernel<V><<<blocks, dim3(gx, gy), 0, s>>>(a, half, cos_out, sin_out);
     return cudaGetLastError();
