@@ -16,21 +16,20 @@
 
 namespace ipe {
 
-#ifndef IPE_QK_UNROLL
-#define IPE_QK_UNROLL 4
-#endif
-#ifndef IPE_QK_MIN_BLOCKS
-#define IPE_QK_MIN_BLOCKS 3
-#endif
 constexpr int kQkWarps = 8;
-constexpr int kQkUnroll = IPE_QK_UNROLL;     // head rows per lane in flight
+// Rows in flight per lane and blocks per SM, by lanes per row (measured:
+// 256-channel bf16 rows prefer four rows at three blocks per SM, narrower
+// rows two rows at four blocks per SM).
+constexpr int qk_unroll(int lpr) { return lpr >= 32 ? 4 : 2; }
+constexpr int qk_min_blocks(int lpr) { return lpr >= 32 ? 3 : 4; }
 
 template <typename T, int LPR>
-__global__ void __launch_bounds__(32 * kQkWarps, IPE_QK_MIN_BLOCKS)
+__global__ void __launch_bounds__(32 * kQkWarps, qk_min_blocks(LPR))
     qk_norm_mrope_kernel(const __grid_constant__ QkNormArgs n, const __grid_constant__ MropeAngles a)
 {
     constexpr int EC = QkElem<T>::EC;
     constexpr int NP = EC / 2;                        // fp32 pairs of a 16-byte chunk
+    constexpr int kQkUnroll = qk_unroll(LPR);
     constexpr int RPW = 32 / LPR;                     // head rows per warp access
     extern __shared__ float4 qk_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
