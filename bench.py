@@ -296,6 +296,8 @@ CASES = {
     "mrope_decode": "decode step, B = 256, Q [256, 24, 256], K / V [256, 4, 256] bf16, norm + KV-cache write",
     "mrope_cos_sin": "cos / sin tables of the large-prefill request (T = 131072, rot 64, interleaved)",
     "vis_pos_interp_batch8": "interpolation of the batch of 8 single images (bf16 table, N = 26528)",
+    "fill_reference": "torch fill_ of the 67 MB the cos / sin kernel writes at T = 131072, rot 64 (a write-stream "
+                      "reference for that kernel; not a library kernel)",
 }
 
 
@@ -348,6 +350,11 @@ def run_case(args):
         out = torch.empty(wl.n_patches(v), v.hidden, dtype=torch.bfloat16, device=dev)
         fn = lambda: ipe.vis_pos_interp(table, v.grid_thw, v.merge, out=out, stream=stream)  # noqa: E731
         nbytes = algorithmic_bytes_vision(v)
+    elif name == "fill_reference":
+        t = wl.WORKLOADS[WORKLOAD].text
+        buf = torch.empty(2 * t.T * t.rot_dim, dtype=torch.float32, device=dev)
+        fn = lambda: buf.fill_(1.5)  # noqa: E731
+        nbytes = buf.numel() * 4
     else:
         t = wl.WORKLOADS[WORKLOAD].text
         B, D = 256, t.head_dim

@@ -33,18 +33,17 @@ cudaError_t launch_mrope_axis_map(int half, const int *section, int interleaved,
 // consecutive frequencies of a token, threadIdx.y a token.  Each thread
 // takes U tokens per pass (their position loads in flight together) and
 // writes both halves of cat(f, f) for cos and sin with V-wide stores.
+// Write-stream bound: the 67 MB of tables at rot 64 / T = 131072 take about
+// 1.2x the time of a plain fill of the same size.  Measured best: one token
+// per pass, six 256-thread blocks per SM, one resident wave.
+constexpr int kCsTokens = 1;
+
 template <int V>
-#ifndef IPE_CS_MIN_BLOCKS
-#define IPE_CS_MIN_BLOCKS 6
-#endif
-#ifndef IPE_CS_TOKENS
-#define IPE_CS_TOKENS 1
-#endif
-__global__ void __launch_bounds__(256, IPE_CS_MIN_BLOCKS) mrope_cos_sin_kernel(const __grid_constant__ MropeAngles a,
+__global__ void __launch_bounds__(256, 6) mrope_cos_sin_kernel(const __grid_constant__ MropeAngles a,
                                                                                int half, float *__restrict__ cos_out,
                                                                                float *__restrict__ sin_out)
 {
-    constexpr int U = IPE_CS_TOKENS;
+    constexpr int U = kCsTokens;
     const int j0 = threadIdx.x * V;
     int ax[V];
     float inv[V];
@@ -54,8 +53,9 @@ __global__ void __launch_bounds__(256, IPE_CS_MIN_BLOCKS) mrope_cos_sin_kernel(c
         inv[e] = a.inv[j0 + e];
     }
     const long long stride = (long long)gridDim.x * blockDim.y;
-    for (long long t0 = (long long)blockIdx.x * blockDim.y + threadIdx.y; t0 < a.T; t0 += U * stride) {
-        int p0[U], p1[U], p2[U];
+    // positions of the next pass are loaded while this pass computes
+    int p0[U], p1[U], p2[U];
+    auto load = [&](long long t0) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const long long t = t0 + u * stride;
@@ -65,6 +65,18 @@ __global__ void __launch_bounds__(256, IPE_CS_MIN_BLOCKS) mrope_cos_sin_kernel(c
                 p2[u] = __ldg(a.positions + 2 * a.T + t);
             }
         }
+    };
+    long long t0 = (long long)blockIdx.x * blockDim.y + threadIdx.y;
+    if (t0 < a.T) load(t0);
+    for (; t0 < a.T; t0 += U * stride) {
+        int q0[U], q1[U], q2[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            q0[u] = p0[u];
+            q1[u] = p1[u];
+            q2[u] = p2[u];
+        }
+        if (t0 + U * stride < a.T) load(t0 + U * stride);
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const long long t = t0 + u * stride;
@@ -72,7 +84,7 @@ __global__ void __launch_bounds__(256, IPE_CS_MIN_BLOCKS) mrope_cos_sin_kernel(c
             Pack<float, V> c, s;
 #pragma unroll
             for (int e = 0; e < V; ++e) {
-                const int pos = ax[e] == 0 ? p0[u] : (ax[e] == 1 ? p1[u] : p2[u]);
+                const int pos = ax[e] == 0 ? q0[u] : (ax[e] == 1 ? q1[u] : q2[u]);
                 const float angle = __fmul_rn(__int2float_rn(pos), inv[e]);
                 sincosf(angle, &s.v[e], &c.v[e]);
             }
@@ -91,8 +103,12 @@ static cudaError_t cos_sin_vec(const MropeAngles &a, int half, float *cos_out, f
 {
     const int gx = half / V;
     const int gy = std::max(1, 256 / gx);
-    const long long need = (a.T + (long long)IPE_CS_TOKENS * gy - 1) / ((long long)IPE_CS_TOKENS * gy);
-    const int blocks = (int)std::max<long long>(1, std::min(need, (long long)sm_count() * 8));
+    const long long need = (a.T + (long long)kCsTokens * gy - 1) / ((long long)kCsTokens * gy);
+    // one resident wave: no second, partial wave to wait for at the end
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mrope_cos_sin_kernel<V>, gx * gy, 0);
+    if (e != cudaSuccess) return e;
+    const int blocks = (int)std::max<long long>(1, std::min(need, (long long)sm_count() * std::max(per_sm, 1)));
     mrope_cos_sin_kernel<V><<<blocks, dim3(gx, gy), 0, s>>>(a, half, cos_out, sin_out);
     return cudaGetLastError();
 }
