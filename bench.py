@@ -296,6 +296,8 @@ CASES = {
     "mrope_decode": "decode step, B = 256, Q [256, 24, 256], K / V [256, 4, 256] bf16, norm + KV-cache write",
     "mrope_cos_sin": "cos / sin tables of the large-prefill request (T = 131072, rot 64, interleaved)",
     "vis_pos_interp_batch8": "interpolation of the batch of 8 single images (bf16 table, N = 26528)",
+    "mrope_apply_short": "fused MRoPE on the 4096-token prompt (text_t4096_qwen35: Q [4096, 24, 256], K [4096, 4, 256])",
+    "qk_norm_mrope_short": "fused QK-RMSNorm + MRoPE on the 4096-token prompt (text_t4096_qwen35)",
     "fill_reference": "torch fill_ of the 67 MB the cos / sin kernel writes at T = 131072, rot 64 (a write-stream "
                       "reference for that kernel; not a library kernel)",
 }
@@ -350,6 +352,21 @@ def run_case(args):
         out = torch.empty(wl.n_patches(v), v.hidden, dtype=torch.bfloat16, device=dev)
         fn = lambda: ipe.vis_pos_interp(table, v.grid_thw, v.merge, out=out, stream=stream)  # noqa: E731
         nbytes = algorithmic_bytes_vision(v)
+    elif name in ("mrope_apply_short", "qk_norm_mrope_short"):
+        w = wl.WORKLOADS["text_t4096_qwen35"]
+        t = w.text
+        tin = wl.text_inputs(w)
+        Q = torch.from_numpy(tin["q"].view(np.int16)).view(torch.bfloat16).to(dev)
+        K = torch.from_numpy(tin["k"].view(np.int16)).view(torch.bfloat16).to(dev)
+        pos = torch.from_numpy(tin["positions"]).to(dev)
+        inv = ipe.rope_inv_freq(t.rot_dim, t.theta)
+        if name == "mrope_apply_short":
+            fn = lambda: ipe.mrope_apply(Q, K, pos, inv, t.section, True, stream=stream)  # noqa: E731
+            nbytes = (t.hq + t.hk) * t.T * t.rot_dim * 2 * 2 + 3 * t.T * 4
+        else:
+            wq = torch.ones(t.head_dim, dtype=torch.bfloat16, device=dev)
+            fn = lambda: ipe.qk_norm_mrope(Q, K, wq, wq, pos, inv, t.section, True, stream=stream)  # noqa: E731
+            nbytes = (t.hq + t.hk) * t.T * t.head_dim * 2 * 2 + 3 * t.T * 4
     elif name == "fill_reference":
         t = wl.WORKLOADS[WORKLOAD].text
         buf = torch.empty(2 * t.T * t.rot_dim, dtype=torch.float32, device=dev)

@@ -106,6 +106,7 @@ struct QkNormArgs {
     long long q_stride, k_stride;
     int hq, hk, head_dim, half, half_pad;
     float eps;
+    int groups, rows_per_item;        // a token's head rows split over `groups` warps (set by the launcher)
 };
 
 cudaError_t launch_qk_norm_mrope(bool bf16, const QkNormArgs &n, const MropeAngles &a, cudaStream_t s);

@@ -7,8 +7,8 @@
 // explains why the two are worth fusing: they run back to back on every
 // q and k of every full-attention layer.
 //
-// One warp per token.  The warp writes the token's (cos, sin) pairs into its
-// shared-memory slot once; each head row is then held by LPR = D / EC lanes
+// One warp per token (for short sequences, per token and group of head rows).
+// The warp writes the token's (cos, sin) pairs into its shared-memory slot once; each head row is then held by LPR = D / EC lanes
 // (EC elements = 16 bytes per lane), its sum of squares reduced with
 // shuffles inside those lanes, and the rotary partner of a chunk fetched from
 // the lane half a rotary slice away.  All D channels are written back.
@@ -50,8 +50,13 @@ __global__ void __launch_bounds__(32 * kQkWarps, qk_min_blocks(LPR))
     const Pack<uint32_t, 4> wq = ld_pack<uint32_t, 4>(reinterpret_cast<const uint32_t *>(static_cast<const T *>(n.q_weight) + e0));
     const Pack<uint32_t, 4> wk = ld_pack<uint32_t, 4>(reinterpret_cast<const uint32_t *>(static_cast<const T *>(n.k_weight) + e0));
     const int H = n.hq + n.hk;
-    const long long stride = (long long)gridDim.x * kQkWarps;
-    for (long long t = (long long)blockIdx.x * kQkWarps + warp; t < n.T; t += stride) {
+    // this warp's group of head rows (the grid holds a multiple of `groups`
+    // warps, so the group stays fixed while the warp strides over tokens)
+    const int gw = blockIdx.x * kQkWarps + warp;
+    const int hbeg = (gw % n.groups) * n.rows_per_item;
+    const int hend = min(H, hbeg + n.rows_per_item);
+    const long long tstride = (long long)gridDim.x * kQkWarps / n.groups;
+    for (long long t = gw / n.groups; t < n.T; t += tstride) {
         Pack<uint32_t, 4> x[kQkUnroll];
         // this lane's chunk of head row h of token t
         auto chunk_ptr = [&](int h) {
@@ -59,12 +64,12 @@ __global__ void __launch_bounds__(32 * kQkWarps, qk_min_blocks(LPR))
                               : static_cast<T *>(n.k) + t * n.k_stride + (long long)(h - n.hq) * D;
             return reinterpret_cast<uint32_t *>(row + e0);
         };
-        // rows h0 + u * RPW + sub of token t (zeros past the last head)
+        // rows h0 + u * RPW + sub of token t (zeros past the item's last row)
         auto load_group = [&](int h0) {
 #pragma unroll
             for (int u = 0; u < kQkUnroll; ++u) {
                 const int h = h0 + u * RPW + sub;
-                if (h < H) {
+                if (h < hend) {
                     x[u] = ld_pack<uint32_t, 4>(chunk_ptr(h));
                 } else {
 #pragma unroll
@@ -73,7 +78,7 @@ __global__ void __launch_bounds__(32 * kQkWarps, qk_min_blocks(LPR))
             }
         };
         // the first rows are in flight while the angles are computed
-        load_group(0);
+        load_group(hbeg);
         // (cos, sin) of every frequency of token t
         for (int j = lane; j < half; j += 32) {
             const int ax = mrope_axis(j, a.section, a.interleaved);
@@ -90,12 +95,12 @@ __global__ void __launch_bounds__(32 * kQkWarps, qk_min_blocks(LPR))
             const float2 sv = rotary ? make_float2(cs_s[j0 + 2 * i], cs_s[j0 + 2 * i + 1]) : make_float2(0.f, 0.f);
             si[i] = first_half ? make_float2(-sv.x, -sv.y) : sv;
         }
-        for (int h0 = 0; h0 < H; h0 += RPW * kQkUnroll) {
-            if (h0 > 0) load_group(h0);
+        for (int h0 = hbeg; h0 < hend; h0 += RPW * kQkUnroll) {
+            if (h0 > hbeg) load_group(h0);
 #pragma unroll
             for (int u = 0; u < kQkUnroll; ++u) {
                 // every lane of the warp takes part in the shuffles, rows past
-                // H included (zeros; never stored)
+                // the item's last included (zeros; never stored)
                 const int h = h0 + u * RPW + sub;
                 const bool is_q = h < n.hq;
                 uint32_t w[4];
@@ -103,7 +108,7 @@ __global__ void __launch_bounds__(32 * kQkWarps, qk_min_blocks(LPR))
                 for (int i = 0; i < 4; ++i) w[i] = is_q ? wq.v[i] : wk.v[i];
                 const Pack<uint32_t, 4> y = rms_norm_chunk<T, LPR>(x[u], w, inv_d, n.eps);
                 const Pack<uint32_t, 4> o = rotate_row_chunk<T>(y, co, si, partner);
-                if (h < H) st_pack<uint32_t, 4>(chunk_ptr(h), o);
+                if (h < hend) st_pack<uint32_t, 4>(chunk_ptr(h), o);
             }
         }
         __syncwarp();
@@ -118,9 +123,22 @@ static cudaError_t qk_launch(const QkNormArgs &n, const MropeAngles &a, cudaStre
     int per_sm = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32 * kQkWarps, smem);
     if (e != cudaSuccess) return e;
-    const long long need = (n.T + kQkWarps - 1) / kQkWarps;
-    const int blocks = (int)std::max<long long>(1, std::min(need, (long long)sm_count() * std::max(per_sm, 1)));
-    kern<<<blocks, 32 * kQkWarps, smem, s>>>(n, a);
+    // Short sequences: a token's head rows are split over several warps
+    // (whole passes of RPW x unroll rows each) until there are about four
+    // warps per resident warp slot; long ones keep one warp per token.
+    QkNormArgs m = n;
+    const int unit = (32 / LPR) * qk_unroll(LPR);
+    const int H = n.hq + n.hk;
+    const int max_groups = (H + unit - 1) / unit;
+    const long long want = 4LL * sm_count() * std::max(per_sm, 1) * kQkWarps;
+    int groups = 1;
+    while (groups < max_groups && n.T * groups < want) ++groups;
+    m.rows_per_item = ((H + groups - 1) / groups + unit - 1) / unit * unit;
+    m.groups = (H + m.rows_per_item - 1) / m.rows_per_item;
+    const long long need = (n.T * m.groups + kQkWarps - 1) / kQkWarps;
+    long long blocks = std::max<long long>(1, std::min(need, (long long)sm_count() * std::max(per_sm, 1)));
+    blocks = (blocks + m.groups - 1) / m.groups * m.groups;   // a whole number of groups per stride
+    kern<<<(unsigned)blocks, 32 * kQkWarps, smem, s>>>(m, a);
     return cudaGetLastError();
 }
 
