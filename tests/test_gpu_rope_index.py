@@ -107,6 +107,37 @@ def test_multi_tile_batches(orc, B, L, pad):
     check(orc, keep_all, None, img, vid)
 
 
+def _many_images_batch(rng, B, L):
+    """B samples of L slots, each a run of small images (2 x 2 merged slots)
+    between single text slots, with a few padded slots at the end."""
+    types = np.zeros((B, L), np.int64)
+    mask = np.ones((B, L), np.int64)
+    img = []
+    for b in range(B):
+        l = 0
+        while l + 6 <= L - 4:
+            types[b, l + 1:l + 5] = 1          # text, then a (1, 4, 4) image: 4 slots
+            img.append([1, 4, 4])
+            l += 5 + int(rng.integers(0, 3))
+        mask[b, L - int(rng.integers(0, 4)):] = 0
+    return types, mask, np.array(img, np.int64)
+
+
+def test_carry_scan_over_many_chunks(orc):
+    # more than 1024 tiles (the carry pass scans them 1024 at a time) and
+    # runs, padding and samples crossing those chunk boundaries
+    types, mask, img, vid = _long_batch(np.random.default_rng(77), 520, 2100, 400)
+    assert 520 * 3 > 1024
+    check(orc, types, mask, img, vid)
+
+
+def test_grid_prefix_over_many_chunks(orc):
+    # more than 1024 image grids (their prefix sums are scanned 1024 at a time)
+    types, mask, img = _many_images_batch(np.random.default_rng(78), 8, 1800)
+    assert img.shape[0] > 2048
+    check(orc, types, mask, img, None)
+
+
 def test_masked_slot_inside_a_run(orc):
     # a dropped slot inside an image run does not split it
     types = [[0, 1, 1, 1, 0, 1, 1, 1, 0] + [0] * 1100]
