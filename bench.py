@@ -296,6 +296,7 @@ CASES = {
     "mrope_decode": "decode step, B = 256, Q [256, 24, 256], K / V [256, 4, 256] bf16, norm + KV-cache write",
     "mrope_cos_sin": "cos / sin tables of the large-prefill request (T = 131072, rot 64, interleaved)",
     "vis_pos_interp_batch8": "interpolation of the batch of 8 single images (bf16 table, N = 26528)",
+    "mrope_apply_prefill": "fused MRoPE of the large-prefill request (Q [131072, 24, 256], K [131072, 4, 256])",
     "mrope_apply_short": "fused MRoPE on the 4096-token prompt (text_t4096_qwen35: Q [4096, 24, 256], K [4096, 4, 256])",
     "qk_norm_mrope_short": "fused QK-RMSNorm + MRoPE on the 4096-token prompt (text_t4096_qwen35)",
     "fill_reference": "torch fill_ of the 67 MB the cos / sin kernel writes at T = 131072, rot 64 (a write-stream "
@@ -352,15 +353,15 @@ def run_case(args):
         out = torch.empty(wl.n_patches(v), v.hidden, dtype=torch.bfloat16, device=dev)
         fn = lambda: ipe.vis_pos_interp(table, v.grid_thw, v.merge, out=out, stream=stream)  # noqa: E731
         nbytes = algorithmic_bytes_vision(v)
-    elif name in ("mrope_apply_short", "qk_norm_mrope_short"):
-        w = wl.WORKLOADS["text_t4096_qwen35"]
+    elif name in ("mrope_apply_short", "qk_norm_mrope_short", "mrope_apply_prefill"):
+        w = wl.WORKLOADS["prefill_t131072_video" if name == "mrope_apply_prefill" else "text_t4096_qwen35"]
         t = w.text
         tin = wl.text_inputs(w)
         Q = torch.from_numpy(tin["q"].view(np.int16)).view(torch.bfloat16).to(dev)
         K = torch.from_numpy(tin["k"].view(np.int16)).view(torch.bfloat16).to(dev)
         pos = torch.from_numpy(tin["positions"]).to(dev)
         inv = ipe.rope_inv_freq(t.rot_dim, t.theta)
-        if name == "mrope_apply_short":
+        if name != "qk_norm_mrope_short":
             fn = lambda: ipe.mrope_apply(Q, K, pos, inv, t.section, True, stream=stream)  # noqa: E731
             nbytes = (t.hq + t.hk) * t.T * t.rot_dim * 2 * 2 + 3 * t.T * 4
         else:
