@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include <cuda.h>   // CUresult / CUdeviceptr types only; the driver call is resolved at run time
@@ -47,18 +48,16 @@ typedef CUresult (*AddressRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
 
 AddressRangeFn address_range_fn()
 {
-    static AddressRangeFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    // resolved once (thread-safe static initialisation)
+    static const AddressRangeFn fn = []() -> AddressRangeFn {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<AddressRangeFn>(p);
-        else
-            cudaGetLastError();
-    }
+            return reinterpret_cast<AddressRangeFn>(p);
+        cudaGetLastError();
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -108,18 +107,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
 
 EncodeTiledFn encode_tiled_fn()
 {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    // resolved once (thread-safe static initialisation)
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-        else
-            cudaGetLastError();
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        cudaGetLastError();
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -246,11 +243,13 @@ namespace ipe {
 unsigned *device_status_word()
 {
     static unsigned *addr[64] = {};
+    static std::mutex lock_addr;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
         return nullptr;
     }
+    std::lock_guard<std::mutex> guard(lock_addr);   // callers on several host threads
     if (!addr[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_ipe_status) != cudaSuccess) {
