@@ -299,6 +299,7 @@ CASES = {
     "mrope_apply_prefill": "fused MRoPE of the large-prefill request (Q [131072, 24, 256], K [131072, 4, 256])",
     "mrope_apply_short": "fused MRoPE on the 4096-token prompt (text_t4096_qwen35: Q [4096, 24, 256], K [4096, 4, 256])",
     "qk_norm_mrope_short": "fused QK-RMSNorm + MRoPE on the 4096-token prompt (text_t4096_qwen35)",
+    "vis_pos_interp_hf": "interpolation in HF rounding mode, 16 x 64 x 64 video of the large-prefill request",
     "fill_reference": "torch fill_ of the 67 MB the cos / sin kernel writes at T = 131072, rot 64 (a write-stream "
                       "reference for that kernel; not a library kernel)",
 }
@@ -346,6 +347,13 @@ def run_case(args):
         sin = torch.empty_like(cos)
         fn = lambda: ipe.mrope_cos_sin(pos, inv, t.section, True, cos, sin, stream=stream)  # noqa: E731
         nbytes = 3 * t.T * 4 + 2 * t.T * t.rot_dim * 4
+    elif name == "vis_pos_interp_hf":
+        w = wl.WORKLOADS[WORKLOAD]
+        v = w.vision
+        table = torch.from_numpy(wl.vision_inputs(w)["table"].view(np.int16)).view(torch.bfloat16).to(dev)
+        out = torch.empty(wl.n_patches(v), v.hidden, dtype=torch.bfloat16, device=dev)
+        fn = lambda: ipe.vis_pos_interp(table, v.grid_thw, v.merge, out=out, stream=stream, rounding="hf")  # noqa: E731
+        nbytes = algorithmic_bytes_vision(v)
     elif name == "vis_pos_interp_batch8":
         w = wl.WORKLOADS["vision_batch8_bf16"]
         v = w.vision
