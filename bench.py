@@ -299,6 +299,8 @@ CASES = {
     "mrope_apply_prefill": "fused MRoPE of the large-prefill request (Q [131072, 24, 256], K [131072, 4, 256])",
     "mrope_apply_short": "fused MRoPE on the 4096-token prompt (text_t4096_qwen35: Q [4096, 24, 256], K [4096, 4, 256])",
     "qk_norm_mrope_short": "fused QK-RMSNorm + MRoPE on the 4096-token prompt (text_t4096_qwen35)",
+    "vis_fused_batch8": "interpolation and vision rotary in one call on the batch of 8 single images (N = 26528)",
+    "vis_fused_prefill": "interpolation and vision rotary in one call on the 16 x 64 x 64 video of the large prefill",
     "vis_pos_interp_hf": "interpolation in HF rounding mode, 16 x 64 x 64 video of the large-prefill request",
     "fill_reference": "torch fill_ of the 67 MB the cos / sin kernel writes at T = 131072, rot 64 (a write-stream "
                       "reference for that kernel; not a library kernel)",
@@ -347,6 +349,16 @@ def run_case(args):
         sin = torch.empty_like(cos)
         fn = lambda: ipe.mrope_cos_sin(pos, inv, t.section, True, cos, sin, stream=stream)  # noqa: E731
         nbytes = 3 * t.T * 4 + 2 * t.T * t.rot_dim * 4
+    elif name in ("vis_fused_batch8", "vis_fused_prefill"):
+        w = wl.WORKLOADS["vision_batch8_bf16" if name == "vis_fused_batch8" else WORKLOAD]
+        v = w.vision
+        vin = wl.vision_inputs(w)
+        bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+        table, qv, kv = bf(vin["table"]), bf(vin["q"]), bf(vin["k"])
+        out = torch.empty(wl.n_patches(v), v.hidden, dtype=torch.bfloat16, device=dev)
+        fn = lambda: ipe.vis_pos_interp_rope2d(table, v.grid_thw, qv, kv, v.merge, v.theta, out=out,  # noqa: E731
+                                               stream=stream)
+        nbytes = algorithmic_bytes_vision(v) + 2 * wl.n_patches(v) * v.heads * v.head_dim * 2 * 2
     elif name == "vis_pos_interp_hf":
         w = wl.WORKLOADS[WORKLOAD]
         v = w.vision

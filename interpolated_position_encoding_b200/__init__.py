@@ -553,7 +553,8 @@ def vis_rope2d(q, k, grid_thw, merge=2, theta=1e4, stream=None):
 
 
 def vis_pos_interp_rope2d(table, grid_thw, q, k, merge=2, theta=1e4, out=None, stream=None):
-    """One launch: interpolated position embeddings (returned) and in-place 2-D rotary of q, k."""
+    """Interpolated position embeddings (returned) and in-place 2-D rotary of q, k in one call, the two
+    kernels running concurrently."""
     G, C = _table_args(table)
     g, n = _grid_host(grid_thw)
     N = sum(g[3 * i] * g[3 * i + 1] * g[3 * i + 2] for i in range(n))

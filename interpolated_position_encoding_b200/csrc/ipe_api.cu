@@ -819,6 +819,38 @@ int ipe_vis_rope2d(void *q, void *k, ipe_dtype dtype, int64_t n_patch, int heads
     return e == cudaSuccess ? ok() : cuda_fail(e, "vis_rope2d launch");
 }
 
+// A second stream per device for work that overlaps the caller's: created on
+// first use, with a ring of events (a wait refers to the record made before
+// it, so the ring may wrap).
+struct AuxStream {
+    bool ready = false;
+    cudaStream_t s = nullptr;
+    cudaEvent_t ring[64] = {};
+    unsigned next = 0;
+};
+
+static std::mutex g_aux_mutex;
+static AuxStream g_aux[64];
+
+static int aux_stream(AuxStream **out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(IPE_ELIMIT, "device index beyond 64");
+    AuxStream &a = g_aux[dev];
+    if (!a.ready) {
+        if ((e = cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamCreate");
+        for (cudaEvent_t &ev : a.ring)
+            if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess)
+                return cuda_fail(e, "cudaEventCreate");
+        a.ready = true;
+    }
+    *out = &a;
+    return IPE_OK;
+}
+
 int ipe_vis_pos_interp_rope2d(const void *table, int grid_side, int hidden, void *out, void *q, void *k, int heads,
                               int head_dim, int64_t q_stride, int64_t k_stride, double theta, ipe_dtype dtype,
                               const int32_t *grid_thw_host, int n_images, int merge, void *stream)
@@ -832,8 +864,24 @@ int ipe_vis_pos_interp_rope2d(const void *table, int grid_side, int hidden, void
     if (int rc = interp_args(table, dtype, grid_side, hidden, out, d, ia)) return rc;
     RotArgs r;
     if (int rc = vis_rot_args(q, k, dtype, d.n_patch, heads, head_dim, q_stride, k_stride, d, r)) return rc;
-    cudaError_t e = launch_vis_fused(dtype == IPE_BF16, d, ia, r, f, (cudaStream_t)stream);
-    return e == cudaSuccess ? ok() : cuda_fail(e, "vis_pos_interp_rope2d launch");
+    // The interpolation (issue-bound on single frames) runs on a second
+    // stream while the rotation (memory-bound) runs on `stream`: the two
+    // kernels' blocks share the SMs, and `stream` waits for both.
+    const cudaStream_t s = (cudaStream_t)stream;
+    std::lock_guard<std::mutex> lock(g_aux_mutex);
+    AuxStream *aux = nullptr;
+    if (int rc = aux_stream(&aux)) return rc;
+    cudaEvent_t fork = aux->ring[aux->next++ % 64], join = aux->ring[aux->next++ % 64];
+    cudaError_t e;
+    if ((e = cudaEventRecord(fork, s)) != cudaSuccess || (e = cudaStreamWaitEvent(aux->s, fork, 0)) != cudaSuccess)
+        return cuda_fail(e, "vis_pos_interp_rope2d fork");
+    if ((e = launch_vis_interp(dtype == IPE_BF16, d, ia, aux->s)) != cudaSuccess)
+        return cuda_fail(e, "vis_pos_interp_rope2d interpolation launch");
+    if ((e = cudaEventRecord(join, aux->s)) != cudaSuccess) return cuda_fail(e, "vis_pos_interp_rope2d join");
+    if ((e = launch_vis_rope(dtype == IPE_BF16, d, r, f, s)) != cudaSuccess)
+        return cuda_fail(e, "vis_pos_interp_rope2d rotation launch");
+    if ((e = cudaStreamWaitEvent(s, join, 0)) != cudaSuccess) return cuda_fail(e, "vis_pos_interp_rope2d join");
+    return ok();
 }
 
 }  // extern "C"

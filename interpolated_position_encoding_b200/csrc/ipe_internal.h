@@ -194,8 +194,6 @@ cudaError_t launch_vis_interp(bool bf16, const VisDesc<1024> &d, const InterpArg
 cudaError_t launch_vis_interp_hf(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, cudaStream_t s);
 cudaError_t launch_vis_rope(bool bf16, const VisDesc<1024> &d, const RotArgs &r,
                             const VisAngleFreqs &f, cudaStream_t s);
-cudaError_t launch_vis_fused(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, const RotArgs &r,
-                             const VisAngleFreqs &f, cudaStream_t s);
 
 // Widest vector (elements, <= 16 bytes) that divides half, head_dim and both
 // strides of `r` and that both base pointers are aligned to.

@@ -1,5 +1,5 @@
 // Vision-tower kernels: position-table interpolation in merge order, the 2-D
-// (row, col) rotary, their fused launch, and the plan read-back.
+// (row, col) rotary, and the plan read-back.
 //
 // "Qwen3-VL" notes (frankmowj.github.io), fast_pos_embed_interpolate,
 // rot_pos_emb, apply_rotary_pos_emb_vision; cortiq-engine qwen3vis.rs
@@ -242,25 +242,6 @@ static bool interp_wide(const InterpArgs &ia)
     return ia.hidden % E == 0 && (uintptr_t)ia.table % 16 == 0 && (uintptr_t)ia.out % 16 == 0;
 }
 
-// --------------------------------------------------------------- fused
-// One persistent launch: every block first takes interpolation work items
-// (strip x channel slice) in a grid-stride loop, using its shared memory as
-// the blend buffer, then runs the TMA rotary pipeline over its tiles of q, k.
-template <typename T, int VEC, int E, int M, int MAXIMG>
-__global__ void __launch_bounds__(kTmaThreads, 2) vis_fused_kernel(const __grid_constant__ VisTmaSrc<MAXIMG> src,
-                                                                const __grid_constant__ InterpArgs ia,
-                                                                const __grid_constant__ TmaRotArgs r)
-{
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char *R = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-    const int n_interp = src.d.n_strips * ia.n_slices;
-    for (int item = blockIdx.x; item < n_interp; item += gridDim.x) {
-        interp_block<T, E, M, MAXIMG>(src.d, ia, item / ia.n_slices, item % ia.n_slices, R);
-        __syncthreads();          // R is reused by the next item / the pipeline
-    }
-    rotary_tma_block<T, VEC, VisTmaSrc<MAXIMG>>(r, src, smem_raw, blockIdx.x, gridDim.x);
-}
-
 // ------------------------------------------------------------- launches
 template <int MAXIMG>
 static VisDesc<MAXIMG> shrink(const VisDesc<1024> &d)
@@ -334,61 +315,6 @@ cudaError_t launch_vis_rope(bool bf16, const VisDesc<1024> &d, const RotArgs &r,
     if (bf16)
         return d.n_images <= 16 ? rope_impl<__nv_bfloat16, 16>(d, r, f, s) : rope_impl<__nv_bfloat16, 1024>(d, r, f, s);
     return d.n_images <= 16 ? rope_impl<float, 16>(d, r, f, s) : rope_impl<float, 1024>(d, r, f, s);
-}
-
-template <typename T, int VEC, int MAXIMG>
-static cudaError_t fused_vec(const VisDesc<1024> &d, const InterpArgs &ia, TmaRotArgs t, const VisAngleFreqs &f,
-                             cudaStream_t s)
-{
-    tma_layout<T, VEC, VisTmaSrc<MAXIMG>>(t);
-    const size_t smem = std::max(interp_smem_bytes(sizeof(T) == 2, d.merge, d.grid_side) + 128,
-                                 tma_smem_bytes(t, false));
-    const bool wide = interp_wide<T>(ia), m2 = d.merge == 2;
-    auto kern = wide ? (m2 ? vis_fused_kernel<T, VEC, 16 / sizeof(T), 2, MAXIMG> : vis_fused_kernel<T, VEC, 16 / sizeof(T), 0, MAXIMG>)
-                     : (m2 ? vis_fused_kernel<T, VEC, 4, 2, MAXIMG> : vis_fused_kernel<T, VEC, 4, 0, MAXIMG>);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kTmaThreads, smem);
-    if (e != cudaSuccess) return e;
-    const long long ntiles = (t.rows + t.P - 1) / t.P;
-    const long long work = std::max(ntiles, (long long)d.n_strips * ia.n_slices);
-    const long long cap = (long long)sm_count() * std::max(per_sm, 1);
-    const int blocks = (int)std::max<long long>(1, std::min(work, cap));
-    VisTmaSrc<MAXIMG> src{shrink<MAXIMG>(d), f};
-    kern<<<blocks, kTmaThreads, smem, s>>>(src, ia, t);
-    return cudaGetLastError();
-}
-
-// The fused launch needs the TMA rotary path; shapes it cannot take run as
-// two launches (interpolation, then the vector-load rotary).
-template <typename T, int MAXIMG>
-static cudaError_t fused_impl(const VisDesc<1024> &d, const InterpArgs &ia, const RotArgs &r,
-                              const VisAngleFreqs &f, cudaStream_t s)
-{
-    TmaRotArgs t;
-    if (tma_rot_args(r, sizeof(T), t) && interp_smem_bytes(sizeof(T) == 2, d.merge, d.grid_side) + 128 <= 200 * 1024) {
-        t.aux_tma = 0;
-        const int v = pick_vec(r, sizeof(T));
-        if constexpr (sizeof(T) == 2) {
-            if (v == 8) return fused_vec<T, 8, MAXIMG>(d, ia, t, f, s);
-        }
-        if (v >= 4) return fused_vec<T, 4, MAXIMG>(d, ia, t, f, s);
-        return fused_vec<T, 2, MAXIMG>(d, ia, t, f, s);
-    }
-    cudaError_t e = interp_impl<T, MAXIMG>(d, ia, s);
-    if (e != cudaSuccess) return e;
-    VisSrc<MAXIMG> src{shrink<MAXIMG>(d), f};
-    return dispatch_vec<T>(r, src, s);
-}
-
-cudaError_t launch_vis_fused(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, const RotArgs &r,
-                             const VisAngleFreqs &f, cudaStream_t s)
-{
-    if (bf16)
-        return d.n_images <= 16 ? fused_impl<__nv_bfloat16, 16>(d, ia, r, f, s)
-                                : fused_impl<__nv_bfloat16, 1024>(d, ia, r, f, s);
-    return d.n_images <= 16 ? fused_impl<float, 16>(d, ia, r, f, s) : fused_impl<float, 1024>(d, ia, r, f, s);
 }
 
 }  // namespace ipe
