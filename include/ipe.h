@@ -32,6 +32,10 @@
  * - Element counts and strides are in elements, not bytes.
  * - Floating-point arithmetic is fp32; bf16 results are rounded once (to
  *   nearest even) at the end.  sin / cos are CUDA's accurate sincosf.
+ * - CUDA graphs: the device entry points can be captured into a graph and
+ *   replayed.  Make one call of each before the capture: a first call may
+ *   create the library's per-device stream and events and look up driver
+ *   entry points, which must not happen inside a capture.
  *
  * Pages cited (title -- section):
  *   [QVL]  "Qwen3-VL" notes, frankmowj.github.io
