@@ -208,6 +208,23 @@ def pin_rms_norm_closed_forms(o):
     assert not (yb.view(np.uint32) & 0xFFFF).any()
 
 
+def pin_rms_norm_matches_torch_literal(o):
+    # The drill's steps evaluated by torch on the CPU in bf16: x.float(),
+    # rsqrt(mean(x^2) + eps), .to(bf16), then * weight (a bf16 product).
+    # The oracle (double, then the two roundings) agrees with it except at
+    # rare fp32-vs-double ties; multiplying by the weight before the cast
+    # agrees on only about three quarters of the elements.
+    import torch
+    rng = _rng(41)
+    x = torch.from_numpy(rng.standard_normal((192, 128)).astype(np.float32)).to(torch.bfloat16)
+    w = torch.from_numpy((1 + 0.3 * rng.standard_normal(128)).astype(np.float32)).to(torch.bfloat16)
+    x32 = x.float()
+    xn = x32 * torch.rsqrt(x32.pow(2).mean(-1, keepdim=True) + 1e-6)
+    want = (xn.to(torch.bfloat16) * w).float().numpy().astype(np.float64)
+    got = o.rms_norm(x.float().numpy().astype(np.float64), w.float().numpy().astype(np.float64), 1e-6, "bf16")
+    assert (got == want).mean() >= 0.999
+
+
 # ------------------------------------------------------------------- vision
 
 

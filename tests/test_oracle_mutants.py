@@ -56,6 +56,8 @@ MUTANTS = {
     "vision_inv_dim": ("orc_rope_inv_freq(dim, theta, inv);", "orc_rope_inv_freq(dim, sqrt(theta), inv);"),
     # RMSNorm: eps added after the square root
     "rms_eps_outside": ("double inv = 1.0 / sqrt(ss / D + eps);", "double inv = 1.0 / (sqrt(ss / D) + eps);"),
+    # RMSNorm: the weight applied before the cast back to the dtype
+    "rms_weight_before_cast": ("double xn = round_to(xr[d] * inv, dtype);", "double xn = xr[d] * inv;"),
     # RMSNorm: sum of squares instead of the mean
     "rms_sum_not_mean": ("double inv = 1.0 / sqrt(ss / D + eps);", "double inv = 1.0 / sqrt(ss + eps);"),
     # position table: a vision run advances by its slot count instead of its longer side
