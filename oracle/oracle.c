@@ -28,9 +28,10 @@
  *          rope_angles(), attention()
  *
  * Parity status: every function here is pinned by the not-gpu tests (worked
- * values printed on the pages, closed forms, invariants, brute force), except
- * that the vision 2-D rotary has no printed numeric example; it is pinned by
- * invariants and a basis-vector read-back only.
+ * values printed on the pages, closed forms, invariants, brute force).  The
+ * vision 2-D rotary has no printed numeric example; it is pinned by
+ * invariants, a basis-vector read-back, and the pages' rot_pos_emb /
+ * apply_rotary_pos_emb_vision steps evaluated by torch in fp32.
  *
  * Return convention: 0 on success, -1 on an argument the definition does not
  * cover.

@@ -343,6 +343,43 @@ def pin_vision_angles_basis(o):
         assert not others.any()
 
 
+def _torch_listing_vision_rotary(q, grids, m, theta):
+    """rot_pos_emb and apply_rotary_pos_emb_vision of the "Qwen3-VL" notes,
+    evaluated by torch in fp32 on the CPU: (row, col) ids per token in merge
+    order, an fp32 frequency table looked up and flattened to [rows | cols],
+    duplicated to the head width, and q cos + rotate_half(q) sin."""
+    import torch
+    head_dim = q.shape[-1]
+    dim = head_dim // 2
+    inv = 1.0 / (theta ** (torch.arange(0, dim, 2, dtype=torch.float) / dim))
+    max_hw = max(max(h, w) for _, h, w in grids)
+    table = torch.outer(torch.arange(max_hw, dtype=torch.float), inv)
+    ids = []
+    for t, h, w in grids:
+        br = torch.arange(h // m)[:, None, None, None] * m + torch.arange(m)[None, None, :, None]
+        bc = torch.arange(w // m)[None, :, None, None] * m + torch.arange(m)[None, None, None, :]
+        rows = br.expand(h // m, w // m, m, m).reshape(-1)
+        cols = bc.expand(h // m, w // m, m, m).reshape(-1)
+        ids.append(torch.stack([rows, cols], -1).repeat(t, 1))
+    emb = table[torch.cat(ids)].flatten(1)
+    emb = torch.cat([emb, emb], -1)
+    cos, sin = emb.cos()[:, None, :], emb.sin()[:, None, :]
+    x = torch.from_numpy(q).float()
+    rh = torch.cat([-x[..., head_dim // 2:], x[..., :head_dim // 2]], -1)
+    return (x * cos + rh * sin).double().numpy()
+
+
+def pin_vision_rotary_matches_torch_listing(o):
+    # fp32 (torch) against double (oracle): agreement to fp32 rounding
+    rng = _rng(43)
+    grids = [(1, 4, 6), (2, 6, 4), (1, 8, 8)]
+    N = sum(t * h * w for t, h, w in grids)
+    q = rng.standard_normal((N, 3, 72)).astype(np.float32)
+    want = _torch_listing_vision_rotary(q, grids, 2, 1e4)
+    got = o.vis_apply_rotary(q.astype(np.float64), grids, 2, 1e4)
+    assert np.abs(got - want).max() <= 2e-5, np.abs(got - want).max()
+
+
 def pin_vision_rotation_complex(o):
     # Whole-head split-half rotation = complex multiply of x_j + i x_(j+36)
     # by exp(i a_j); norm of every pair preserved.
