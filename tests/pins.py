@@ -592,6 +592,19 @@ def pin_interp_hf_matches_torch_listing(o):
             assert got.shape == want.shape and (got == want).all(), (dt, grids)
 
 
+def pin_interp_matches_torch_listing(o):
+    # The default interpolation (exact sample points, double) against the
+    # listing run by torch in float64 with its fp32 linspace: they differ only
+    # by the rounding of the sample points (a few 1e-7 of a table value).
+    import torch
+    rng = _rng(47)
+    table = rng.standard_normal((48 * 48, 12))
+    for grids, m in [([(1, 4, 6), (2, 10, 14), (1, 48, 64)], 2), ([(1, 5, 7), (3, 1, 9)], 1)]:
+        want = _torch_listing_interp(torch.from_numpy(table), grids, m).numpy()
+        got = o.vis_pos_embed_interpolate(table, grids, m)
+        assert np.abs(got - want).max() <= 2e-5 * np.abs(table).max(), np.abs(got - want).max()
+
+
 def pin_rotary_hf_matches_torch(o):
     import torch
     rng = _rng(31)
