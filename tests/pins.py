@@ -639,4 +639,53 @@ def pin_hf_rounding_close_to_exact(o):
     assert np.abs(hf - exact).max() <= 1e-5 * (1 + np.abs(exact).max())
 
 
+def _torch_listing_mrope_freqs(pos, inv):
+    """The text rotary's angle table as the pages' forward() builds it: the
+    shared inv_freq against each axis's positions, both as fp32, by a
+    one-column matmul, then transposed to [3, B, L, half]."""
+    import torch
+    p = torch.from_numpy(pos)[:, None, :]                      # [3, B=1, L]
+    inv_e = torch.from_numpy(inv)[None, None, :, None].float().expand(3, 1, -1, 1)
+    return (inv_e @ p[:, :, None, :].float()).transpose(2, 3)   # [3, 1, L, half]
+
+
+def _torch_listing_interleave(f, sec):
+    """Axis T everywhere, then H on frequencies 1, 4, 7, ... and W on 2, 5,
+    8, ..., each up to 3 x its section, then the halves duplicated."""
+    import torch
+    ft = f[0].clone()
+    for axis, offset in ((1, 1), (2, 2)):
+        sl = slice(offset, sec[axis] * 3, 3)
+        ft[..., sl] = f[axis][..., sl]
+    return torch.cat((ft, ft), dim=-1)
+
+
+def pin_mrope_cos_sin_matches_torch_listings(o):
+    # The interleaved text cos / sin against the two forms the pages print,
+    # run by torch in fp32: selection of the angles before the cos
+    # ("Qwen3-VL" notes, Qwen3VLTextRotaryEmbedding.forward and
+    # apply_interleaved_mrope) and selection of the cos / sin tables after it
+    # ("Interleaved Rotary Position Embedding", Qwen3_5TextRotaryEmbedding and
+    # recomposition_frequencies).  The angles must agree exactly (the cos of
+    # torch's fp32 angles in double equals the oracle's), the fp32 cos / sin
+    # within their own rounding.
+    rng = _rng(53)
+    for half, sec, theta in [(64, (24, 20, 20), 5e6), (32, (11, 11, 10), 1e7), (10, (4, 3, 3), 1e4)]:
+        L = 40
+        pos = rng.integers(0, 300000, (3, L)).astype(np.int64)
+        pos[:, 0] = (1 << 24) + 1                  # rounded by the fp32 conversion
+        pos[:, 1] = [7, 7, 7]
+        inv = o.rope_inv_freq(2 * half, theta)
+        cos, sin = o.mrope_cos_sin(pos, inv, sec, True)
+        f = _torch_listing_mrope_freqs(pos, inv)
+        emb = _torch_listing_interleave(f, sec)[0]               # [L, 2 half]
+        e64 = emb.double().numpy()
+        assert np.abs(np.cos(e64) - cos).max() <= 4e-16 and np.abs(np.sin(e64) - sin).max() <= 4e-16
+        c1, s1 = emb.cos().numpy(), emb.sin().numpy()
+        c2 = _torch_listing_interleave(f.cos(), sec)[0].numpy()
+        s2 = _torch_listing_interleave(f.sin(), sec)[0].numpy()
+        for c, s in ((c1, s1), (c2, s2)):
+            assert np.abs(c - cos).max() <= 1.2e-7 and np.abs(s - sin).max() <= 1.2e-7, (half, sec)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

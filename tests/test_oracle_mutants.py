@@ -89,6 +89,8 @@ MUTANTS = {
     # HF rotation: the product x cos not rounded
     "hf_product_unrounded": ("const double a = round_to(xr[j] * c, dtype);", "const double a = xr[j] * c;"),
     # position table: image temporal index dropped
+    "angle_product_double": ("freqs[a * plane + t * half + i] = (double)f32_mul(p, inv_freq[i]);",
+                             "freqs[a * plane + t * half + i] = (double)p * (double)inv_freq[i];"),
     "rope_image_time": ("table[0 * n + cols] = tt * 1 + cur;", "table[0 * n + cols] = cur;"),
 }
 
