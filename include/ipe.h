@@ -370,7 +370,8 @@ int ipe_vis_interp_plan(const int32_t *grid_thw_host, int n_images, int merge, i
  * (1-dx)((1-dy) T[y0,x0] + dy T[y1,x0]) + dx((1-dy) T[y0,x1] + dy T[y1,x1]),
  * equal to the four-weight sum in exact arithmetic, rounded once.
  *   table      device [G*G, hidden], dtype (row id = y G + x)
- *   hidden     channels, multiple of 4 (1152 in Qwen3-VL)
+ *   hidden     channels, multiple of 4 (1152 in Qwen3-VL); at most
+ *              65535 x 128 bytes (IPE_ELIMIT above)
  *   out        device [N, hidden], dtype, written; N = sum t h w.
  * ------------------------------------------------------------------------- */
 int ipe_vis_pos_interp(const void *table, ipe_dtype dtype, int grid_side, int hidden,

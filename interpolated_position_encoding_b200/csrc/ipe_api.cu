@@ -750,7 +750,8 @@ static int interp_args(const void *table, ipe_dtype dtype, int grid_side, int hi
     ia.out = out;
     ia.hidden = hidden;
     ia.n_slices = (hidden + cs - 1) / cs;
-    if ((long long)d.n_strips * ia.n_slices > (1LL << 31) - 1) return fail(IPE_ELIMIT, "grid too large");
+    if (ia.n_slices > 65535)   // slices are the second grid dimension
+        return fail(IPE_ELIMIT, "hidden %d exceeds %d channels", hidden, 65535 * cs);
     return IPE_OK;
 }
 

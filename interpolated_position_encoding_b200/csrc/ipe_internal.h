@@ -199,7 +199,8 @@ cudaError_t launch_vis_rope(bool bf16, const VisDesc<1024> &d, const RotArgs &r,
 // strides of `r` and that both base pointers are aligned to.
 int pick_vec(const RotArgs &r, int elem_bytes);
 
-// Shared-memory bytes of one interpolation block (host check of the limit).
-size_t interp_smem_bytes(bool bf16, int merge, int grid_side);
+// Shared-memory bytes of one interpolation block covering `slices` 128-byte
+// channel slices (the host checks the limit at one slice).
+size_t interp_smem_bytes(bool bf16, int merge, int grid_side, int slices = 1);
 
 }  // namespace ipe
