@@ -50,15 +50,6 @@ template <> __device__ __forceinline__ void pairs_to_chunk<float>(const float2 *
     }
 }
 
-// Product of two bf16 pairs rounded once to bf16 (the exact product of two
-// bf16 values fits in fp32, so this equals rounding the fp32 product).
-__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b)
-{
-    uint32_t d;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
 // RMSNorm of the row whose chunk x this lane holds: y = dtype(dtype(x r) * w)
 // with r = rsqrt(mean(x^2) + eps) in fp32 (inv_d = 1 / D, exact: D is a power
 // of two).  Every lane of the warp must call it (shuffles over LPR lanes).

@@ -22,6 +22,26 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(v);
 }
 
+// Packed bf16 arithmetic with one rounding per result.  For bf16 operands
+// these equal the fp32 operation followed by rounding to bf16:
+//   * the exact product of two bf16 values (8-bit significands) fits in fp32;
+//   * an fp32 sum of two bf16 values is inexact only when their exponents
+//     differ by 16 or more.  The sum then lies within 2^(e-15) of the larger
+//     operand a (exponent e), while the nearest bf16 rounding midpoints are
+//     at least 2^(e-9) from a, so both roundings give a.
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 // v rounded to the dtype T and back to fp32 (round to nearest even; exact for fp32).
 template <typename T> __device__ __forceinline__ float round_to_dtype(float v) { return to_f32(from_f32<T>(v)); }
 

@@ -18,7 +18,9 @@
 // fp32 with one rounding; this one evaluates the four-corner sum directly:
 // a block takes one merge-row strip of frame 0 and 32 chunks of 16 bytes of
 // the channels, each warp one output row at a time, and each result chunk
-// is written once per frame.
+// is written once per frame.  For bf16 the products and sums run as packed
+// bf16x2 operations, which round exactly where the fp32-then-round steps
+// above do (mul_bf16x2 / add_bf16x2).
 #include "ipe_internal.h"
 #include "ipe_device.cuh"
 
@@ -65,20 +67,45 @@ __global__ void __launch_bounds__(32 * kHfWarps) vis_interp_hf_kernel(const __gr
         const long long idx[4] = {(long long)y0 * G + x0, (long long)y0 * G + x1, (long long)y1 * G + x0,
                                   (long long)y1 * G + x1};
         if (ch >= chunks) continue;
-        Pack<T, EC> c[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) c[k] = ld_pack<T, EC>(table + idx[k] * ia.hidden + (long long)ch * EC);
-        Pack<T, EC> o;
-#pragma unroll
-        for (int e = 0; e < EC; ++e) {
-            float acc = round_to_dtype<T>(__fmul_rn(to_f32(c[0].v[e]), wt[0]));
-#pragma unroll
-            for (int k = 1; k < 4; ++k)
-                acc = round_to_dtype<T>(__fadd_rn(acc, round_to_dtype<T>(__fmul_rn(to_f32(c[k].v[e]), wt[k]))));
-            o.v[e] = from_f32<T>(acc);
-        }
         const long long row = im.row0 + (long long)sl * m * w + q;
-        for (int f = 0; f < im.t; ++f) st_pack<T, EC>(out + (row + f * hw) * ia.hidden + (long long)ch * EC, o);
+        if constexpr (sizeof(T) == 2) {
+            // eight bf16 channels as four bf16x2 words; weights broadcast to both halves
+            Pack<uint32_t, 4> c[4], o;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                c[k] = ld_pack<uint32_t, 4>(reinterpret_cast<const uint32_t *>(table + idx[k] * ia.hidden) + ch * 4);
+            uint32_t w2[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const __nv_bfloat162 b = __floats2bfloat162_rn(wt[k], wt[k]);   // exact: wt[k] is a bf16 value
+                w2[k] = *reinterpret_cast<const uint32_t *>(&b);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t acc = mul_bf16x2(c[0].v[i], w2[0]);
+#pragma unroll
+                for (int k = 1; k < 4; ++k) acc = add_bf16x2(acc, mul_bf16x2(c[k].v[i], w2[k]));
+                o.v[i] = acc;
+            }
+#pragma unroll 1
+            for (int f = 0; f < im.t; ++f)
+                st_pack<uint32_t, 4>(reinterpret_cast<uint32_t *>(out + (row + f * hw) * ia.hidden) + ch * 4, o);
+        } else {
+            Pack<T, EC> c[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) c[k] = ld_pack<T, EC>(table + idx[k] * ia.hidden + (long long)ch * EC);
+            Pack<T, EC> o;
+#pragma unroll
+            for (int e = 0; e < EC; ++e) {
+                float acc = round_to_dtype<T>(__fmul_rn(to_f32(c[0].v[e]), wt[0]));
+#pragma unroll
+                for (int k = 1; k < 4; ++k)
+                    acc = round_to_dtype<T>(__fadd_rn(acc, round_to_dtype<T>(__fmul_rn(to_f32(c[k].v[e]), wt[k]))));
+                o.v[e] = from_f32<T>(acc);
+            }
+#pragma unroll 1
+            for (int f = 0; f < im.t; ++f) st_pack<T, EC>(out + (row + f * hw) * ia.hidden + (long long)ch * EC, o);
+        }
     }
 }
 
