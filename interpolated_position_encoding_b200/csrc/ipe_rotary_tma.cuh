@@ -243,6 +243,33 @@ __device__ __forceinline__ void rotate_chunk(T *p, int half, int u, bool swap, c
     const float *S1 = (swap ? (HI ? cs.sh : cs.s) : cs.ns) + o;
     const float *S2 = (swap ? cs.ns : (HI ? cs.sh : cs.s)) + o;
     float2 v1[VEC / 2], v2[VEC / 2], c1[VEC / 2], c2[VEC / 2], s1[VEC / 2], s2[VEC / 2], w1[VEC / 2], w2[VEC / 2];
+    if constexpr (HF && sizeof(T) == 2) {
+        // bf16 HF: every product and the sum as one packed bf16x2 operation
+        // each, rounding where the fp32-then-cast steps do (mul_bf16x2 /
+        // add_bf16x2); cos / sin already hold bf16 values, so packing them is
+        // exact.
+        using W = Pack<uint32_t, VEC / 2>;
+        load_coef<VEC>(C1, c1);
+        load_coef<VEC>(S1, s1);
+        load_coef<VEC>(S2, s2);
+        if constexpr (HI) load_coef<VEC>(C2, c2);
+        const W r1 = ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(p1));
+        const W r2 = ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(p2));
+        W o1, o2;
+        auto bf2 = [](float2 f) {
+            const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+            return *reinterpret_cast<const uint32_t *>(&b);
+        };
+#pragma unroll
+        for (int i = 0; i < VEC / 2; ++i) {
+            const uint32_t C1w = bf2(c1[i]), S1w = bf2(s1[i]), C2w = HI ? bf2(c2[i]) : C1w, S2w = bf2(s2[i]);
+            o1.v[i] = add_bf16x2(mul_bf16x2(r1.v[i], C1w), mul_bf16x2(r2.v[i], S1w));
+            o2.v[i] = add_bf16x2(mul_bf16x2(r2.v[i], C2w), mul_bf16x2(r1.v[i], S2w));
+        }
+        st_pack<uint32_t, VEC / 2>(reinterpret_cast<uint32_t *>(p1), o1);
+        st_pack<uint32_t, VEC / 2>(reinterpret_cast<uint32_t *>(p2), o2);
+        return;
+    }
     load_pairs<T, VEC>(p1, v1);
     load_pairs<T, VEC>(p2, v2);
     load_coef<VEC>(C1, c1);
