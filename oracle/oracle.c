@@ -31,7 +31,10 @@
  * values printed on the pages, closed forms, invariants, brute force).  The
  * vision 2-D rotary has no printed numeric example; it is pinned by
  * invariants, a basis-vector read-back, and the pages' rot_pos_emb /
- * apply_rotary_pos_emb_vision steps evaluated by torch in fp32.
+ * apply_rotary_pos_emb_vision steps evaluated by torch in fp32.  The text
+ * cos / sin are also pinned to both printed forms of the interleaved
+ * selection ([QVL] apply_interleaved_mrope before the cos, [IRPE]
+ * recomposition_frequencies after it) evaluated by torch in fp32.
  *
  * Return convention: 0 on success, -1 on an argument the definition does not
  * cover.
