@@ -168,3 +168,120 @@ def test_error_message_is_thread_local_and_cleared():
     assert b"even" in L.ipe_last_error()
     assert L.ipe_rope_inv_freq(8, 1e4, out) == ipe.IPE_OK
     assert L.ipe_last_error() == b""
+
+
+# ------------------------------------------------ entry points around the path
+def test_rope_index_workspace_sizes():
+    ws = L.ipe_mrope_rope_index_workspace
+    assert ws(-1, 16, 0, 0) == 0 and ws(1, -1, 0, 0) == 0
+    assert ws(1, (1 << 30) + 1, 0, 0) == 0                # L above 2^30
+    assert ws(1 << 20, 1 << 12, 0, 0) == 0                # B * L above 2^31 - 1
+    assert ws(1, 16, 16385, 0) == 0 and ws(1, 16, 0, -1) == 0
+    small, large = ws(2, 4096, 3, 1), ws(2, 65536, 3, 1)
+    assert 0 < small < large
+
+
+def _ri(id_bytes=4, B=1, Lx=16, n_img=0, n_vid=0, grid_bytes=4, merge=2, types=FAKE, ws_bytes=1 << 20):
+    return L.ipe_mrope_rope_index(types, None, id_bytes, B, Lx, FAKE if n_img else None, n_img,
+                                  FAKE if n_vid else None, n_vid, grid_bytes, merge, FAKE, FAKE, FAKE, ws_bytes, None)
+
+
+def test_rope_index_rejects():
+    _err(_ri(id_bytes=2), ipe.IPE_EINVAL)
+    _err(_ri(grid_bytes=3), ipe.IPE_EINVAL)
+    _err(_ri(merge=0), ipe.IPE_EINVAL)
+    _err(_ri(merge=65), ipe.IPE_EINVAL)
+    _err(_ri(B=-1), ipe.IPE_EINVAL)
+    _err(_ri(Lx=(1 << 30) + 1), ipe.IPE_ELIMIT)
+    _err(_ri(n_img=16385), ipe.IPE_ELIMIT)
+    need = L.ipe_mrope_rope_index_workspace(1, 16, 0, 0)
+    _err(_ri(ws_bytes=need - 1), ipe.IPE_EINVAL)
+    _err(_ri(types=ctypes.c_void_p(0x1002)), ipe.IPE_EALIGN)      # int32 ids on a 2-byte boundary
+    assert _ri(B=0) == ipe.IPE_OK                                 # nothing to do, no device access
+
+
+def _dec(head_dim=128, rot=64, invf=None, qw=FAKE, kw=FAKE, eps=1e-6, k_cache=FAKE, v_cache=FAKE, v=FAKE,
+         cache_stride=256, num_slots=100, slots=FAKE, q=FAKE, B=4, hk=2):
+    invf = inv(rot // 2) if invf is None else invf
+    return L.ipe_mrope_decode(q, FAKE, v, ipe.IPE_BF16, B, 8, hk, head_dim, 8 * head_dim, hk * head_dim,
+                              hk * head_dim, FAKE, None, qw, kw, eps, invf, rot, k_cache, v_cache, cache_stride,
+                              num_slots, slots, None)
+
+
+def test_decode_rejects():
+    _err(_dec(head_dim=100), ipe.IPE_EINVAL)                      # not a multiple of 8 bf16
+    _err(_dec(head_dim=8, rot=8), ipe.IPE_ELIMIT)                 # one chunk per row
+    _err(_dec(rot=63), ipe.IPE_EINVAL)
+    _err(_dec(rot=8), ipe.IPE_EINVAL)                             # rot / 2 not a multiple of 8
+    bad = inv(32)
+    bad[5] = float("inf")
+    _err(_dec(invf=bad), ipe.IPE_EINVAL)
+    _err(_dec(kw=None), ipe.IPE_EINVAL)                           # one norm weight only
+    _err(_dec(eps=-1.0), ipe.IPE_EINVAL)
+    _err(_dec(slots=None), ipe.IPE_EINVAL)                        # caches without slot_mapping
+    _err(_dec(k_cache=None), ipe.IPE_EINVAL)                      # slot_mapping without k_cache
+    _err(_dec(v=None), ipe.IPE_EINVAL)                            # v_cache without v
+    _err(_dec(cache_stride=255), ipe.IPE_EINVAL)
+    _err(_dec(num_slots=-1), ipe.IPE_EINVAL)
+    _err(_dec(B=0, q=ctypes.c_void_p(0x1008)), ipe.IPE_EALIGN)    # q not 16-byte aligned
+    assert _dec(B=0) == ipe.IPE_OK
+    # no norm and no cache: weights, caches and slot_mapping all NULL
+    assert _dec(B=0, qw=None, kw=None, k_cache=None, v_cache=None, slots=None) == ipe.IPE_OK
+
+
+def _qkn(head_dim=128, rot=64, eps=1e-6, s=(11, 11, 10), qw=FAKE, T=16, q=FAKE):
+    return L.ipe_qk_norm_mrope(q, FAKE, ipe.IPE_BF16, T, 8, 2, head_dim, 8 * head_dim, 2 * head_dim, qw, FAKE,
+                               eps, FAKE, inv(rot // 2), rot, sec(*s), 1, None)
+
+
+def test_qk_norm_rejects():
+    _err(_qkn(head_dim=100), ipe.IPE_EINVAL)
+    _err(_qkn(head_dim=8, rot=8, s=(4, 0, 0)), ipe.IPE_ELIMIT)    # one chunk per row
+    _err(_qkn(head_dim=512, rot=64), ipe.IPE_ELIMIT)              # 64 chunks per row
+    _err(_qkn(rot=63, s=(11, 11, 9)), ipe.IPE_EINVAL)
+    _err(_qkn(rot=8, s=(2, 1, 1)), ipe.IPE_EINVAL)                # rot / 2 not a multiple of 8
+    _err(_qkn(eps=float("nan")), ipe.IPE_EINVAL)
+    _err(_qkn(eps=-1e-6), ipe.IPE_EINVAL)
+    _err(_qkn(s=(11, 11, 9)), ipe.IPE_EINVAL)                     # section does not sum to rot / 2
+    _err(_qkn(T=0, qw=ctypes.c_void_p(0x1004)), ipe.IPE_EALIGN)
+    _err(_qkn(T=0, q=ctypes.c_void_p(0x1008)), ipe.IPE_EALIGN)
+    assert _qkn(T=0) == ipe.IPE_OK
+
+
+def test_hf_entry_points_reject():
+    g, n = grid((1, 16, 16))
+    _err(L.ipe_vis_pos_interp_hf(FAKE, ipe.IPE_BF16, 48, 1148, g, n, 2, FAKE, None), ipe.IPE_EINVAL)  # hidden % 8
+    _err(L.ipe_vis_pos_interp_hf(ctypes.c_void_p(0x1008), ipe.IPE_BF16, 48, 1152, g, n, 2, FAKE, None),
+         ipe.IPE_EALIGN)
+    _err(L.ipe_vis_pos_interp_hf(FAKE, 9, 48, 1152, g, n, 2, FAKE, None), ipe.IPE_EINVAL)
+    g0, n0 = grid((1, 15, 16))
+    _err(L.ipe_vis_pos_interp_hf(FAKE, ipe.IPE_BF16, 48, 1152, g0, n0, 2, FAKE, None), ipe.IPE_EINVAL)
+    _err(L.ipe_mrope_apply_hf(FAKE, FAKE, ipe.IPE_BF16, 16, 24, 4, 256, 6144, 1024, FAKE, inv(32), 64,
+                              sec(11, 10, 10), 1, None), ipe.IPE_EINVAL)
+    _err(L.ipe_apply_rotary_partial_hf(FAKE, FAKE, ipe.IPE_BF16, 8, 2, 2, 16, 32, 32, FAKE, FAKE, 5, None),
+         ipe.IPE_EINVAL)
+
+
+def test_host_entry_points_reject():
+    # ipe_mrope_apply_host: chunk size, sizes, missing buffers
+    def mah(chunk=4096, T=16, qh=FAKE, pos=FAKE):
+        return L.ipe_mrope_apply_host(qh, FAKE, qh, FAKE, ipe.IPE_BF16, T, 24, 4, 256, pos, inv(32), 64,
+                                      sec(11, 11, 10), 1, FAKE, FAKE, FAKE, chunk, 1, None)
+    _err(mah(chunk=0), ipe.IPE_EINVAL)
+    _err(mah(T=-1), ipe.IPE_EINVAL)
+    _err(mah(qh=None), ipe.IPE_EINVAL)
+    _err(mah(pos=None), ipe.IPE_EINVAL)
+    g, n = grid((1, 16, 16))
+    gz, nz = grid((1, 0, 16))
+    _err(L.ipe_vis_rope2d_host(FAKE, FAKE, FAKE, FAKE, ipe.IPE_BF16, 16, 72, g, n, 2, 1e4, FAKE, FAKE, 0, 1, None),
+         ipe.IPE_EINVAL)
+    _err(L.ipe_vis_rope2d_host(FAKE, FAKE, FAKE, FAKE, ipe.IPE_BF16, 16, 72, gz, nz, 2, 1e4, FAKE, FAKE, 64, 1,
+                               None), ipe.IPE_EINVAL)
+    _err(L.ipe_vis_rope2d_host(None, FAKE, FAKE, FAKE, ipe.IPE_BF16, 16, 72, g, n, 2, 1e4, FAKE, FAKE, 64, 1, None),
+         ipe.IPE_EINVAL)
+    _err(L.ipe_vis_pos_interp_host(FAKE, ipe.IPE_BF16, 48, 1152, g, n, 2, FAKE, FAKE, FAKE, 0, 1, None),
+         ipe.IPE_EINVAL)
+    _err(L.ipe_vis_pos_interp_host(FAKE, ipe.IPE_BF16, 48, 1152, gz, nz, 2, FAKE, FAKE, FAKE, 64, 1, None),
+         ipe.IPE_EINVAL)
+    _err(L.ipe_vis_pos_interp_host(FAKE, ipe.IPE_BF16, 48, 1152, g, n, 2, FAKE, None, FAKE, 64, 1, None),
+         ipe.IPE_EINVAL)
