@@ -5,7 +5,7 @@
  *
  *   vision tower   vis_pos_interp      bilinear 48x48 position table -> patch grid, 2x2 merge order
  *                  vis_rope2d          2-D (row, col) rotary over the whole head
- *                  vis_pos_interp_rope2d  both in one launch
+ *                  vis_pos_interp_rope2d  both in one call (two kernels, concurrent)
  *   language model rope_inv_freq       default RoPE inverse frequencies (host)
  *                  mrope_axis_map      per-frequency T/H/W axis (interleaved or chunked)
  *                  mrope_cos_sin       multimodal cos / sin tables
