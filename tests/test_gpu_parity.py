@@ -260,7 +260,7 @@ def test_interp_workload(name, orc):
     ([(1, 8, 12)], 2, 4, 36), ([(2, 4, 6), (1, 2, 2), (3, 6, 4)], 2, 48, 1000), ([(1, 2, 4)] * 20, 2, 48, 132),
     ([(1, 96, 2)], 2, 48, 1152),
     # enough strips for two channel slices per block, with a ragged last group
-    ([(1, 24, 4)] * 100, 2, 48, 1000), ([(1, 12, 4)] * 400, 2, 48, 100)])
+    ([(1, 24, 4)] * 100, 2, 48, 1000), ([(1, 12, 4)] * 400, 2, 48, 100), ([(1, 8, 4)] * 300, 1, 48, 1152)])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_interp_edges(grids, merge, G, C, dtype, orc):
     rng = GEN(G * 7 + C)
