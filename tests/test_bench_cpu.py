@@ -29,3 +29,32 @@ def test_reference_arm_other_ranks_exit_quietly():
     p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
                         "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=ROOT, env=env)
     assert p.returncode == 0 and not [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_traffic_is_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
+    # roofline.traffic comes from profiles/dram_traffic.json only while the
+    # kernel sources hash to the value recorded with the capture
+    sys.path.insert(0, ROOT)
+    import bench
+    (tmp_path / "profiles").mkdir()
+    entry = {"bytes_per_launch": 123456, "source_sha": "aaaa"}
+    (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps({bench.WORKLOAD: {"mrope_apply": entry}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "aaaa")
+    assert bench.dram_traffic("mrope_apply") == 123456
+    assert bench.dram_traffic("vis_rope2d") is None
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "bbbb")
+    assert bench.dram_traffic("mrope_apply") is None
+
+
+def test_kernel_source_hash_covers_every_kernel_file(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    csrc = tmp_path / "interpolated_position_encoding_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "a.cu").write_text("one")
+    (csrc / "b.cuh").write_text("two")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_sha()
+    (csrc / "b.cuh").write_text("two!")
+    assert bench.kernel_source_sha() != h0
