@@ -100,6 +100,12 @@ def _cuda(t, name):
     return t
 
 
+def _cuda_device(device):
+    if torch.device(device).type != "cuda":
+        raise TypeError(f"device must be a CUDA device, not {device!r} (the library has no CPU path)")
+    return device
+
+
 try:
     _raw_stream = torch._C._cuda_getCurrentRawStream
 except AttributeError:  # pragma: no cover - older torch
@@ -179,7 +185,7 @@ def rope_inv_freq(rot_dim, theta):
 
 def mrope_axis_map(half, section, interleaved=True, device="cuda", stream=None):
     """int8 [half]: axis (0 = T, 1 = H, 2 = W) of each frequency."""
-    out = torch.empty(half, dtype=torch.int8, device=device)
+    out = torch.empty(half, dtype=torch.int8, device=_cuda_device(device))
     _check(_lib.ipe_mrope_axis_map(int(half), _i32_host(section, 3), int(bool(interleaved)), _ptr(out),
                                    _stream(stream)))
     return out
@@ -504,6 +510,7 @@ def vis_interp_plan(grid_thw, merge=2, grid_side=48, device="cuda", stream=None)
     """(idx4 int32 [4, N], w4 float32 [4, N], rowcol int32 [2, N]) in output order."""
     g, n = _grid_host(grid_thw)
     N = sum(g[3 * i] * g[3 * i + 1] * g[3 * i + 2] for i in range(n))
+    device = _cuda_device(device)
     idx4 = torch.empty(4, N, dtype=torch.int32, device=device)
     w4 = torch.empty(4, N, dtype=torch.float32, device=device)
     rowcol = torch.empty(2, N, dtype=torch.int32, device=device)
