@@ -32,7 +32,7 @@ def _rank(rank, world, port, ms_by_rank, out):
 def test_two_ranks_take_the_slowest_rank():
     world = 2
     ms_by_rank = [0.40, 0.55]
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:     # no fork after torch's threads start
         out = m.dict()
         mp.spawn(_rank, args=(world, _free_port(), ms_by_rank, out), nprocs=world, join=True)
         res = dict(out)
