@@ -46,3 +46,38 @@ def test_single_rank_needs_no_group():
     import bench
     ms, value = bench.job_time_and_value(0.5, 1000, 1, None)
     assert ms == 0.5 and value == pytest.approx(2e6)
+
+
+def _rank_leaves(rank, world, port, out):
+    from datetime import timedelta
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=10))
+    if rank == 1:
+        os._exit(0)                      # leaves between steps, nothing in flight
+    import bench
+    try:
+        bench.dist_max(0.5, "cpu")
+        out[rank] = "completed"
+    except Exception as e:  # noqa: BLE001 - any error is the expected outcome
+        out[rank] = "error: " + type(e).__name__
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_ends_the_others_with_an_error():
+    # The surviving rank's step-time reduction must end with an error (peer
+    # gone or timeout), not wait for good.
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        procs = [ctx.Process(target=_rank_leaves, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+        alive = [p for p in procs if p.is_alive()]
+        for p in alive:
+            p.kill()
+        assert not alive, "a rank did not finish"
+        assert str(out.get(0, "")).startswith("error"), dict(out)
