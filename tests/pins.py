@@ -343,39 +343,52 @@ def pin_vision_angles_basis(o):
         assert not others.any()
 
 
-def _torch_listing_vision_rotary(q, grids, m, theta):
-    """rot_pos_emb and apply_rotary_pos_emb_vision of the "Qwen3-VL" notes,
-    evaluated by torch in fp32 on the CPU: (row, col) ids per token in merge
-    order, an fp32 frequency table looked up and flattened to [rows | cols],
-    duplicated to the head width, and q cos + rotate_half(q) sin."""
-    import torch
-    head_dim = q.shape[-1]
-    dim = head_dim // 2
-    inv = 1.0 / (theta ** (torch.arange(0, dim, 2, dtype=torch.float) / dim))
-    max_hw = max(max(h, w) for _, h, w in grids)
-    table = torch.outer(torch.arange(max_hw, dtype=torch.float), inv)
-    ids = []
+def _patch_rowcol(grids, m):
+    """(row, col) of every output row from its index alone.  Inside a frame,
+    patch q = r mod (h w) is patch q mod m^2 (row-major, m x m) of merge
+    block q div m^2, and the blocks run row-major over the (h/m) x (w/m)
+    block grid; frames repeat and images follow one another."""
+    out = []
     for t, h, w in grids:
-        br = torch.arange(h // m)[:, None, None, None] * m + torch.arange(m)[None, None, :, None]
-        bc = torch.arange(w // m)[None, :, None, None] * m + torch.arange(m)[None, None, None, :]
-        rows = br.expand(h // m, w // m, m, m).reshape(-1)
-        cols = bc.expand(h // m, w // m, m, m).reshape(-1)
-        ids.append(torch.stack([rows, cols], -1).repeat(t, 1))
-    emb = table[torch.cat(ids)].flatten(1)
-    emb = torch.cat([emb, emb], -1)
-    cos, sin = emb.cos()[:, None, :], emb.sin()[:, None, :]
-    x = torch.from_numpy(q).float()
-    rh = torch.cat([-x[..., head_dim // 2:], x[..., :head_dim // 2]], -1)
-    return (x * cos + rh * sin).double().numpy()
+        q = np.arange(t * h * w) % (h * w)
+        blk, inner = q // (m * m), q % (m * m)
+        by, bx = blk // (w // m), blk % (w // m)
+        out.append(np.stack([by * m + inner // m, bx * m + inner % m], 1))
+    return np.concatenate(out).astype(np.int64)
 
 
-def pin_vision_rotary_matches_torch_listing(o):
-    # fp32 (torch) against double (oracle): agreement to fp32 rounding
+def _vision_rotary_fp32(q, grids, m, theta):
+    """The vision rotary evaluated in fp32 from its definition: channel pair
+    (j, j + D/2) of every head turns by a_j, with a_j = row * w_j for
+    j < D/4 and col * w_(j - D/4) above, w_i = theta^(-2i / (D/2)) (formed
+    here as exp(-(2i / (D/2)) ln theta) in fp32), and (row, col) the patch's
+    grid point in merge order."""
+    N, H, D = q.shape
+    rc = _patch_rowcol(grids, m).astype(np.float32)
+    i = np.arange(D // 4, dtype=np.float32)
+    w = np.exp(-(np.float32(2) * i / np.float32(D // 2)) * np.float32(np.log(theta)))
+    ang = np.concatenate([rc[:, :1] * w[None], rc[:, 1:] * w[None]], 1)          # [N, D/2] fp32
+    c, s = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+    a, b = q[..., :D // 2].astype(np.float32), q[..., D // 2:].astype(np.float32)
+    return np.concatenate([a * c - b * s, b * c + a * s], -1).astype(np.float64)
+
+
+def pin_patch_rowcol_closed_form(o):
+    # the closed form of the merge order against the brute-force loops
+    for grids, m in [([(1, 4, 6), (2, 6, 4), (1, 8, 8)], 2), ([(3, 6, 9)], 3), ([(1, 1, 5), (2, 3, 1)], 1)]:
+        brute = np.concatenate([_merge_order_rowcol(t, h, w, m) for t, h, w in grids])
+        assert np.array_equal(_patch_rowcol(grids, m), brute)
+        assert np.array_equal(o.vis_rot_pos_ids(grids, m), brute)
+
+
+def pin_vision_rotary_matches_fp32_angles(o):
+    # fp32 evaluation of the definition against the double oracle: agreement
+    # to fp32 rounding (angles up to 7 rad, so a few 1e-6)
     rng = _rng(43)
     grids = [(1, 4, 6), (2, 6, 4), (1, 8, 8)]
     N = sum(t * h * w for t, h, w in grids)
     q = rng.standard_normal((N, 3, 72)).astype(np.float32)
-    want = _torch_listing_vision_rotary(q, grids, 2, 1e4)
+    want = _vision_rotary_fp32(q, grids, 2, 1e4)
     got = o.vis_apply_rotary(q.astype(np.float64), grids, 2, 1e4)
     assert np.abs(got - want).max() <= 2e-5, np.abs(got - want).max()
 
@@ -556,51 +569,75 @@ def pin_decode_closed_forms(o):
 # ------------------------------------------------------------ HF rounding
 
 
-def _torch_listing_interp(table, grids, m):
-    """The interpolation listing's steps evaluated by torch in the table's
-    dtype on the table's device (torch's bf16 arithmetic computes in fp32 and
-    rounds back); the sample points come from torch.linspace on the CPU."""
+def _round_to(x, dtype):
+    """fp32 values rounded to the dtype (nearest, ties to even); fp32 as is."""
+    x = np.asarray(x, np.float32)
+    if dtype == "bf16":
+        import workloads as wl
+        return wl.bf16_bits_to_f32(wl.f32_to_bf16_bits(x))
+    return x
+
+
+def _interp_by_sample_points(table, grids, m, rounding):
+    """Every output row as the bilinear blend of the table at its own sample
+    point.  The point of grid row i of an n-row image is the fp32
+    torch.linspace(0, G-1, n)[i] (torch's own routine, which fixes the HF
+    sample points); its corners are the floor y0 and min(y0 + 1, G - 1), its
+    fraction f = point - y0, and the four weights (1-fy)(1-fx), (1-fy)fx,
+    fy(1-fx), fy fx are fp32 products, in the corner order TL, TR, BL, BR.
+      rounding "f64":  weights widened to double, blend in double;
+      "f32" / "bf16":  the HF rounding points -- each weight rounded to the
+                       dtype, each weight x value product and each partial
+                       sum, taken left to right over the corners, computed
+                       in fp32 and rounded to the dtype.
+    table: [G*G, C] float64 holding values of the dtype.  Frames repeat
+    their image; rows are in merge order."""
     import torch
     G = int(round(table.shape[0] ** 0.5))
-    outs = []
+    out = []
     for t, h, w in grids:
-        ys, xs = torch.linspace(0, G - 1, h), torch.linspace(0, G - 1, w)
-        y0, x0 = ys.int(), xs.int()
-        y1, x1 = (y0 + 1).clip(max=G - 1), (x0 + 1).clip(max=G - 1)
-        dy, dx = ys - y0, xs - x0
-        corners = torch.stack([(y0[:, None] * G + x0[None]), (y0[:, None] * G + x1[None]),
-                               (y1[:, None] * G + x0[None]), (y1[:, None] * G + x1[None])]).reshape(4, -1)
-        wts = torch.stack([torch.outer(1 - dy, 1 - dx), torch.outer(1 - dy, dx), torch.outer(dy, 1 - dx),
-                           torch.outer(dy, dx)]).reshape(4, -1).to(table.dtype).to(table.device)
-        prod = table[corners.long().to(table.device)] * wts[:, :, None]
-        frame = ((prod[0] + prod[1]) + prod[2]) + prod[3]
-        merged = frame.repeat(t, 1).view(t, h // m, m, w // m, m, -1).permute(0, 1, 3, 2, 4, 5).reshape(t * h * w, -1)
-        outs.append(merged)
-    return torch.cat(outs)
+        rc = _patch_rowcol([(1, h, w)], m)
+        sy = torch.linspace(0, G - 1, h).numpy()[rc[:, 0]]
+        sx = torch.linspace(0, G - 1, w).numpy()[rc[:, 1]]
+        y0, x0 = np.floor(sy).astype(np.int64), np.floor(sx).astype(np.int64)
+        y1, x1 = np.minimum(y0 + 1, G - 1), np.minimum(x0 + 1, G - 1)
+        fy, fx = sy - y0.astype(np.float32), sx - x0.astype(np.float32)
+        one = np.float32(1)
+        weights = [(one - fy) * (one - fx), (one - fy) * fx, fy * (one - fx), fy * fx]
+        corners = [y0 * G + x0, y0 * G + x1, y1 * G + x0, y1 * G + x1]
+        if rounding == "f64":
+            frame = sum(wt.astype(np.float64)[:, None] * table[c] for wt, c in zip(weights, corners))
+        else:
+            frame = None
+            for wt, c in zip(weights, corners):
+                p = _round_to(_round_to(wt, rounding)[:, None] * table[c].astype(np.float32), rounding)
+                frame = p if frame is None else _round_to(frame + p, rounding)
+            frame = frame.astype(np.float64)
+        out.append(np.tile(frame, (t, 1)))
+    return np.concatenate(out)
 
 
-def pin_interp_hf_matches_torch_listing(o):
-    import torch
+def pin_interp_hf_matches_sample_points(o):
+    # The oracle's HF mode (the listing's tensor steps, in C) against the
+    # per-element statement above, bit for bit
     rng = _rng(29)
     cases = [([(1, 4, 6), (2, 6, 4), (1, 48, 48), (1, 10, 14)], 2), ([(1, 5, 7), (3, 1, 9)], 1)]
-    for dt, tdt in (("bf16", torch.bfloat16), ("f32", torch.float32)):
-        table = torch.from_numpy(rng.standard_normal((48 * 48, 24)).astype(np.float32)).to(tdt)
-        vals = table.float().numpy().astype(np.float64)
+    for dt in ("bf16", "f32"):
+        vals = _round_to(rng.standard_normal((48 * 48, 24)), dt).astype(np.float64)
         for grids, m in cases:
-            want = _torch_listing_interp(table, grids, m).float().numpy().astype(np.float64)
+            want = _interp_by_sample_points(vals, grids, m, dt)
             got = o.vis_pos_interp_hf(vals, grids, m, dt)
             assert got.shape == want.shape and (got == want).all(), (dt, grids)
 
 
-def pin_interp_matches_torch_listing(o):
+def pin_interp_matches_sample_points(o):
     # The default interpolation (exact sample points, double) against the
-    # listing run by torch in float64 with its fp32 linspace: they differ only
-    # by the rounding of the sample points (a few 1e-7 of a table value).
-    import torch
+    # per-element blend at the fp32 linspace points: they differ only by the
+    # rounding of the sample points (a few 1e-7 of a table value).
     rng = _rng(47)
     table = rng.standard_normal((48 * 48, 12))
     for grids, m in [([(1, 4, 6), (2, 10, 14), (1, 48, 64)], 2), ([(1, 5, 7), (3, 1, 9)], 1)]:
-        want = _torch_listing_interp(torch.from_numpy(table), grids, m).numpy()
+        want = _interp_by_sample_points(table, grids, m, "f64")
         got = o.vis_pos_embed_interpolate(table, grids, m)
         assert np.abs(got - want).max() <= 2e-5 * np.abs(table).max(), np.abs(got - want).max()
 
@@ -639,53 +676,39 @@ def pin_hf_rounding_close_to_exact(o):
     assert np.abs(hf - exact).max() <= 1e-5 * (1 + np.abs(exact).max())
 
 
-def _torch_listing_mrope_freqs(pos, inv):
-    """The text rotary's angle table as the pages' forward() builds it: the
-    shared inv_freq against each axis's positions, both as fp32, by a
-    one-column matmul, then transposed to [3, B, L, half]."""
-    import torch
-    p = torch.from_numpy(pos)[:, None, :]                      # [3, B=1, L]
-    inv_e = torch.from_numpy(inv)[None, None, :, None].float().expand(3, 1, -1, 1)
-    return (inv_e @ p[:, :, None, :].float()).transpose(2, 3)   # [3, 1, L, half]
+def _interleaved_axis(j, sec):
+    """Axis of frequency j in the interleaved layout, from the selection
+    rule: H on frequencies 1, 4, 7, ... below 3 s_h, W on 2, 5, 8, ... below
+    3 s_w, T on every other one."""
+    if j % 3 == 1 and j < 3 * sec[1]:
+        return 1
+    if j % 3 == 2 and j < 3 * sec[2]:
+        return 2
+    return 0
 
 
-def _torch_listing_interleave(f, sec):
-    """Axis T everywhere, then H on frequencies 1, 4, 7, ... and W on 2, 5,
-    8, ..., each up to 3 x its section, then the halves duplicated."""
-    import torch
-    ft = f[0].clone()
-    for axis, offset in ((1, 1), (2, 2)):
-        sl = slice(offset, sec[axis] * 3, 3)
-        ft[..., sl] = f[axis][..., sl]
-    return torch.cat((ft, ft), dim=-1)
-
-
-def pin_mrope_cos_sin_matches_torch_listings(o):
-    # The interleaved text cos / sin against the two forms the pages print,
-    # run by torch in fp32: selection of the angles before the cos
-    # ("Qwen3-VL" notes, Qwen3VLTextRotaryEmbedding.forward and
-    # apply_interleaved_mrope) and selection of the cos / sin tables after it
-    # ("Interleaved Rotary Position Embedding", Qwen3_5TextRotaryEmbedding and
-    # recomposition_frequencies).  The angles must agree exactly (the cos of
-    # torch's fp32 angles in double equals the oracle's), the fp32 cos / sin
-    # within their own rounding.
+def pin_mrope_cos_sin_fp32_angles(o):
+    # The interleaved text angles are fp32 products fl32(fl32(pos) * inv_j)
+    # of the frequency's own axis; the oracle's cos / sin are the double cos /
+    # sin of exactly those angles, and fp32 cos / sin (numpy) agree with them
+    # to fp32 rounding.  Selecting axes before or after the cos is the same
+    # table (the cos is elementwise).  A position above 2^24 is rounded by
+    # the fp32 conversion.
     rng = _rng(53)
     for half, sec, theta in [(64, (24, 20, 20), 5e6), (32, (11, 11, 10), 1e7), (10, (4, 3, 3), 1e4)]:
         L = 40
         pos = rng.integers(0, 300000, (3, L)).astype(np.int64)
-        pos[:, 0] = (1 << 24) + 1                  # rounded by the fp32 conversion
+        pos[:, 0] = (1 << 24) + 1
         pos[:, 1] = [7, 7, 7]
         inv = o.rope_inv_freq(2 * half, theta)
         cos, sin = o.mrope_cos_sin(pos, inv, sec, True)
-        f = _torch_listing_mrope_freqs(pos, inv)
-        emb = _torch_listing_interleave(f, sec)[0]               # [L, 2 half]
-        e64 = emb.double().numpy()
-        assert np.abs(np.cos(e64) - cos).max() <= 4e-16 and np.abs(np.sin(e64) - sin).max() <= 4e-16
-        c1, s1 = emb.cos().numpy(), emb.sin().numpy()
-        c2 = _torch_listing_interleave(f.cos(), sec)[0].numpy()
-        s2 = _torch_listing_interleave(f.sin(), sec)[0].numpy()
-        for c, s in ((c1, s1), (c2, s2)):
-            assert np.abs(c - cos).max() <= 1.2e-7 and np.abs(s - sin).max() <= 1.2e-7, (half, sec)
+        axis = np.array([_interleaved_axis(j, sec) for j in range(half)])
+        p32 = pos.astype(np.float32)[axis]                       # [half, L]: the axis each column reads
+        ang = (p32 * inv[:, None].astype(np.float32)).T           # [L, half] fp32 products
+        ang = np.concatenate([ang, ang], 1).astype(np.float64)
+        assert np.abs(np.cos(ang) - cos).max() <= 4e-16 and np.abs(np.sin(ang) - sin).max() <= 4e-16
+        c32, s32 = np.cos(ang.astype(np.float32)), np.sin(ang.astype(np.float32))
+        assert np.abs(c32 - cos).max() <= 1.2e-7 and np.abs(s32 - sin).max() <= 1.2e-7, (half, sec)
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -1,6 +1,7 @@
 """HF rounding mode (through the C ABI): bit for bit against the oracle's
-emulation of the listings' rounding points, and against those listings run
-by torch on the GPU.
+emulation of the listings' rounding points, against a per-element statement
+of the same rounding points (the interpolation), and against torch's own
+arithmetic on the GPU (the rotation).
 
 The interpolation has no transcendental step, so the oracle comparison is
 exact.  The rotation's cos / sin are fp32 values of sincosf on the GPU and
@@ -16,7 +17,7 @@ import torch
 import interpolated_position_encoding_b200 as ipe
 import workloads as wl
 from gpu_helpers import F32_ATOL, gpu_to_f64, host_f64, to_gpu, ulp_bf16
-from pins import _torch_listing_interp
+from pins import _interp_by_sample_points
 
 pytestmark = pytest.mark.gpu
 
@@ -44,9 +45,8 @@ def test_interp_hf_bitwise(dtype, grids, m, G, orc):
     assert g.shape == want.shape
     bad = np.argwhere(g != want)
     assert bad.size == 0, f"{len(bad)} values differ from the oracle, first at {bad[:4].tolist()}"
-    # and the listing itself, run by torch on the GPU
-    ref = _torch_listing_interp(gt, grids, m)
-    assert torch.equal(got, ref)
+    # and the per-element statement of the same rounding points
+    assert (g == _interp_by_sample_points(host_f64(table, dtype), grids, m, dtype)).all()
 
 
 @pytest.mark.parametrize("name", ["vision_batch8_bf16", "prefill_t131072_video"])
@@ -57,10 +57,11 @@ def test_interp_hf_workloads(name, orc):
     gt = to_gpu(vin["table"], v.dtype)
     got = ipe.vis_pos_interp(gt, v.grid_thw, v.merge, rounding="hf")
     ipe.device_status()
-    assert torch.equal(got, _torch_listing_interp(gt, v.grid_thw, v.merge))
+    g = gpu_to_f64(got)
+    assert (g == _interp_by_sample_points(host_f64(vin["table"], v.dtype), v.grid_thw, v.merge, v.dtype)).all()
     if name == "vision_batch8_bf16":
         want = orc.vis_pos_interp_hf(host_f64(vin["table"], v.dtype), v.grid_thw, v.merge, v.dtype)
-        assert (gpu_to_f64(got) == want).all()
+        assert (g == want).all()
 
 
 def _torch_rotation(x, cos, sin, rot):
@@ -178,3 +179,18 @@ def test_rounding_argument_rejected():
     with pytest.raises(ValueError):
         ipe.mrope_apply(q, None, torch.zeros(3, 4, dtype=torch.int32, device="cuda"), ipe.rope_inv_freq(64, 1e4),
                         (12, 10, 10), rounding="bf16")
+
+
+def test_interp_hf_linspace_sweep():
+    # Every grid side from 2 to 1024 (G = 48, merge 1): the HF kernel's sample
+    # points are torch.linspace's fp32 points bit for bit, seen through the
+    # blend of a random fp32 table (a point one ulp off changes its weights).
+    rng = np.random.default_rng(77)
+    table = wl.normal_f32(rng, (48 * 48, 8), 1.0)
+    gt = to_gpu(table, "f32")
+    sides = range(2, 1025)
+    for grids in ([(1, n, 2) for n in sides], [(1, 2, n) for n in sides]):
+        got = gpu_to_f64(ipe.vis_pos_interp(gt, grids, 1, rounding="hf"))
+        want = _interp_by_sample_points(host_f64(table, "f32"), grids, 1, "f32")
+        bad = np.argwhere(got != want)
+        assert bad.size == 0, f"{len(bad)} values differ, first rows {bad[:4, 0].tolist()}"
