@@ -15,18 +15,27 @@
 //   * frames repeat frame 0; rows in merge order.
 //
 // The default kernel (vis_interp_kernel) evaluates the separable form in
-// fp32 with one rounding; this one evaluates the four-corner sum directly:
-// a block takes one merge-row strip of frame 0 and 32 chunks of 16 bytes of
-// the channels, each warp one output row at a time, and each result chunk
-// is written once per frame.  For bf16 the products and sums run as packed
-// bf16x2 operations, which round exactly where the fp32-then-round steps
-// above do (mul_bf16x2 / add_bf16x2).
+// fp32 with one rounding; this one evaluates the four-corner sum directly.
+// A block takes one merge-row strip of an image, 32 chunks of 16 bytes of
+// the channels and a range of the video's frames:
+//   * set-up: each patch of the strip gets its four corner rows and four
+//     weights (rounded to the dtype) once, in shared memory;
+//   * each warp then takes two output rows at a time (eight 16-byte table
+//     loads in flight per lane), forms the four products and the
+//     left-to-right sums, and writes each result chunk to every frame of
+//     its range (frames repeat frame 0).
+// The frame ranges split a video over more blocks, so that a request of few
+// strips still puts about four blocks on every SM.  For bf16 the products
+// and sums run as packed bf16x2 operations, which round exactly where the
+// fp32-then-round steps above do (mul_bf16x2 / add_bf16x2).
 #include "ipe_internal.h"
 #include "ipe_device.cuh"
+#include "ipe_rotary.cuh"
 
 namespace ipe {
 
 constexpr int kHfWarps = 8;
+constexpr int kHfPlanCache = 1024;   // strips of at most this many patches keep their plan in shared memory
 
 // torch.linspace(0, G - 1, n)[i] in fp32.
 __device__ __forceinline__ float hf_linspace(int i, int n, int G)
@@ -38,85 +47,147 @@ __device__ __forceinline__ float hf_linspace(int i, int n, int G)
     return __fmaf_rn(-(float)(n - 1 - i), step, end);
 }
 
+// Corner table rows and weights of one output patch.  For bf16 the weights
+// are bf16x2 words (the weight in both halves); for fp32 their bits.
+struct HfPatch {
+    int4 idx;
+    uint4 w;
+};
+
+template <typename T>
+__device__ __forceinline__ HfPatch hf_patch(int q, int sl, int m, int h, int w, int G)
+{
+    // merge order inside the strip: block column, then the m x m block row-major
+    const int bx = q / (m * m), rr = q - bx * m * m;
+    const int ih = sl * m + rr / m, iw = bx * m + rr % m;
+    const float fy = hf_linspace(ih, h, G), fx = hf_linspace(iw, w, G);
+    const int y0 = (int)fy, x0 = (int)fx;
+    const int y1 = min(y0 + 1, G - 1), x1 = min(x0 + 1, G - 1);
+    const float dh = __fsub_rn(fy, (float)y0), dw = __fsub_rn(fx, (float)x0);
+    const float oh = __fsub_rn(1.f, dh), ow = __fsub_rn(1.f, dw);
+    const float wt[4] = {round_to_dtype<T>(__fmul_rn(oh, ow)), round_to_dtype<T>(__fmul_rn(oh, dw)),
+                         round_to_dtype<T>(__fmul_rn(dh, ow)), round_to_dtype<T>(__fmul_rn(dh, dw))};
+    HfPatch p;
+    p.idx = make_int4(y0 * G + x0, y0 * G + x1, y1 * G + x0, y1 * G + x1);
+    uint32_t wb[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        if constexpr (sizeof(T) == 2) {
+            const __nv_bfloat162 b = __floats2bfloat162_rn(wt[k], wt[k]);   // exact: wt[k] is a bf16 value
+            wb[k] = *reinterpret_cast<const uint32_t *>(&b);
+        } else {
+            wb[k] = __float_as_uint(wt[k]);
+        }
+    }
+    p.w = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+    return p;
+}
+
+// One 16-byte chunk of an output row: the four products and the sums.
+template <typename T>
+__device__ __forceinline__ uint4 hf_blend(const uint4 (&c)[4], const uint4 &w)
+{
+    const uint32_t wk[4] = {w.x, w.y, w.z, w.w};
+    if constexpr (sizeof(T) == 2) {
+        const uint32_t cv[4][4] = {{c[0].x, c[0].y, c[0].z, c[0].w}, {c[1].x, c[1].y, c[1].z, c[1].w},
+                                   {c[2].x, c[2].y, c[2].z, c[2].w}, {c[3].x, c[3].y, c[3].z, c[3].w}};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t acc = mul_bf16x2(cv[0][i], wk[0]);
+#pragma unroll
+            for (int k = 1; k < 4; ++k) acc = add_bf16x2(acc, mul_bf16x2(cv[k][i], wk[k]));
+            o[i] = acc;
+        }
+        return make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+        const float cv[4][4] = {{__uint_as_float(c[0].x), __uint_as_float(c[0].y), __uint_as_float(c[0].z), __uint_as_float(c[0].w)},
+                                {__uint_as_float(c[1].x), __uint_as_float(c[1].y), __uint_as_float(c[1].z), __uint_as_float(c[1].w)},
+                                {__uint_as_float(c[2].x), __uint_as_float(c[2].y), __uint_as_float(c[2].z), __uint_as_float(c[2].w)},
+                                {__uint_as_float(c[3].x), __uint_as_float(c[3].y), __uint_as_float(c[3].z), __uint_as_float(c[3].w)}};
+        float o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float acc = __fmul_rn(cv[0][e], __uint_as_float(wk[0]));
+#pragma unroll
+            for (int k = 1; k < 4; ++k) acc = __fadd_rn(acc, __fmul_rn(cv[k][e], __uint_as_float(wk[k])));
+            o[e] = acc;
+        }
+        return make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]), __float_as_uint(o[3]));
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(32 * kHfWarps) vis_interp_hf_kernel(const __grid_constant__ VisDesc<1024> d,
-                                                                      const __grid_constant__ InterpArgs ia)
+                                                                      const __grid_constant__ InterpArgs ia, int fpb)
 {
-    constexpr int EC = 16 / sizeof(T);
+    __shared__ HfPatch plan[kHfPlanCache];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int s = blockIdx.x;
     const VisImage im = d.img[find_image_of_strip(d, s)];
+    const int f0 = blockIdx.z * fpb, f1 = min(im.t, f0 + fpb);
+    if (f0 >= f1) return;                             // this image has fewer frames (whole block: no barrier yet)
     const int m = d.merge, G = d.grid_side, h = im.h, w = im.w;
     const int sl = s - im.strip0;                     // merge-row strip within the frame
+    const int nq = m * w;                             // patches of the strip
+    const bool cached = nq <= kHfPlanCache;
+    if (cached)
+        for (int q = threadIdx.x; q < nq; q += blockDim.x) plan[q] = hf_patch<T>(q, sl, m, h, w, G);
+    __syncthreads();
+    constexpr int EC = 16 / sizeof(T);
     const int chunks = ia.hidden / EC;
     const int ch = blockIdx.y * 32 + lane;            // this lane's 16-byte chunk
+    if (ch >= chunks) return;
     const long long hw = (long long)h * w;
-    const T *table = static_cast<const T *>(ia.table);
-    T *out = static_cast<T *>(ia.out);
-    for (int q = warp; q < m * w; q += kHfWarps) {
-        // merge order inside the strip: block column, then the m x m block row-major
-        const int bx = q / (m * m), rr = q - bx * m * m;
-        const int ih = sl * m + rr / m, iw = bx * m + rr % m;
-        const float fy = hf_linspace(ih, h, G), fx = hf_linspace(iw, w, G);
-        const int y0 = (int)fy, x0 = (int)fx;
-        const int y1 = min(y0 + 1, G - 1), x1 = min(x0 + 1, G - 1);
-        const float dh = __fsub_rn(fy, (float)y0), dw = __fsub_rn(fx, (float)x0);
-        const float oh = __fsub_rn(1.f, dh), ow = __fsub_rn(1.f, dw);
-        const float wt[4] = {round_to_dtype<T>(__fmul_rn(oh, ow)), round_to_dtype<T>(__fmul_rn(oh, dw)),
-                             round_to_dtype<T>(__fmul_rn(dh, ow)), round_to_dtype<T>(__fmul_rn(dh, dw))};
-        const long long idx[4] = {(long long)y0 * G + x0, (long long)y0 * G + x1, (long long)y1 * G + x0,
-                                  (long long)y1 * G + x1};
-        if (ch >= chunks) continue;
-        const long long row = im.row0 + (long long)sl * m * w + q;
-        if constexpr (sizeof(T) == 2) {
-            // eight bf16 channels as four bf16x2 words; weights broadcast to both halves
-            Pack<uint32_t, 4> c[4], o;
+    const uint4 *tab = reinterpret_cast<const uint4 *>(ia.table) + ch;
+    uint4 *out = reinterpret_cast<uint4 *>(ia.out) + ch;
+    const long long rstride = chunks;                 // uint4 per table / output row
+    const long long row0 = im.row0 + (long long)sl * nq;
+    for (int q = warp; q < nq; q += 2 * kHfWarps) {
+        const int qb = q + kHfWarps;
+        const bool two = qb < nq;
+        const HfPatch pa = cached ? plan[q] : hf_patch<T>(q, sl, m, h, w, G);
+        const HfPatch pb = two ? (cached ? plan[qb] : hf_patch<T>(qb, sl, m, h, w, G)) : pa;
+        uint4 ca[4], cb[4];
+        const int ia4[4] = {pa.idx.x, pa.idx.y, pa.idx.z, pa.idx.w};
+        const int ib4[4] = {pb.idx.x, pb.idx.y, pb.idx.z, pb.idx.w};
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                c[k] = ld_pack<uint32_t, 4>(reinterpret_cast<const uint32_t *>(table + idx[k] * ia.hidden) + ch * 4);
-            uint32_t w2[4];
+        for (int k = 0; k < 4; ++k) ca[k] = tab[ia4[k] * rstride];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const __nv_bfloat162 b = __floats2bfloat162_rn(wt[k], wt[k]);   // exact: wt[k] is a bf16 value
-                w2[k] = *reinterpret_cast<const uint32_t *>(&b);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint32_t acc = mul_bf16x2(c[0].v[i], w2[0]);
-#pragma unroll
-                for (int k = 1; k < 4; ++k) acc = add_bf16x2(acc, mul_bf16x2(c[k].v[i], w2[k]));
-                o.v[i] = acc;
-            }
+        for (int k = 0; k < 4; ++k) cb[k] = tab[ib4[k] * rstride];
+        const uint4 oa = hf_blend<T>(ca, pa.w), ob = hf_blend<T>(cb, pb.w);
 #pragma unroll 1
-            for (int f = 0; f < im.t; ++f)
-                st_pack<uint32_t, 4>(reinterpret_cast<uint32_t *>(out + (row + f * hw) * ia.hidden) + ch * 4, o);
-        } else {
-            Pack<T, EC> c[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) c[k] = ld_pack<T, EC>(table + idx[k] * ia.hidden + (long long)ch * EC);
-            Pack<T, EC> o;
-#pragma unroll
-            for (int e = 0; e < EC; ++e) {
-                float acc = round_to_dtype<T>(__fmul_rn(to_f32(c[0].v[e]), wt[0]));
-#pragma unroll
-                for (int k = 1; k < 4; ++k)
-                    acc = round_to_dtype<T>(__fadd_rn(acc, round_to_dtype<T>(__fmul_rn(to_f32(c[k].v[e]), wt[k]))));
-                o.v[e] = from_f32<T>(acc);
-            }
-#pragma unroll 1
-            for (int f = 0; f < im.t; ++f) st_pack<T, EC>(out + (row + f * hw) * ia.hidden + (long long)ch * EC, o);
+        for (int f = f0; f < f1; ++f) {
+            out[(row0 + q + f * hw) * rstride] = oa;
+            if (two) out[(row0 + qb + f * hw) * rstride] = ob;
         }
     }
+}
+
+// Frames per block: enough blocks for about four per SM, each block taking
+// a whole range of a video's frames.
+static int hf_frames_per_block(const VisDesc<1024> &d, long long blocks_xy)
+{
+    int max_t = 1;
+    for (int i = 0; i < d.n_images; ++i) max_t = std::max(max_t, d.img[i].t);
+    const long long want = 4LL * sm_count();
+    long long groups = (want + blocks_xy - 1) / std::max<long long>(blocks_xy, 1);
+    groups = std::max<long long>(1, std::min<long long>(groups, std::min(max_t, 65535)));
+    return (max_t + (int)groups - 1) / (int)groups;
 }
 
 cudaError_t launch_vis_interp_hf(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, cudaStream_t s)
 {
     const int ec = bf16 ? 8 : 4;
-    const dim3 grid((unsigned)d.n_strips, (unsigned)((ia.hidden / ec + 31) / 32));
+    const unsigned gy = (unsigned)((ia.hidden / ec + 31) / 32);
+    const int fpb = hf_frames_per_block(d, (long long)d.n_strips * gy);
+    int max_t = 1;
+    for (int i = 0; i < d.n_images; ++i) max_t = std::max(max_t, d.img[i].t);
+    const dim3 grid((unsigned)d.n_strips, gy, (unsigned)((max_t + fpb - 1) / fpb));
     if (bf16)
-        vis_interp_hf_kernel<__nv_bfloat16><<<grid, 32 * kHfWarps, 0, s>>>(d, ia);
+        vis_interp_hf_kernel<__nv_bfloat16><<<grid, 32 * kHfWarps, 0, s>>>(d, ia, fpb);
     else
-        vis_interp_hf_kernel<float><<<grid, 32 * kHfWarps, 0, s>>>(d, ia);
+        vis_interp_hf_kernel<float><<<grid, 32 * kHfWarps, 0, s>>>(d, ia, fpb);
     return cudaGetLastError();
 }
 

@@ -27,11 +27,13 @@ GRIDS = [
     ([(1, 4, 6), (2, 6, 4), (1, 48, 48), (1, 48, 64), (2, 28, 28), (1, 80, 56)], 2, 48),
     ([(1, 5, 7), (3, 1, 9), (1, 33, 17)], 1, 48),
     ([(1, 10, 14), (1, 64, 96)], 2, 32),
+    # strips of more patches than the per-block plan holds (computed per row)
+    ([(1, 4, 1100), (2, 2, 6)], 2, 48),
 ]
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("grids,m,G", GRIDS, ids=["m2_g48", "m1_g48", "m2_g32"])
+@pytest.mark.parametrize("grids,m,G", GRIDS, ids=["m2_g48", "m1_g48", "m2_g32", "m2_wide"])
 def test_interp_hf_bitwise(dtype, grids, m, G, orc):
     rng = np.random.default_rng([G, m, len(grids)])
     C = 40 if dtype == "bf16" else 20
