@@ -5,7 +5,8 @@
 
 One step is one pass of the whole path over one prefill request of the
 large-prefill workload: a 16 x 64 x 64 video (65536 patches) through the
-vision position-table interpolation and the vision 2-D rotary, and the
+vision position-table interpolation and the vision 2-D rotary (one call of
+the library's one-call vision entry: the two kernels run concurrently), and the
 language model's interleaved multimodal RoPE on Q [131072, 24, 256] and
 K [131072, 4, 256] (bf16, rotary dim 64, theta 1e7, mrope_section
 [11, 11, 10]).  Inputs are seeded and synthetic, resident in HBM when the
@@ -16,8 +17,9 @@ With N > 1 (torchrun, one process per GPU) every rank runs its own request:
 weak scaling with no data-path collective; the step time is the maximum over
 ranks.  Rank 0 prints one JSON line.
 
---impl reference times the CPU oracle (double precision, one thread) on a
-bounded sample of the same workload instead (rank 0 only).
+--impl reference times the CPU oracle (double precision) on every host core
+instead: one single-threaded oracle process per core, each on its own
+1/16-request slice of the same workload (rank 0 only).
 """
 import argparse
 import hashlib
@@ -44,7 +46,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ipe", "reference"], default="ipe")
-    ap.add_argument("--e2e-steps", type=int, default=3, help="steps of the end-to-end (host buffers) measurement")
+    ap.add_argument("--e2e-steps", type=int, default=50,
+                    help="steps of the end-to-end (host buffers) measurement (about 22 ms each)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-variant side measurements")
@@ -105,9 +108,11 @@ def algorithmic_bytes(w):
     N = wl.n_patches(v)
     eb_v = 2 if v.dtype == "bf16" else 4
     rot_bytes = (t.hq + t.hk) * t.T * t.rot_dim * 2 * 2
+    interp, rope = algorithmic_bytes_vision(v), 2 * N * v.heads * v.head_dim * eb_v * 2
     return {
-        "vis_pos_interp": algorithmic_bytes_vision(v),
-        "vis_rope2d": 2 * N * v.heads * v.head_dim * eb_v * 2,
+        "vis_pos_interp": interp,
+        "vis_rope2d": rope,
+        "vis_pos_interp_rope2d": interp + rope,
         "mrope_apply": rot_bytes + 3 * t.T * 4,
         "mrope_cos_sin": 3 * t.T * 4 + 2 * t.T * t.rot_dim * 4,
         "apply_rotary_partial": rot_bytes + 2 * t.T * t.rot_dim * 4,
@@ -228,61 +233,189 @@ def oracle_sample(w, text_tokens, frames, seed_text_offset=8192):
             "vq": f64(vin["q"]), "vk": f64(vin["k"]), "grid": [(frames, h, ww)]}
 
 
-def run_oracle(orc, w, s):
+def run_oracle(orc, w, s, text_reps=1):
+    """One pass of the oracle over a sample: the text rotary on Q and K
+    (text_reps times over the same window) and the vision interpolation and
+    rotary on its frames."""
     t, v = w.text, w.vision
     inv = orc.rope_inv_freq(t.rot_dim, t.theta)
-    orc.mrope_apply(s["q"], s["pos"], inv, t.section, True)
-    orc.mrope_apply(s["k"], s["pos"], inv, t.section, True)
+    for _ in range(text_reps):
+        orc.mrope_apply(s["q"], s["pos"], inv, t.section, True)
+        orc.mrope_apply(s["k"], s["pos"], inv, t.section, True)
     orc.vis_pos_embed_interpolate(s["table"], s["grid"], v.merge)
     orc.vis_apply_rotary(s["vq"], s["grid"], v.merge, v.theta)
     orc.vis_apply_rotary(s["vk"], s["grid"], v.merge, v.theta)
 
 
-def cpu_baseline(w, text_tokens=65536, frames=8):
-    """Oracle throughput on a bounded sample, scaled to tokens/s of the whole step."""
-    import oracle
-    orc = oracle.get()
-    s = oracle_sample(w, text_tokens, frames)
-    t0 = time.perf_counter()
-    run_oracle(orc, w, s)
-    sec = time.perf_counter() - t0
-    import workloads as wl
-    N = wl.n_patches(w.vision)
-    # the sample keeps the step's token : patch ratio (T / N = 2)
-    frac = text_tokens / w.text.T
-    assert abs(frames * 64 * 64 / N - frac) < 1e-9
-    return {"value": text_tokens / sec, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{text_tokens} tokens (Q and K) + {frames} video frames ({frames * 4096} patches: "
-                      f"interpolation, q and k rotary) = 1/{round(1 / frac)} of a step, {sec:.2f} s"}
+# One oracle slice: a 2048-token window rotated four times (8192 tokens of
+# work) and one 64 x 64 video frame -- 1/16 of a request, with the request's
+# 2 : 1 token : patch ratio.  Windows rotate through the request by worker.
+SLICE_WINDOW, SLICE_REPS, SLICE_FRAMES = 2048, 4, 1
+SLICE_TOKENS = SLICE_WINDOW * SLICE_REPS
+SLICE_TEXT = (f"{SLICE_TOKENS} tokens (Q and K; a {SLICE_WINDOW}-token window x {SLICE_REPS}) + "
+              f"{SLICE_FRAMES * 4096} patches (one 64 x 64 frame: interpolation, q and k rotary)")
 
 
-def reference_arm(args):
-    """--impl reference: the CPU oracle as the reference implementation.  Each
-    step is 1/16 of a request: 8192 tokens (Q and K) and one 64 x 64 video
-    frame (4096 patches: interpolation and q, k rotary), the step's own
-    2 : 1 token : patch ratio.  Rank 0 alone runs it."""
-    if int(os.environ.get("RANK", "0")) != 0:
-        return
+def _slice_sample(w, wid):
+    n_windows = (w.text.T - 8192) // SLICE_WINDOW
+    return oracle_sample(w, SLICE_WINDOW, SLICE_FRAMES, seed_text_offset=8192 + (wid % n_windows) * SLICE_WINDOW)
+
+
+def _oracle_worker(wid, conn):
+    """An oracle process: builds its slice's inputs, reports ready, then runs
+    `rounds` passes over them each time it is asked, returning the
+    (monotonic) start and end of those passes."""
     import oracle
     import workloads as wl
     w = wl.WORKLOADS[WORKLOAD]
     orc = oracle.get()
-    tokens, frames = 8192, 1
-    s = oracle_sample(w, tokens, frames)
-    for _ in range(max(args.warmup, 0)):
-        run_oracle(orc, w, s)
+    s = _slice_sample(w, wid)
+    conn.send("ready")
+    while True:
+        rounds = conn.recv()
+        if rounds is None:
+            break
+        t0 = time.monotonic()
+        for _ in range(rounds):
+            run_oracle(orc, w, s, SLICE_REPS)
+        conn.send((t0, time.monotonic()))
+    conn.close()
+
+
+def oracle_workers():
+    """Worker processes for the all-core oracle run: one per host core this
+    process may use, at most 64, and at most one per 0.5 GB of available
+    memory (a worker holds about 0.4 GB of float64 inputs and outputs)."""
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    avail = None
+    try:
+        with open("/proc/meminfo") as f:
+            for line in f:
+                if line.startswith("MemAvailable:"):
+                    avail = int(line.split()[1]) * 1024
+    except OSError:
+        pass
+    try:
+        with open("/sys/fs/cgroup/memory.max") as f:
+            lim = f.read().strip()
+        if lim.isdigit():
+            avail = min(avail or int(lim), int(lim))
+    except OSError:
+        pass
+    n = min(cores, 64)
+    if avail:
+        n = min(n, max(1, int(avail // (512 << 20))))
+    return max(1, n), cores
+
+
+class OraclePool:
+    """n oracle processes (started with spawn, one thread each), each on its
+    own slice of the request; run(r) has every worker make r passes and
+    returns the wall time from the first start to the last end."""
+
+    def __init__(self, n, timeout=900):
+        import multiprocessing as mp
+        ctx = mp.get_context("spawn")
+        self.timeout = timeout
+        saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+        for k in saved:
+            os.environ[k] = "1"
+        self.conns, self.procs = [], []
+        try:
+            for i in range(n):
+                a, b = ctx.Pipe()
+                p = ctx.Process(target=_oracle_worker, args=(i, b), daemon=True)
+                p.start()
+                b.close()
+                self.conns.append(a)
+                self.procs.append(p)
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        for c in self.conns:
+            if self._recv(c) != "ready":
+                raise RuntimeError("oracle worker failed to start")
+
+    def _recv(self, c):
+        if not c.poll(self.timeout):
+            raise RuntimeError("oracle worker did not answer")
+        return c.recv()
+
+    def run(self, rounds):
+        for c in self.conns:
+            c.send(rounds)
+        spans = [self._recv(c) for c in self.conns]
+        return max(t1 for _, t1 in spans) - min(t0 for t0, _ in spans)
+
+    def close(self):
+        for c in self.conns:
+            try:
+                c.send(None)
+            except (BrokenPipeError, OSError):
+                pass
+        for p in self.procs:
+            p.join(timeout=30)
+            if p.is_alive():
+                p.terminate()
+
+
+def cpu_baseline(w, rounds=6):
+    """The oracle on the host cores: every worker (one per core) runs
+    `rounds` passes over its own 1/16-request slice; throughput is the tokens
+    of all passes over the wall time.  The same slice on one thread in this
+    process gives the single-thread figure."""
+    import oracle
+    orc = oracle.get()
+    s = _slice_sample(w, 0)
+    run_oracle(orc, w, s, SLICE_REPS)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        run_oracle(orc, w, s)
-    sec = time.perf_counter() - t0
-    value = tokens * args.steps / sec
-    sample = f"{tokens} tokens (Q and K) + {frames * 4096} patches per step (1/16 of a request)"
+    for _ in range(2):
+        run_oracle(orc, w, s, SLICE_REPS)
+    single = 2 * SLICE_TOKENS / (time.perf_counter() - t0)
+    n, cores = oracle_workers()
+    pool = OraclePool(n)
+    try:
+        pool.run(1)
+        sec = pool.run(rounds)
+    finally:
+        pool.close()
+    value = n * rounds * SLICE_TOKENS / sec
+    return {"value": value, "unit": UNIT, "cores": n, "host_cores": cores, "kind": "oracle",
+            "sample": f"{n} processes x {rounds} passes over their own slice of {SLICE_TEXT} = "
+                      f"{n * rounds / 16:g} requests in {sec:.2f} s wall; tokens/s of the whole step",
+            "single_thread": {"value": single, "unit": UNIT, "cores": 1,
+                              "sample": f"2 passes over one slice ({SLICE_TEXT})"}}
+
+
+def reference_arm(args):
+    """--impl reference: the CPU oracle as the reference implementation, on
+    every host core (one single-threaded process per core, each on its own
+    1/16-request slice).  One step = one pass of every worker.  Rank 0
+    alone runs it."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import workloads as wl
+    w = wl.WORKLOADS[WORKLOAD]
+    n, cores = oracle_workers()
+    pool = OraclePool(n)
+    try:
+        for _ in range(max(args.warmup, 0)):
+            pool.run(1)
+        sec = sum(pool.run(1) for _ in range(args.steps))
+    finally:
+        pool.close()
+    value = n * SLICE_TOKENS * args.steps / sec
+    sample = f"{n} processes, each one pass over its own slice of {SLICE_TEXT} per step ({n / 16:g} requests)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec / max(args.steps, 1) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "step_sample": sample, "l2": "n/a (CPU)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": n, "host_cores": cores, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -496,20 +629,20 @@ def main():
     grid = v.grid_thw
     stream = torch.cuda.current_stream()
 
-    names = ["vis_pos_interp", "vis_rope2d", "mrope_apply"]
+    # the vision pair through the library's one-call entry: the interpolation
+    # runs on the library's second stream beside the rotation on `stream`,
+    # and `stream` waits for both, so the events on `stream` bracket both
+    names = ["vis_pos_interp_rope2d", "mrope_apply"]
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        ipe.vis_pos_interp(table, grid, v.merge, out=out, stream=stream)
+        ipe.vis_pos_interp_rope2d(table, grid, qv, kv, v.merge, v.theta, out=out, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        ipe.vis_rope2d(qv, kv, grid, v.merge, v.theta, stream=stream)
-        if ev is not None:
-            ev[2].record(stream)
         ipe.mrope_apply(Q, K, pos, inv, t.section, True, stream=stream)
         if ev is not None:
-            ev[3].record(stream)
+            ev[2].record(stream)
 
     def barrier():
         if world > 1:
@@ -527,7 +660,7 @@ def main():
         step()
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
@@ -589,7 +722,7 @@ def main():
         "step_hbm_gbs": step_bytes / (ms_step / 1e3) / 1e9,
         "roofline": roofline,
         "kernels": kernels,
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 3 * args.steps,     # interpolation, vision rotary, fused MRoPE
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,
@@ -774,7 +907,7 @@ def next_rows(ipe, dev, stream, peak, reps):
         nbytes = Bn * Ln * 4 * (1 + (mk is not None) + 3) + Bn * 4
         ms = _time_flushed(torch, stream, lambda: ipe.mrope_rope_index(gty, None, gvg, gmk, t.merge, posb, dl, ws,
                                                                        stream=stream), reps, flush)
-        res[f"rope_index/{name}"] = entry(ms, nbytes, slots=Bn * Ln, launches=3)
+        res[f"rope_index/{name}"] = entry(ms, nbytes, slots=Bn * Ln, launches=2)
 
     # decode step with the prefill model's heads: norm, rotation, cache write
     D, hq, hk, rot = t.head_dim, t.hq, t.hk, t.rot_dim
