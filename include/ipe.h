@@ -78,6 +78,16 @@ const char *ipe_last_error(void);
 int ipe_version(void);
 
 /* ---------------------------------------------------------------------------
+ * ipe_kernel_arch -- the compute capability a library kernel was compiled
+ * for, as the CUDA runtime loaded it on the current device
+ * (cudaFuncGetAttributes: binaryVersion and ptxVersion, major * 10 + minor;
+ * 100 for sm_100a).  Needs a CUDA device; IPE_ECUDA when the library's code
+ * cannot run on it.  Not part of any page: a check of this build.
+ *   binary_version, ptx_version   host int*, written.
+ * ------------------------------------------------------------------------- */
+int ipe_kernel_arch(int *binary_version, int *ptx_version);
+
+/* ---------------------------------------------------------------------------
  * ipe_device_status -- failure report of the kernels that ran on the current
  * device.  The TMA-fed rotation kernels wait on shared-memory barriers; every
  * such wait gives up after a time limit (about one second), records a fault
@@ -325,7 +335,9 @@ size_t ipe_mrope_rope_index_workspace(int64_t B, int64_t L, int n_images, int n_
  * (ipe_mrope_rope_index_workspace) exceeds that are rejected with IPE_ELIMIT.
  * The first call on each device looks the array's address up (with that
  * device current) and so does the set-up work: make it before any stream
- * capture.  Nothing in the scratch needs clearing between calls.  All calls on
+ * capture.  After a device reset in the same process the next call on that
+ * device finds the remembered address stale and does the set-up again.
+ * Nothing in the scratch needs clearing between calls.  All calls on
  * one device share the array: calls whose kernels overlap in time (on other
  * streams or from other host threads) race.  Arguments and results as
  * ipe_mrope_rope_index without workspace / workspace_bytes.

@@ -30,6 +30,7 @@ _P, _I, _I64, _D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_doubl
 _SIGS = {
     "ipe_last_error": (ctypes.c_char_p, []),
     "ipe_version": (_I, []),
+    "ipe_kernel_arch": (_I, [_P, _P]),
     "ipe_device_status": (_I, [_P]),
     "ipe_debug_inject": (_I, [_I64, _I64]),
     "ipe_rope_inv_freq": (_I, [_I, _D, _P]),
@@ -166,6 +167,13 @@ def _row_stride(t, heads, head_dim, name):
 def device_status(stream=None):
     """Synchronise the stream and raise IpeError(IPE_EDEVICE) if a kernel gave up a bounded wait."""
     _check(_lib.ipe_device_status(_stream(stream)))
+
+
+def kernel_arch():
+    """(binaryVersion, ptxVersion) of a library kernel as loaded on the current device (100 = sm_100a)."""
+    b, p = ctypes.c_int(0), ctypes.c_int(0)
+    _check(_lib.ipe_kernel_arch(ctypes.byref(b), ctypes.byref(p)))
+    return b.value, p.value
 
 
 def debug_inject(skip_tile=-1, wait_cycles=0):
@@ -408,18 +416,22 @@ def mrope_rope_index_static(mm_token_type_ids, image_grid_thw, video_grid_thw, a
     here.  Calls on one device share that buffer, so calls that overlap in
     time race; the first call on a device does a one-time set-up and should
     come before any stream capture."""
+    if not isinstance(mm_token_type_ids, torch.Tensor) or mm_token_type_ids.dim() != 2:
+        raise ValueError("mm_token_type_ids must be a [B, L] tensor")
+    B, L = mm_token_type_ids.shape
+    n_img = 0 if image_grid_thw is None else image_grid_thw.shape[0]
+    n_vid = 0 if video_grid_thw is None else video_grid_thw.shape[0]
+    need = rope_index_workspace_bytes(B, L, n_img, n_vid)
+    if need > ROPE_INDEX_STATIC_BYTES:
+        raise IpeError(IPE_ELIMIT, f"these sizes need {need} bytes of scratch, above the {ROPE_INDEX_STATIC_BYTES} "
+                                   "bytes of the library's fixed buffer")
     ty = _int_tensor(mm_token_type_ids, "mm_token_type_ids")
-    if ty.dim() != 2:
-        raise ValueError("mm_token_type_ids must be [B, L]")
-    B, L = ty.shape
     if attention_mask is not None:
         _int_tensor(attention_mask, "attention_mask", (B, L))
     grids = [g for g in (image_grid_thw, video_grid_thw) if g is not None]
     for g in grids:
         _int_tensor(g, "grid")
     gbytes = grids[0].element_size() if grids else 4
-    n_img = 0 if image_grid_thw is None else image_grid_thw.shape[0]
-    n_vid = 0 if video_grid_thw is None else video_grid_thw.shape[0]
     for t, nm, shp in ((position_ids, "position_ids", (3, B, L)), (rope_deltas, "rope_deltas", (B,))):
         _cuda(t, nm)
         if t.dtype != torch.int32 or tuple(t.shape) != shp or not t.is_contiguous():
@@ -582,5 +594,5 @@ def vis_pos_interp_rope2d(table, grid_thw, q, k, merge=2, theta=1e4, out=None, s
     return out, q, k
 
 
-__all__ = ["IpeError", "lib", "EXPORTS", "device_status", "debug_inject", "rope_inv_freq", "mrope_axis_map", "mrope_cos_sin", "apply_rotary_partial",
+__all__ = ["IpeError", "lib", "EXPORTS", "device_status", "kernel_arch", "debug_inject", "rope_inv_freq", "mrope_axis_map", "mrope_cos_sin", "apply_rotary_partial",
            "mrope_apply", "qk_norm_mrope", "vis_interp_plan", "vis_pos_interp", "vis_rope2d", "vis_pos_interp_rope2d"]

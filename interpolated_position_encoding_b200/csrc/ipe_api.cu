@@ -332,6 +332,17 @@ const char *ipe_last_error(void) { return g_err.c_str(); }
 
 int ipe_version(void) { return 100; }
 
+int ipe_kernel_arch(int *binary_version, int *ptx_version)
+{
+    if (binary_version == nullptr || ptx_version == nullptr) return fail(IPE_EINVAL, "output pointer is NULL");
+    cudaFuncAttributes attr{};
+    cudaError_t e = mrope_axis_map_attributes(&attr);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+    *binary_version = attr.binaryVersion;
+    *ptx_version = attr.ptxVersion;
+    return ok();
+}
+
 int ipe_device_status(void *stream)
 {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

@@ -181,6 +181,9 @@ bool encode_tmap(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void 
 // Launchers (return cudaGetLastError() of the launch).
 cudaError_t launch_mrope_cos_sin(const MropeAngles &a, int half, float *cos_out, float *sin_out,
                                  cudaStream_t s);
+// Attributes of a library kernel as loaded on the current device (the
+// architecture its code was built for).
+cudaError_t mrope_axis_map_attributes(cudaFuncAttributes *attr);
 cudaError_t launch_mrope_axis_map(int half, const int *section, int interleaved, int8_t *axis,
                                   cudaStream_t s);
 cudaError_t launch_rotary_mrope(bool bf16, const RotArgs &r, const MropeAngles &a, cudaStream_t s,

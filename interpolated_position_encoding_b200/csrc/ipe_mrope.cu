@@ -28,6 +28,11 @@ cudaError_t launch_mrope_axis_map(int half, const int *section, int interleaved,
     return cudaGetLastError();
 }
 
+cudaError_t mrope_axis_map_attributes(cudaFuncAttributes *attr)
+{
+    return cudaFuncGetAttributes(attr, mrope_axis_map_kernel);
+}
+
 // ---------------------------------------------------------- cos / sin
 // Block (G, 256 / G): threadIdx.x is one of the G = half / V groups of V
 // consecutive frequencies of a token, threadIdx.y a token.  Each thread

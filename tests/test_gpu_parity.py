@@ -100,6 +100,24 @@ def test_mrope_apply_small(case, dtype, interleaved, orc):
         assert np.array_equal(out[..., rot:], host_f64(x, dtype)[..., rot:]), "pass-through changed"
 
 
+@pytest.mark.parametrize("T,half,section", [(1000, 32, (11, 11, 10)), (777, 64, (24, 20, 20)),
+                                             (1001, 256, (86, 85, 85)), (5, 12, (4, 4, 4)), (3, 3, (1, 1, 1))])
+@pytest.mark.parametrize("interleaved", [True, False])
+def test_cos_sin_tiles_and_tail(T, half, section, interleaved, orc):
+    # the tables alone against the oracle: many tiles of tokens and a ragged
+    # last one (tiles of 2048 / half tokens when half is a multiple of 4),
+    # both halves of every row equal
+    rng = GEN(T + half)
+    pos = _rand_positions(rng, T)
+    ginv = ipe.rope_inv_freq(2 * half, 1e6)
+    cos, sin = ipe.mrope_cos_sin(torch.from_numpy(pos).cuda(), ginv, section, interleaved)
+    rc, rs = orc.mrope_cos_sin(pos, orc.rope_inv_freq(2 * half, 1e6), section, interleaved)
+    check(cos.cpu().numpy(), rc, None, "f32", "cos")
+    check(sin.cpu().numpy(), rs, None, "f32", "sin")
+    c = cos.cpu().numpy()
+    assert np.array_equal(c[:, :half], c[:, half:])
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_apply_rotary_partial_independent_tables(dtype, orc):
     # cos / sin are inputs: arbitrary tables whose halves differ exercise the
@@ -258,7 +276,7 @@ def test_interp_workload(name, orc):
 @pytest.mark.parametrize("grids,merge,G,C", [
     ([(1, 48, 48)], 2, 48, 64), ([(1, 1, 5), (1, 3, 1)], 1, 48, 1152), ([(1, 6, 9)], 3, 48, 100),
     ([(1, 8, 12)], 2, 4, 36), ([(2, 4, 6), (1, 2, 2), (3, 6, 4)], 2, 48, 1000), ([(1, 2, 4)] * 20, 2, 48, 132),
-    ([(1, 96, 2)], 2, 48, 1152),
+    ([(1, 96, 2)], 2, 48, 1152), ([(1, 2, 1030), (1, 4, 4)], 2, 48, 64),   # wider than the column cache
     # enough strips for two channel slices per block, with a ragged last group
     ([(1, 24, 4)] * 100, 2, 48, 1000), ([(1, 12, 4)] * 400, 2, 48, 100), ([(1, 8, 4)] * 300, 1, 48, 1152)])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -328,7 +346,21 @@ def test_vis_rope_basis_readback(orc):
         assert np.abs(out[:, j, j + 36] - np.sin(a)).max() <= 2e-7
 
 
-@pytest.mark.parametrize("name", ["vision_batch8_bf16", "vision_16x16_f32"])
+def _frame_sample(grids, N, seed, n_random=4096, edge=256, around=8):
+    """Patch rows for a sampled check at full size: both ends, a few rows on
+    either side of every frame and image boundary, and random rows."""
+    rows = [np.arange(min(edge, N)), np.arange(max(N - edge, 0), N)]
+    r0 = 0
+    for t, h, w in grids:
+        for f in range(t + 1):
+            b = r0 + f * h * w
+            rows.append(np.arange(max(b - around, 0), min(b + around, N)))
+        r0 += t * h * w
+    rows.append(np.random.default_rng(seed).choice(N, min(n_random, N), replace=False))
+    return np.unique(np.concatenate(rows))
+
+
+@pytest.mark.parametrize("name", ["vision_batch8_bf16", "vision_16x16_f32", "prefill_t131072_video"])
 def test_vis_fused_workload(name, orc):
     w, inp = _vision_case(name)
     v = w.vision
@@ -339,8 +371,13 @@ def test_vis_fused_workload(name, orc):
     out2 = ipe.vis_pos_interp(table, v.grid_thw, v.merge)
     ipe.vis_rope2d(q2, k2, v.grid_thw, v.merge, v.theta)
     assert torch.equal(out, out2) and torch.equal(q, q2) and torch.equal(k, k2)
+    # the interpolation is checked whole (the oracle blends a video's first
+    # frame once and repeats it); the rotary on sampled rows at full size
     _interp_check(inp["table"], v.grid_thw, v.merge, v.dtype, out, orc, name)
-    _rope_check(inp["q"], v.grid_thw, v.merge, v.theta, v.dtype, q, orc, name + " q")
+    N = q.shape[0]
+    sample = _frame_sample(v.grid_thw, N, seed=5) if N > 30000 else None
+    _rope_check(inp["q"], v.grid_thw, v.merge, v.theta, v.dtype, q, orc, name + " q", sample)
+    _rope_check(inp["k"], v.grid_thw, v.merge, v.theta, v.dtype, k, orc, name + " k", sample)
 
 
 def test_interp_writes_nothing_outside_out():
@@ -370,3 +407,11 @@ def test_rejects_host_memory():
     rc = L.ipe_mrope_apply(ctypes.c_void_p(q.data_ptr()), None, ipe.IPE_BF16, 16, 24, 0, 256, 6144, 0,
                            ctypes.c_void_p(pos.data_ptr()), invh, 64, sec, 1, None)
     assert rc == ipe.IPE_EINVAL and b"not device memory" in L.ipe_last_error()
+
+
+def test_kernels_built_for_sm100a():
+    # The CUDA runtime reports the architecture of the library's kernel code
+    # as it loaded it on this device: sm_100a machine code.
+    binary, ptx = ipe.kernel_arch()
+    assert binary == 100, (binary, ptx)
+    assert torch.cuda.get_device_capability() == (10, 0)
