@@ -10,6 +10,8 @@
 // The buffer's address is looked up once per device (cudaGetSymbolAddress,
 // with that device current) by the first call made on that device; that call
 // therefore does the set-up work and should come before any stream capture.
+// Later calls check that the remembered address still names device memory of
+// that device, and look it up again after a device reset.
 // Every word of the scratch is written by the kernels before they read it, so
 // nothing has to be cleared between calls.  All calls on one device share the
 // buffer: calls whose kernels overlap in time (other streams, other host
@@ -48,6 +50,18 @@ int scratch_address(void **out)
         return ipe::set_error(IPE_ELIMIT, msg);
     }
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_addr[dev] != nullptr) {
+        // A device reset (cudaDeviceReset, or the primary context released
+        // and created again) unloads the library's module and may map it
+        // elsewhere: an address that no longer names device memory of this
+        // device is looked up again.
+        cudaPointerAttributes at;
+        if (cudaPointerGetAttributes(&at, g_scratch_addr[dev]) != cudaSuccess || at.type != cudaMemoryTypeDevice ||
+            at.device != dev) {
+            cudaGetLastError();
+            g_scratch_addr[dev] = nullptr;
+        }
+    }
     if (g_scratch_addr[dev] == nullptr) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_rope_index_scratch);

@@ -27,6 +27,9 @@ def _calls():
         "qk_norm_mrope": lambda: ipe.qk_norm_mrope(q, k, w, w, pos, inv, sec),
         "mrope_decode": lambda: ipe.mrope_decode(q, k, torch.zeros(T, dtype=torch.int32), inv),
         "mrope_rope_index": lambda: ipe.mrope_rope_index(torch.zeros(1, 16, dtype=torch.int32)),
+        "mrope_rope_index_static": lambda: ipe.mrope_rope_index_static(
+            torch.zeros(1, 16, dtype=torch.int32), None, None, None, 2, torch.zeros(3, 1, 16, dtype=torch.int32),
+            torch.zeros(1, dtype=torch.int32)),
         "vis_pos_interp": lambda: ipe.vis_pos_interp(table, [(1, 4, 4)]),
         "vis_pos_interp hf": lambda: ipe.vis_pos_interp(table, [(1, 4, 4)], rounding="hf"),
         "vis_rope2d": lambda: ipe.vis_rope2d(qv, kv, [(1, 4, 4)]),
@@ -45,3 +48,13 @@ def test_host_tensors_are_refused(name):
 def test_unknown_rounding_is_refused():
     with pytest.raises(ValueError):
         ipe._rounding("bf16")
+
+
+def test_static_scratch_size_refused_before_any_device_work():
+    # sizes whose scratch exceeds the library's fixed buffer are refused on
+    # the sizes alone, whatever the tensors are
+    B, L = 64, 1 << 20
+    ty = torch.zeros(1, 1, dtype=torch.int32).expand(B, L)
+    with pytest.raises(ipe.IpeError, match="bytes of scratch") as e:
+        ipe.mrope_rope_index_static(ty, None, None, None, 2, None, None)
+    assert e.value.status == ipe.IPE_ELIMIT

@@ -45,8 +45,12 @@ def test_static_scratch_rejects_sizes_beyond_its_buffer():
     B, L = 64, 1 << 20     # needs more scratch than the library holds
     assert ipe.rope_index_workspace_bytes(B, L) > ipe.ROPE_INDEX_STATIC_BYTES
     ty = torch.zeros(1, 1, dtype=torch.int32, device="cuda").expand(B, L)
-    # a [B, L] view without the memory: rejected on size before anything is read
-    with pytest.raises(ValueError):
+    # a [B, L] view without the memory behind it: the binding refuses it on
+    # its size alone, before it looks at layout, outputs or contents
+    with pytest.raises(ipe.IpeError, match="bytes of scratch") as e:
         ipe.mrope_rope_index_static(ty, None, None, None, 2, None, None)
+    assert e.value.status == ipe.IPE_ELIMIT
+    # and the C entry point itself, before it reads any pointer
     rc = ipe.lib().ipe_mrope_rope_index_static(None, None, 4, B, L, None, 0, None, 0, 4, 2, None, None, None)
     assert rc == ipe.IPE_ELIMIT
+    assert b"bytes of scratch" in ipe.lib().ipe_last_error()
