@@ -60,33 +60,6 @@ __global__ void vis_plan_kernel(const __grid_constant__ VisDesc<MAXIMG> d, int32
 }
 
 // -------------------------------------------------------- interpolation
-// One lane access of E table elements as raw 32-bit words, and its widening
-// to fp32 pairs (the same values load_pairs gives).
-template <typename T, int E>
-using Raw = Pack<uint32_t, E * (int)sizeof(T) / 4>;
-
-template <typename T, int E>
-__device__ __forceinline__ Raw<T, E> load_raw(const T *p)
-{
-    return ld_pack<uint32_t, E * (int)sizeof(T) / 4>(reinterpret_cast<const uint32_t *>(p));
-}
-
-template <typename T, int E>
-__device__ __forceinline__ void raw_pairs(const Raw<T, E> &w, float2 *v)
-{
-#pragma unroll
-    for (int i = 0; i < E / 2; ++i) {
-        if constexpr (sizeof(T) == 2)
-            v[i] = make_float2(__uint_as_float(w.v[i] << 16), __uint_as_float(w.v[i] & 0xffff0000u));
-        else
-            v[i] = make_float2(__uint_as_float(w.v[2 * i]), __uint_as_float(w.v[2 * i + 1]));
-    }
-}
-
-// Phase-1 entries a lane loads together: two (a third spills registers at
-// the occupancy the kernel is built for).
-constexpr int kP1 = 2;
-
 // One block = one merge-row strip (m patch rows of one image, all w columns)
 // x U consecutive 128-byte channel slices.  Bilinear interpolation is
 // separable:
@@ -149,63 +122,44 @@ __device__ __forceinline__ void interp_block(const VisDesc<MAXIMG> &d, const Int
 
     // phase 1: y-blend of the strip's m patch rows.  R entry (iy, gx) holds
     // U x NV4 float4; lane v keeps chunk u at float4 u NV4 + v + NVM q, so
-    // neighbouring lanes touch neighbouring banks in both phases.  A lane's
-    // entries (rstep apart) go kP1 at a time, with all their table loads
-    // issued before any arithmetic: one L2 round trip covers them.
+    // neighbouring lanes touch neighbouring banks in both phases.
     const T *tab_v = static_cast<const T *>(ia.table) + c0 + E * v;
     const int nrows = m * ncols;
     if (use[0]) {
         int r = threadIdx.x / NVM;
         int iy = r / ncols, gx = r - iy * ncols;
-        while (r < nrows) {
-            Raw<T, E> ra[kP1][U], rb[kP1][U];
-            float dyk[kP1];
-            int rk[kP1];
+        for (; r < nrows; r += rstep) {
+            const int2 rs = rows[iy];
+            const int y0 = rs.x & 0xffff, y1 = rs.x >> 16;
+            const float dy = __int_as_float(rs.y);
+            const float2 DY = make_float2(dy, dy);
+            const float omdy = __fsub_rn(1.f, dy);
+            const float2 OMDY = make_float2(omdy, omdy);
+            const T *ra = tab_v + (size_t)(y0 * G + gx) * C;
+            const T *rb = tab_v + (size_t)(y1 * G + gx) * C;
+            float4 *dst = R + r * NVU + v;
+            float2 a[U][E / 2], b[U][E / 2];
 #pragma unroll
-            for (int kk = 0; kk < kP1; ++kk) {
-                rk[kk] = r;
-                if (r < nrows) {
-                    const int2 rs = rows[iy];
-                    const int y0 = rs.x & 0xffff, y1 = rs.x >> 16;
-                    dyk[kk] = __int_as_float(rs.y);
-                    const T *pa = tab_v + (size_t)(y0 * G + gx) * C;
-                    const T *pb = tab_v + (size_t)(y1 * G + gx) * C;
+            for (int u = 0; u < U; ++u)
+                if (use[u]) {
+                    load_pairs<T, E>(ra + u * CS, a[u]);
+                    load_pairs<T, E>(rb + u * CS, b[u]);
+                }
 #pragma unroll
-                    for (int u = 0; u < U; ++u)
-                        if (use[u]) {
-                            ra[kk][u] = load_raw<T, E>(pa + u * CS);
-                            rb[kk][u] = load_raw<T, E>(pb + u * CS);
-                        }
-                    r += rstep;                    // next entry of this lane
-                    gx += rstep;
-                    while (gx >= ncols) {
-                        gx -= ncols;
-                        ++iy;
+            for (int u = 0; u < U; ++u)
+                if (use[u]) {
+#pragma unroll
+                    for (int q = 0; q < E / 4; ++q) {
+                        // (1-dy) a + dy b, as fma(dy, b, (1-dy) a)
+                        const float2 lo = fma2(DY, b[u][2 * q], mul2(OMDY, a[u][2 * q]));
+                        const float2 hi = fma2(DY, b[u][2 * q + 1], mul2(OMDY, a[u][2 * q + 1]));
+                        dst[u * NV4 + NVM * q] = make_float4(lo.x, lo.y, hi.x, hi.y);
                     }
                 }
-            }
-#pragma unroll
-            for (int kk = 0; kk < kP1; ++kk) {
-                if (rk[kk] >= nrows) break;
-                const float dy = dyk[kk];
-                const float2 DY = make_float2(dy, dy);
-                const float omdy = __fsub_rn(1.f, dy);
-                const float2 OMDY = make_float2(omdy, omdy);
-                float4 *dst = R + rk[kk] * NVU + v;
-#pragma unroll
-                for (int u = 0; u < U; ++u)
-                    if (use[u]) {
-                        float2 a[E / 2], b[E / 2];
-                        raw_pairs<T, E>(ra[kk][u], a);
-                        raw_pairs<T, E>(rb[kk][u], b);
-#pragma unroll
-                        for (int q = 0; q < E / 4; ++q) {
-                            // (1-dy) a + dy b, as fma(dy, b, (1-dy) a)
-                            const float2 lo = fma2(DY, b[2 * q], mul2(OMDY, a[2 * q]));
-                            const float2 hi = fma2(DY, b[2 * q + 1], mul2(OMDY, a[2 * q + 1]));
-                            dst[u * NV4 + NVM * q] = make_float4(lo.x, lo.y, hi.x, hi.y);
-                        }
-                    }
+            gx += rstep;                           // next row of this thread
+            while (gx >= ncols) {
+                gx -= ncols;
+                ++iy;
             }
         }
     }
