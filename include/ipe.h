@@ -105,7 +105,9 @@ int ipe_device_status(void *stream);
  * ipe_debug_inject -- test hook for the failure path above.  From the next
  * launch on, the producer of the TMA rotation kernels skips the loads of tile
  * `skip_tile` (-1: none), so the consumers waiting for it give up after
- * `wait_cycles` SM clock cycles (0: the default limit).  Host state, not
+ * `wait_cycles` SM clock cycles (0: the default limit); in the position-table
+ * scan (ipe_mrope_rope_index) tile `skip_tile` publishes nothing, so the
+ * tiles after it give up their look-back the same way.  Host state, not
  * thread-safe; reset with ipe_debug_inject(-1, 0).
  * ------------------------------------------------------------------------- */
 int ipe_debug_inject(int64_t skip_tile, int64_t wait_cycles);
@@ -310,8 +312,11 @@ int ipe_mrope_decode(void *q, void *k, const void *v, ipe_dtype dtype, int64_t B
  * grid's cell count (the pages' listing only fails when a sample's totals
  * differ; here every run is checked); 18 a kept slot of a type other than
  * 0 .. 3 (laid out as text); 19 a grid with t, h or w outside 1 .. 32768;
- * 20 a coordinate beyond the int32 range.  The table is written regardless.
- * Uses three kernel launches on `stream`.
+ * 20 a coordinate beyond the int32 range; 23 a tile of the scan gave up
+ * waiting (about a second) for an earlier tile's counts (the table and the
+ * deltas are then incomplete).  Otherwise the table is written regardless.
+ * Runs on `stream` as a memset of the workspace's tile flags and sample
+ * records, then one kernel: a single-pass scan over tiles of 1024 slots.
  * ------------------------------------------------------------------------- */
 int ipe_mrope_rope_index(const void *mm_token_type_ids, const void *attention_mask, int id_bytes,
                          int64_t B, int64_t L, const void *image_grid_thw, int n_images,
@@ -336,8 +341,9 @@ size_t ipe_mrope_rope_index_workspace(int64_t B, int64_t L, int n_images, int n_
  * The first call on each device looks the array's address up (with that
  * device current) and so does the set-up work: make it before any stream
  * capture.  After a device reset in the same process the next call on that
- * device finds the remembered address stale and does the set-up again.
- * Nothing in the scratch needs clearing between calls.  All calls on
+ * device finds the remembered address stale and does the set-up again.  The
+ * call itself first clears what must start at zero (a memset on `stream`),
+ * so the caller clears nothing between calls.  All calls on
  * one device share the array: calls whose kernels overlap in time (on other
  * streams or from other host threads) race.  Arguments and results as
  * ipe_mrope_rope_index without workspace / workspace_bytes.

@@ -362,6 +362,7 @@ int ipe_device_status(void *stream)
                      : v == 20 ? "position table: a coordinate beyond the int32 range"
                      : v == 21 ? "decode: seq_pos + rope delta outside [0, 2^24)"
                      : v == 22 ? "decode: a cache slot at or beyond num_slots (that write was skipped)"
+                     : v == 23 ? "position table: a tile gave up waiting for an earlier tile's counts"
                               : "unknown";
     return fail(IPE_EDEVICE, "device fault %u: %s", v, what);
 }
@@ -709,12 +710,22 @@ int ipe_mrope_rope_index(const void *mm_token_type_ids, const void *attention_ma
     a.merge = spatial_merge;
     a.pos = position_ids;
     a.deltas = rope_deltas;
-    a.agg = w;
-    a.carry = w + lay.agg;
-    a.sample = w + lay.agg + lay.carry;
-    a.img_adv = reinterpret_cast<long long *>(w + lay.agg + lay.carry + lay.sample);
-    a.vid_slices = reinterpret_cast<long long *>(w + lay.agg + lay.carry + lay.sample + lay.img_adv);
-    a.vid_adv = reinterpret_cast<long long *>(w + lay.agg + lay.carry + lay.sample + lay.img_adv + lay.vid_slices);
+    size_t off = 0;
+    auto section = [&](size_t bytes) {
+        char *p = w + off;
+        off += bytes;
+        return p;
+    };
+    a.agg = section(lay.agg);
+    a.state = section(lay.state);
+    a.flags = reinterpret_cast<unsigned *>(section(lay.flags));
+    a.sample = section(lay.sample);
+    a.ticket = reinterpret_cast<unsigned *>(section(lay.ticket));
+    a.img_adv = reinterpret_cast<long long *>(section(lay.img_adv));
+    a.vid_slices = reinterpret_cast<long long *>(section(lay.vid_slices));
+    a.vid_adv = reinterpret_cast<long long *>(section(lay.vid_adv));
+    a.wait_limit = debug_wait_limit();
+    a.skip_tile = debug_skip_tile();
     a.status = device_status_word();
     if (!a.status) return fail(IPE_ECUDA, "device status word unavailable");
     cudaError_t e = launch_rope_index(a, (cudaStream_t)stream);

@@ -150,15 +150,19 @@ struct RopeIndexArgs {
     int n_img, n_vid, merge;
     int32_t *pos;                      // [3, B, L]
     int32_t *deltas;                   // [B]
-    void *agg, *carry, *sample;        // workspace sections
+    void *agg, *state, *sample;        // workspace sections: per tile counts and states, per sample records
+    unsigned *flags;                   // [B * tiles_per_row] publication flag of each tile
+    unsigned *ticket;                  // next tile to hand out
     long long *img_adv;                // [n_img + 1] prefix of the image advances
     long long *vid_slices, *vid_adv;   // [n_vid + 1] prefixes of slices and of slice advances
     unsigned *status;
+    long long wait_limit;              // SM cycles before a look-back wait gives up
+    long long skip_tile;               // test hook: this tile never publishes (-1: none)
 };
 
 // Bytes of each workspace section for a call; the sum is the workspace size.
 struct RopeIndexLayout {
-    size_t agg, carry, sample, img_adv, vid_slices, vid_adv, total;
+    size_t agg, state, flags, sample, ticket, img_adv, vid_slices, vid_adv, total;
 };
 RopeIndexLayout rope_index_layout(long long B, long long L, int n_img, int n_vid);
 cudaError_t launch_rope_index(const RopeIndexArgs &a, cudaStream_t s);

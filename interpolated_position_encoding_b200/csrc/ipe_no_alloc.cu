@@ -12,8 +12,9 @@
 // therefore does the set-up work and should come before any stream capture.
 // Later calls check that the remembered address still names device memory of
 // that device, and look it up again after a device reset.
-// Every word of the scratch is written by the kernels before they read it, so
-// nothing has to be cleared between calls.  All calls on one device share the
+// Every call first clears what must start at zero (a memset of the tile
+// flags, the per-sample records and the tile ticket) and every other word is
+// written before it is read, so the caller clears nothing between calls.  All calls on one device share the
 // buffer: calls whose kernels overlap in time (other streams, other host
 // threads) race with each other.
 #include <cstdio>

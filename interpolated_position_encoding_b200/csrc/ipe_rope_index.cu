@@ -18,20 +18,28 @@
 //     + (advances of the sample's vision runs that start before it);
 //   * a vision run starts at that same value and its k-th slot is the k-th
 //     cell of its grid.
-// Three launches, all on the caller's stream:
-//   1. ri_tile_kernel   -- per tile of 1024 slots: kept / text counts, run
-//      starts by kind, and where the last run start lies;
-//   2. ri_carry_kernel  -- one block: the grid prefix sums, then per sample a
-//      scan over its tiles giving the state before each tile (counts, the
-//      summed advances, and the run still open at the tile's first slot);
-//   3. ri_write_kernel  -- per tile: every slot's coordinates, the tile's
-//      largest one, and in the last tile of a sample to finish, the delta.
+// One kernel on the caller's stream, after a memset of the tile flags, the
+// per-sample records and the tile ticket:
+//   ri_scan_kernel -- one block per tile of 1024 slots, in the order the
+//   blocks start (a ticket), as a single-pass scan with decoupled
+//   look-back: the block publishes its tile's own counts, looks back to the
+//   nearest earlier tile that has published its inclusive state, folds the
+//   counts of the tiles in between onto it (32 tiles per warp step),
+//   publishes its own inclusive state, then writes every slot's
+//   coordinates; the last tile of a sample to finish writes the delta.  The
+//   block with the first ticket also writes the grid prefix sums (image
+//   advances, video slices and slice advances) and flags them ready; the
+//   others wait for that flag before their write pass.
+// Every wait is bounded: a tile that gives up records code 23 in the device
+// status word and marks itself failed, so that the tiles waiting on it give
+// up at once instead of waiting out their own limit.
 // Slots of a kind the method does not define, grids that run out, and vision
 // runs whose length differs from their grid's cell count are reported through
 // the device status word (ipe_device_status); the table is still written.
 #include <climits>
 
 #include "ipe_internal.h"
+#include "ipe_rotary.cuh"
 #include "ipe_tma.cuh"
 
 namespace ipe {
@@ -42,7 +50,14 @@ constexpr unsigned kRiRunLength = 17;   // a vision run's length differs from it
 constexpr unsigned kRiBadType = 18;     // a kept slot of a type other than 0, 1, 2, 3
 constexpr unsigned kRiBadGrid = 19;     // a grid with t, h or w outside 1 .. kRiMaxSide
 constexpr unsigned kRiOverflow = 20;    // a coordinate beyond the int32 range
+constexpr unsigned kRiLookback = 23;    // a tile gave up waiting for an earlier tile's counts
 constexpr int kRiMaxSide = 1 << 15;
+
+// Publication flag of a tile (cleared by ri_init_kernel); it only grows.
+constexpr unsigned kRiNone = 0;         // nothing yet
+constexpr unsigned kRiAgg = 1;          // the tile's own counts (RiTileAgg)
+constexpr unsigned kRiPrefix = 2;       // ... and the inclusive state after it (RiState)
+constexpr unsigned kRiFailed = 3;       // the tile gave up: nothing will follow
 
 struct RiTileAgg {
     int kept, text;               // kept slots; kept text-like slots (type 0 or 3)
@@ -53,24 +68,24 @@ struct RiTileAgg {
     int ls_cls, pad;
 };
 
-struct RiCarry {
-    int k0, text0;                // kept and kept-text slots of the sample before the tile
-    int img0, vid0;               // image / video runs of the batch before the tile
-    long long vadv0;              // advances of the sample's vision runs started before the tile
-    int prev_cls;                 // class of the last kept slot before the tile (-1: none)
-    int open_k, open_grid;        // the run open at the tile's first slot: first kept index, grid
-    int own_k, own_grid;          // the tile's own last run start (read by later tiles)
-    int pad;
-    long long open_start, own_start;
+// What the tiles of the batch up to and including one tile leave for the
+// next tile.  The latest run start keeps its grid indices, not its first
+// position, so that folding tiles needs no grid look-ups.
+struct RiState {
+    int K, TX;                     // kept / kept text-like slots of the current sample
+    int IMG, VID;                  // image / video runs of the batch
+    int IMGB, VIDB;                // image / video runs of the batch before the current sample
+    int PC;                        // class of the sample's last kept slot (-1: none)
+    int open_cls;                  // class of the sample's latest run (-1: none)
+    int open_k, open_tx;           // its first kept index; the text slots of the sample before it
+    int open_ib, open_vb;          // image / video runs of the batch before it
 };
 
 struct RiSample {
-    int kept;                     // kept slots of the sample
-    int img, vid;                 // image / video runs of the batch before the sample
-    int max_pos;                  // largest coordinate written
-    unsigned done;                // tiles finished
-    int k_base, text_base;        // kept / kept-text slots of the batch before the sample
-    int pad;
+    int kept;                      // kept slots of the sample (written by its last tile)
+    int max_pos1;                  // largest coordinate written + 1 (0: none)
+    unsigned done;                 // tiles finished
+    int tail_bad1;                 // kept index + 1 of a tile-final vision slot whose run is incomplete (0: none)
 };
 
 RopeIndexLayout rope_index_layout(long long B, long long L, int n_img, int n_vid)
@@ -79,12 +94,14 @@ RopeIndexLayout rope_index_layout(long long B, long long L, int n_img, int n_vid
     const long long tiles = B * ((L + kRiTile - 1) / kRiTile);
     RopeIndexLayout l;
     l.agg = up((size_t)tiles * sizeof(RiTileAgg));
-    l.carry = up((size_t)tiles * sizeof(RiCarry));
+    l.state = up((size_t)tiles * sizeof(RiState));
+    l.flags = up((size_t)tiles * sizeof(unsigned));
     l.sample = up((size_t)B * sizeof(RiSample));
+    l.ticket = 256;
     l.img_adv = up((size_t)(n_img + 1) * sizeof(long long));
     l.vid_slices = up((size_t)(n_vid + 1) * sizeof(long long));
     l.vid_adv = up((size_t)(n_vid + 1) * sizeof(long long));
-    l.total = l.agg + l.carry + l.sample + l.img_adv + l.vid_slices + l.vid_adv;
+    l.total = l.agg + l.state + l.flags + l.sample + l.ticket + l.img_adv + l.vid_slices + l.vid_adv;
     return l;
 }
 
@@ -220,74 +237,8 @@ __device__ RiSums ri_block_exclusive(const RiSums &v, RiSums *warp_tot, RiSums &
     return ri_op(pre, exc);
 }
 
-// ------------------------------------------------------- 1. tile aggregates
+// ------------------------------------------------- grid prefix sums (init)
 
-__global__ void __launch_bounds__(kRiThreads) ri_tile_kernel(const __grid_constant__ RopeIndexArgs a)
-{
-    __shared__ RiSums warp_tot[kRiThreads / 32];
-    __shared__ RiTileAgg s;
-    const long long tile = blockIdx.x;
-    const long long b = tile / a.tiles_per_row;
-    const int local0 = threadIdx.x * kRiPer;
-    const long long l0 = (tile % a.tiles_per_row) * kRiTile + local0;
-    int cls[kRiPer];
-    bool kept[kRiPer];
-    load_slots(a, b, l0, cls, kept, false);
-    if (threadIdx.x == 0) s = RiTileAgg{0, 0, -1, -1, 0, 0, -1, 0, 0, 0, -1, 0};
-
-    // class of the last kept slot before each thread's slots
-    RiSums v{0, 0, 0, 0, 0}, tot1, tot2;
-#pragma unroll
-    for (int i = 0; i < kRiPer; ++i)
-        if (kept[i]) v.last = (local0 + i + 1) * 4 + cls[i];
-    const RiSums ex1 = ri_block_exclusive(v, warp_tot, tot1);
-    int prev = ex1.last ? (ex1.last & 3) : -1;
-
-    // counts; run starts other than at the tile's first kept slot
-    RiSums c{0, 0, 0, 0, 0};
-    int ls_off = 0, ls_text = 0, ls_img = 0, ls_vid = 0, ls_cls = -1;
-#pragma unroll
-    for (int i = 0; i < kRiPer; ++i) {
-        if (!kept[i]) continue;
-        if (prev < 0) {
-            s.first_cls = cls[i];
-        } else if (cls[i] != prev) {
-            ls_off = c.kept;
-            ls_text = c.text;
-            ls_img = c.img;
-            ls_vid = c.vid;
-            ls_cls = cls[i];
-            c.last = local0 + i + 1;
-            c.img += cls[i] == 1;
-            c.vid += cls[i] == 2;
-        }
-        c.kept += 1;
-        c.text += cls[i] == 0;
-        prev = cls[i];
-    }
-    const RiSums ex2 = ri_block_exclusive(c, warp_tot, tot2);
-    if (c.last != 0 && c.last == tot2.last) {
-        s.ls_off = ex2.kept + ls_off;
-        s.ls_text = ex2.text + ls_text;
-        s.ls_img = ex2.img + ls_img;
-        s.ls_vid = ex2.vid + ls_vid;
-        s.ls_cls = ls_cls;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        RiTileAgg o = s;
-        o.kept = tot2.kept;
-        o.text = tot2.text;
-        o.img = tot2.img;
-        o.vid = tot2.vid;
-        o.last_cls = tot1.last ? (tot1.last & 3) : -1;
-        static_cast<RiTileAgg *>(a.agg)[tile] = o;
-    }
-}
-
-// --------------------------------------------------- 2. carries (one block)
-
-constexpr int kRiCarryThreads = 1024;
 
 // Exclusive block scan of long long pairs (1024 threads); tot = the total.
 __device__ longlong2 scan_pair(longlong2 v, longlong2 *warp_tot, longlong2 &tot)
@@ -318,29 +269,12 @@ __device__ longlong2 scan_pair(longlong2 v, longlong2 *warp_tot, longlong2 &tot)
     return make_longlong2(pre.x + inc.x - v.x, pre.y + inc.y - v.y);
 }
 
-// One thread per tile of the whole batch (in chunks of the block size), two
-// block scans per chunk carried across chunks:
-//   1. the latest tile with a kept slot (key (g + 1) * 4 + class, max):
-//      the class before each tile, and whether its first kept slot starts a
-//      run (the same sample only: the key's tile must not precede the
-//      sample's first tile);
-//   2. kept, text, image-run and video-run counts (sums over the batch) and
-//      the latest tile with a run start (max).  Image / video runs of the
-//      batch are plain prefix sums (the grid sequences serve the batch in
-//      order); kept and text counts are taken relative to the sample's first
-//      tile.
-__global__ void __launch_bounds__(kRiCarryThreads) ri_carry_kernel(const __grid_constant__ RopeIndexArgs a)
+// The grid prefix sums (image advances, video slices and slice advances),
+// written by the block that takes the first ticket; the others wait for
+// `ready` before their write pass.
+__device__ void ri_grid_prefix(const RopeIndexArgs &a, longlong2 *warp_tot2)
 {
-    __shared__ longlong2 warp_tot2[kRiCarryThreads / 32];
-    __shared__ RiSums warp_tot[kRiCarryThreads / 32];
-    long long *img_adv = reinterpret_cast<long long *>(a.img_adv);
-    long long *vid_slices = reinterpret_cast<long long *>(a.vid_slices);
-    long long *vid_adv = reinterpret_cast<long long *>(a.vid_adv);
-    RiSample *smp = static_cast<RiSample *>(a.sample);
-    RiCarry *carry = static_cast<RiCarry *>(a.carry);
-    const RiTileAgg *agg = static_cast<const RiTileAgg *>(a.agg);
-
-    // grid prefix sums: image advances; video slices and slice advances
+    long long *img_adv = a.img_adv, *vid_slices = a.vid_slices, *vid_adv = a.vid_adv;
     longlong2 run{0, 0}, tot;
     for (int c0 = 0; c0 < a.n_img; c0 += blockDim.x) {
         const int j = c0 + threadIdx.x;
@@ -380,127 +314,356 @@ __global__ void __launch_bounds__(kRiCarryThreads) ri_carry_kernel(const __grid_
         vid_slices[a.n_vid] = run.x;
         vid_adv[a.n_vid] = run.y;
     }
-    if (a.tiles_per_row == 0) {          // L = 0: no tiles, every delta is 0
-        for (long long b = threadIdx.x; b < a.B; b += blockDim.x) a.deltas[b] = 0;
-        return;
-    }
-    __syncthreads();
-
-    const long long tiles = a.B * a.tiles_per_row;
-    int run_last_kept = 0;
-    RiSums run2{0, 0, 0, 0, 0};
-    for (long long c0 = 0; c0 < tiles; c0 += blockDim.x) {
-        const long long g = c0 + threadIdx.x;
-        const bool valid = g < tiles;
-        RiTileAgg r = RiTileAgg{0, 0, -1, -1, 0, 0, -1, 0, 0, 0, -1, 0};
-        if (valid) r = agg[g];
-        const long long b = valid ? g / a.tiles_per_row : 0;
-        const long long g0 = b * a.tiles_per_row;
-        const int t = (int)(g - g0);
-
-        // 1. class of the last kept slot before the tile, within the sample
-        RiSums v1{0, 0, 0, 0, r.kept > 0 ? (int)((g + 1) * 4 + r.last_cls) : 0}, tot1;
-        RiSums ex1 = ri_block_exclusive(v1, warp_tot, tot1);
-        const int key = max(ex1.last, run_last_kept);
-        run_last_kept = max(run_last_kept, tot1.last);
-        const int prev = (key > 0 && (key >> 2) - 1 >= g0) ? (key & 3) : -1;
-        const bool fs = r.kept > 0 && r.first_cls != prev;
-        const int img_t = r.img + (fs && r.first_cls == 1), vid_t = r.vid + (fs && r.first_cls == 2);
-        const bool has = r.ls_off >= 0 || fs;
-
-        // 2. counts over the batch and the latest tile with a run start
-        RiSums v2{r.kept, r.text, img_t, vid_t, has ? (int)(g + 1) : 0}, tot2;
-        const RiSums ex2 = ri_op(run2, ri_block_exclusive(v2, warp_tot, tot2));
-        run2 = ri_op(run2, tot2);
-        if (valid && t == 0) {
-            smp[b].k_base = ex2.kept;
-            smp[b].text_base = ex2.text;
-            smp[b].img = ex2.img;
-            smp[b].vid = ex2.vid;
-        }
-        __syncthreads();
-
-        int k0 = 0, text0 = 0;
-        long long base_adv = 0;
-        if (valid) {
-            const RiSample sm = smp[b];
-            k0 = ex2.kept - sm.k_base;
-            text0 = ex2.text - sm.text_base;
-            base_adv = img_adv_before(a, sm.img) + vid_adv_before(a, sm.vid);
-            // this tile's own last run start
-            int own_k = 0, own_grid = -1;
-            long long own_start = 0;
-            if (has) {
-                const bool fs_img = fs && r.first_cls == 1, fs_vid = fs && r.first_cls == 2;
-                int off = 0, text_b = 0, ib = ex2.img, vb = ex2.vid, cls = r.first_cls;
-                if (r.ls_off >= 0) {
-                    off = r.ls_off;
-                    text_b = r.ls_text;
-                    ib = ex2.img + fs_img + r.ls_img;
-                    vb = ex2.vid + fs_vid + r.ls_vid;
-                    cls = r.ls_cls;
-                }
-                own_k = k0 + off;
-                own_start = text0 + text_b + img_adv_before(a, ib) + vid_adv_before(a, vb) - base_adv;
-                own_grid = cls == 1 ? ib : cls == 2 ? vb : -1;
-            }
-            carry[g].own_k = own_k;
-            carry[g].own_grid = own_grid;
-            carry[g].own_start = own_start;
-        }
-        __syncthreads();
-        if (valid) {
-            // the run open at the tile's first slot: the latest start before it, same sample
-            const long long src = (long long)ex2.last - 1;
-            const bool open = src >= g0;
-            RiCarry &cr = carry[g];
-            cr.k0 = k0;
-            cr.text0 = text0;
-            cr.img0 = ex2.img;
-            cr.vid0 = ex2.vid;
-            cr.vadv0 = img_adv_before(a, ex2.img) + vid_adv_before(a, ex2.vid) - base_adv;
-            cr.prev_cls = prev;
-            cr.open_k = open ? carry[src].own_k : 0;
-            cr.open_grid = open ? carry[src].own_grid : -1;
-            cr.open_start = open ? carry[src].own_start : 0;
-            if (t == a.tiles_per_row - 1) {
-                smp[b].kept = k0 + r.kept;
-                smp[b].max_pos = -1;
-                smp[b].done = 0u;
-            }
-        }
-    }
 }
 
-// -------------------------------------------------------- 3. coordinates
+// ------------------------------------------------------------ look-back
 
-__global__ void __launch_bounds__(kRiThreads) ri_write_kernel(const __grid_constant__ RopeIndexArgs a)
+__device__ __forceinline__ unsigned ld_flag(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_flag(unsigned *p, unsigned v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ RiState ri_start_state()
+{
+    return RiState{0, 0, 0, 0, 0, 0, -1, -1, 0, 0, 0, 0};
+}
+
+// A sample begins: its counts, class and latest run start the empty ones.
+__device__ __forceinline__ void ri_begin_sample(RiState &x)
+{
+    x.K = 0;
+    x.TX = 0;
+    x.PC = -1;
+    x.IMGB = x.IMG;
+    x.VIDB = x.VID;
+    x.open_cls = -1;
+    x.open_k = x.open_tx = x.open_ib = x.open_vb = 0;
+}
+
+// The state after a tile from the state before it (a sample's first tile
+// already begun) and the tile's own counts.  The tile's first kept slot
+// starts a run when its class differs from the sample's last kept class.
+__device__ __forceinline__ void ri_fold(RiState &x, const RiTileAgg &r)
+{
+    const bool fs = r.kept > 0 && r.first_cls != x.PC;
+    const int fs_img = fs && r.first_cls == 1, fs_vid = fs && r.first_cls == 2;
+    if (r.ls_off >= 0) {               // the tile's latest run start lies past its first kept slot
+        x.open_k = x.K + r.ls_off;
+        x.open_tx = x.TX + r.ls_text;
+        x.open_ib = x.IMG + fs_img + r.ls_img;
+        x.open_vb = x.VID + fs_vid + r.ls_vid;
+        x.open_cls = r.ls_cls;
+    } else if (fs) {                   // ... or is its first kept slot
+        x.open_k = x.K;
+        x.open_tx = x.TX;
+        x.open_ib = x.IMG;
+        x.open_vb = x.VID;
+        x.open_cls = r.first_cls;
+    }
+    x.K += r.kept;
+    x.TX += r.text;
+    x.IMG += r.img + fs_img;
+    x.VID += r.vid + fs_vid;
+    if (r.kept > 0) x.PC = r.last_cls;
+}
+
+__device__ __forceinline__ RiTileAgg ld_agg(const RiTileAgg *p)
+{
+    const int4 *q = reinterpret_cast<const int4 *>(p);
+    const int4 u = __ldcg(q), v = __ldcg(q + 1), w = __ldcg(q + 2);
+    return RiTileAgg{u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w, w.x, w.y, w.z, w.w};
+}
+
+__device__ __forceinline__ RiState ld_state(const RiState *p)
+{
+    const int4 *q = reinterpret_cast<const int4 *>(p);
+    const int4 u = __ldcg(q), v = __ldcg(q + 1), w = __ldcg(q + 2);
+    return RiState{u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w, w.x, w.y, w.z, w.w};
+}
+
+__device__ __forceinline__ int warp_incl_sum(int v)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, v, d);
+        if (lane >= d) v += t;
+    }
+    return v;
+}
+
+__device__ __forceinline__ int warp_incl_max(int v)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, v, d);
+        if (lane >= d) v = max(v, t);
+    }
+    return v;
+}
+
+// Warp: fold the counts of tiles c .. c + n - 1 (1 <= n <= 32, lane i holds
+// tile c + i) onto x, the state after tile c - 1 (the same in every lane).
+// The folds of ri_fold, done for the window at once:
+//   * the class before each tile: the latest earlier tile of the window with
+//     a kept slot in the same sample (a max-scan of keys), else x's class,
+//     else none when the tile's sample starts inside the window;
+//   * whether each tile's first kept slot starts a run, hence its image /
+//     video run starts;
+//   * kept and text counts, reset at sample starts, and the batch's image
+//     and video run counts (sum-scans);
+//   * the latest run start of the last tile's sample (a max-scan).
+__device__ void ri_fold_window(const RopeIndexArgs &a, RiState &x, long long c, int n)
+{
+    const unsigned full = 0xffffffffu;
+    const int lane = threadIdx.x & 31;
+    const bool valid = lane < n;
+    const RiTileAgg r = valid ? ld_agg(static_cast<const RiTileAgg *>(a.agg) + c + lane)
+                              : RiTileAgg{0, 0, -1, -1, 0, 0, -1, 0, 0, 0, -1, 0};
+    const bool start = valid && (c + lane) % a.tiles_per_row == 0;
+    const int ss = warp_incl_max(start ? lane : -1);           // this tile's sample start in the window (-1: before it)
+    const int kinc = warp_incl_max(valid && r.kept > 0 ? (lane + 1) * 4 + r.last_cls : 0);
+    int kex = __shfl_up_sync(full, kinc, 1);
+    if (lane == 0) kex = 0;
+    const int prev = (kex > 0 && (kex >> 2) - 1 >= ss) ? (kex & 3) : (ss < 0 ? x.PC : -1);
+    const bool fs = valid && r.kept > 0 && r.first_cls != prev;
+    const int fi = fs && r.first_cls == 1, fv = fs && r.first_cls == 2;
+    const int img_t = r.img + fi, vid_t = r.vid + fv;
+    const int pk = warp_incl_sum(r.kept) - r.kept, ptx = warp_incl_sum(r.text) - r.text;
+    const int pimg = warp_incl_sum(img_t) - img_t, pvid = warp_incl_sum(vid_t) - vid_t;
+    const int src = ss < 0 ? 0 : ss;
+    const int pk_s = __shfl_sync(full, pk, src), ptx_s = __shfl_sync(full, ptx, src);
+    const int pimg_s = __shfl_sync(full, pimg, src), pvid_s = __shfl_sync(full, pvid, src);
+    // values before this lane's tile
+    const int K0 = ss < 0 ? x.K + pk : pk - pk_s;
+    const int TX0 = ss < 0 ? x.TX + ptx : ptx - ptx_s;
+    const int IMG0 = x.IMG + pimg, VID0 = x.VID + pvid;
+    const int IMGB = ss < 0 ? x.IMGB : x.IMG + pimg_s, VIDB = ss < 0 ? x.VIDB : x.VID + pvid_s;
+    // this tile's latest run start
+    int ok = 0, otx = 0, oib = 0, ovb = 0, ocls = -1;
+    if (valid && r.ls_off >= 0) {
+        ok = K0 + r.ls_off;
+        otx = TX0 + r.ls_text;
+        oib = IMG0 + fi + r.ls_img;
+        ovb = VID0 + fv + r.ls_vid;
+        ocls = r.ls_cls;
+    } else if (fs) {
+        ok = K0;
+        otx = TX0;
+        oib = IMG0;
+        ovb = VID0;
+        ocls = r.first_cls;
+    }
+    const int hj = warp_incl_max(ocls >= 0 ? lane : -1);
+    // the state after the window's last tile
+    const int L = n - 1;
+    RiState y;
+    y.K = __shfl_sync(full, K0 + r.kept, L);
+    y.TX = __shfl_sync(full, TX0 + r.text, L);
+    y.IMG = __shfl_sync(full, IMG0 + img_t, L);
+    y.VID = __shfl_sync(full, VID0 + vid_t, L);
+    y.IMGB = __shfl_sync(full, IMGB, L);
+    y.VIDB = __shfl_sync(full, VIDB, L);
+    y.PC = __shfl_sync(full, r.kept > 0 ? r.last_cls : prev, L);
+    const int ssL = __shfl_sync(full, ss, L), hL = __shfl_sync(full, hj, L);
+    const int hs = hL < 0 ? 0 : hL;
+    const int ok_h = __shfl_sync(full, ok, hs), otx_h = __shfl_sync(full, otx, hs);
+    const int oib_h = __shfl_sync(full, oib, hs), ovb_h = __shfl_sync(full, ovb, hs);
+    const int ocls_h = __shfl_sync(full, ocls, hs);
+    if (hL >= 0 && hL >= ssL) {                    // a run starts in the last tile's sample, in the window
+        y.open_k = ok_h;
+        y.open_tx = otx_h;
+        y.open_ib = oib_h;
+        y.open_vb = ovb_h;
+        y.open_cls = ocls_h;
+    } else if (ssL < 0) {                          // the sample continues from x with no new run
+        y.open_k = x.open_k;
+        y.open_tx = x.open_tx;
+        y.open_ib = x.open_ib;
+        y.open_vb = x.open_vb;
+        y.open_cls = x.open_cls;
+    } else {                                       // the sample started in the window with no run yet
+        y.open_k = y.open_tx = y.open_ib = y.open_vb = 0;
+        y.open_cls = -1;
+    }
+    x = y;
+}
+
+// Warp 0: the state before tile `tile` (of the whole batch so far; the
+// caller begins the sample when the tile is a sample's first).  Looks back
+// 32 tiles at a time for the nearest tile with its inclusive state
+// published, every tile in between having published its counts, then folds
+// those counts onto it, 32 tiles per step.  False when a wait ran out or an
+// earlier tile failed.
+__device__ bool ri_look_back(const RopeIndexArgs &a, long long tile, RiState &out)
+{
+    const int lane = threadIdx.x & 31;
+    const RiState *st = static_cast<const RiState *>(a.state);
+    const long long t0 = clock64();
+    long long hi = tile - 1, p = -1;   // p: the tile whose state starts the fold (-1: the batch start)
+    while (hi >= 0) {
+        const long long j = hi - lane;
+        unsigned f = kRiPrefix;        // before the batch start: the empty state
+        if (j >= 0) {
+            f = ld_flag(a.flags + j);
+            while (f == kRiNone && clock64() - t0 <= a.wait_limit) f = ld_flag(a.flags + j);
+        }
+        // lane l reads tile hi - l: lanes below the nearest prefix are the
+        // tiles after it, whose counts the fold needs
+        const unsigned bad = __ballot_sync(0xffffffffu, f == kRiNone || f == kRiFailed);
+        const unsigned pre = __ballot_sync(0xffffffffu, f == kRiPrefix);
+        if (pre) {
+            const int l = __ffs(pre) - 1;
+            if (bad & ((1u << l) - 1u)) return false;
+            p = hi - l;
+            break;
+        }
+        if (bad) return false;
+        hi -= 32;
+    }
+    // every lane reads data that other lanes saw published
+    __syncwarp();
+    __threadfence();
+    RiState x = p >= 0 ? ld_state(st + p) : ri_start_state();
+    for (long long c = p + 1; c < tile; c += 32) ri_fold_window(a, x, c, (int)min(32LL, tile - c));
+    out = x;
+    return true;
+}
+
+// ------------------------------------------------------------- the scan
+
+__global__ void __launch_bounds__(kRiThreads) ri_scan_kernel(const __grid_constant__ RopeIndexArgs a)
 {
     __shared__ RiSums warp_tot[kRiThreads / 32];
+    __shared__ RiTileAgg s;
+    __shared__ RiState before;
+    __shared__ long long tile_sh;
+    __shared__ int ok_sh;
     __shared__ int rec_k[kRiTile], rec_grid[kRiTile], rec_cls[kRiTile];
     __shared__ long long rec_start[kRiTile];
     __shared__ int warp_max[kRiThreads / 32];
-    const long long tile = blockIdx.x;
+
+    // tiles in the order the blocks start, so every tile waited on is running
+    __shared__ longlong2 warp_tot2[kRiThreads / 32];
+    if (threadIdx.x == 0) tile_sh = (long long)atomicAdd(a.ticket, 1u);
+    __syncthreads();
+    const long long tile = tile_sh;
+    if (tile == 0) {
+        ri_grid_prefix(a, warp_tot2);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            st_flag(a.ticket + 1, 1u);
+        }
+    }
+    if (tile == a.skip_tile) return;   // test hook: this tile never publishes anything
     const long long b = tile / a.tiles_per_row;
+    const int t_in_row = (int)(tile % a.tiles_per_row);
     const int local0 = threadIdx.x * kRiPer;
-    const long long l0 = (tile % a.tiles_per_row) * kRiTile + local0;
-    const RiCarry C = static_cast<const RiCarry *>(a.carry)[tile];
-    RiSample *smp = static_cast<RiSample *>(a.sample);
-    const int sample_kept = smp[b].kept;
-    const long long plane = a.B * a.L;
+    const long long l0 = (long long)t_in_row * kRiTile + local0;
     int cls[kRiPer];
     bool kept[kRiPer];
     load_slots(a, b, l0, cls, kept, true);
 
-    RiSums v{0, 0, 0, 0, 0}, tot;
+    // ---- the tile's own counts, nothing before it known
+    if (threadIdx.x == 0) s = RiTileAgg{0, 0, -1, -1, 0, 0, -1, 0, 0, 0, -1, 0};
+    RiSums v{0, 0, 0, 0, 0}, tot1, tot2;
 #pragma unroll
     for (int i = 0; i < kRiPer; ++i)
         if (kept[i]) v.last = (local0 + i + 1) * 4 + cls[i];
-    const RiSums ex1 = ri_block_exclusive(v, warp_tot, tot);
-    const int prev0 = ex1.last ? (ex1.last & 3) : C.prev_cls;
+    const RiSums ex1 = ri_block_exclusive(v, warp_tot, tot1);
+    const int prev_in_tile = ex1.last ? (ex1.last & 3) : -1;   // last kept class before this thread's slots
+    {
+        RiSums c{0, 0, 0, 0, 0};
+        int prev = prev_in_tile;
+        int ls_off = 0, ls_text = 0, ls_img = 0, ls_vid = 0, ls_cls = -1;
+#pragma unroll
+        for (int i = 0; i < kRiPer; ++i) {
+            if (!kept[i]) continue;
+            if (prev < 0) {
+                s.first_cls = cls[i];
+            } else if (cls[i] != prev) {
+                ls_off = c.kept;
+                ls_text = c.text;
+                ls_img = c.img;
+                ls_vid = c.vid;
+                ls_cls = cls[i];
+                c.last = local0 + i + 1;
+                c.img += cls[i] == 1;
+                c.vid += cls[i] == 2;
+            }
+            c.kept += 1;
+            c.text += cls[i] == 0;
+            prev = cls[i];
+        }
+        const RiSums ex2 = ri_block_exclusive(c, warp_tot, tot2);
+        if (c.last != 0 && c.last == tot2.last) {
+            s.ls_off = ex2.kept + ls_off;
+            s.ls_text = ex2.text + ls_text;
+            s.ls_img = ex2.img + ls_img;
+            s.ls_vid = ex2.vid + ls_vid;
+            s.ls_cls = ls_cls;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        s.kept = tot2.kept;
+        s.text = tot2.text;
+        s.img = tot2.img;
+        s.vid = tot2.vid;
+        s.last_cls = tot1.last ? (tot1.last & 3) : -1;
+        static_cast<RiTileAgg *>(a.agg)[tile] = s;
+        st_flag(a.flags + tile, kRiAgg);
+    }
 
-    // counts and run starts, the tile's first kept slot included
-    RiSums c{0, 0, 0, 0, 0};
+    // ---- the state before the tile, then the state after it
+    if (threadIdx.x < 32) {
+        RiState x;
+        const bool ok = ri_look_back(a, tile, x);
+        if (threadIdx.x == 0) {
+            ok_sh = ok;
+            if (ok) {
+                if (t_in_row == 0) ri_begin_sample(x);
+                before = x;
+                ri_fold(x, s);
+                static_cast<RiState *>(a.state)[tile] = x;
+                st_flag(a.flags + tile, kRiPrefix);
+                if (t_in_row == a.tiles_per_row - 1) static_cast<RiSample *>(a.sample)[b].kept = x.K;
+            } else {
+                record_fault(a.status, kRiLookback);
+                st_flag(a.flags + tile, kRiFailed);
+            }
+        }
+    }
+    if (threadIdx.x == 0 && ok_sh) {
+        // the grid prefix sums of the first tile's block
+        const long long t0 = clock64();
+        unsigned r = ld_flag(a.ticket + 1);
+        while (r == 0u && clock64() - t0 <= a.wait_limit) r = ld_flag(a.ticket + 1);
+        if (r == 0u) {
+            record_fault(a.status, kRiLookback);
+            ok_sh = 0;
+        }
+    }
+    __syncthreads();
+    if (!ok_sh) return;
+    const RiState X = before;
+    RiSample *smp = static_cast<RiSample *>(a.sample);
+    const long long plane = a.B * a.L;
+    const long long base_adv = img_adv_before(a, X.IMGB) + vid_adv_before(a, X.VIDB);
+    const long long vadv0 = img_adv_before(a, X.IMG) + vid_adv_before(a, X.VID) - base_adv;
+
+    // ---- counts and run starts with the class before the tile known
+    const int prev0 = ex1.last ? (ex1.last & 3) : X.PC;
+    RiSums c{0, 0, 0, 0, 0}, tot;
     int prev = prev0;
 #pragma unroll
     for (int i = 0; i < kRiPer; ++i) {
@@ -517,8 +680,8 @@ __global__ void __launch_bounds__(kRiThreads) ri_write_kernel(const __grid_const
     const RiSums ex = ri_block_exclusive(c, warp_tot, tot);
 
     // pass 1: records of the runs starting here; text slots
-    long long vadv = C.vadv0 + img_adv_before(a, C.img0 + ex.img) - img_adv_before(a, C.img0) +
-                     vid_adv_before(a, C.vid0 + ex.vid) - vid_adv_before(a, C.vid0);
+    long long vadv = vadv0 + img_adv_before(a, X.IMG + ex.img) - img_adv_before(a, X.IMG) +
+                     vid_adv_before(a, X.VID + ex.vid) - vid_adv_before(a, X.VID);
     int kept_b = ex.kept, text_b = ex.text, img_b = ex.img, vid_b = ex.vid;
     long long mx = -1;
     prev = prev0;
@@ -533,15 +696,15 @@ __global__ void __launch_bounds__(kRiThreads) ri_write_kernel(const __grid_const
             a.pos[2 * plane + at] = 0;
             continue;
         }
-        const long long here = C.text0 + text_b + vadv;
+        const long long here = X.TX + text_b + vadv;
         if (cls[i] != prev) {
             const int r = local0 + i;
-            rec_k[r] = C.k0 + kept_b;
+            rec_k[r] = X.K + kept_b;
             rec_start[r] = here;
             rec_cls[r] = cls[i];
             rec_grid[r] = -1;
             if (cls[i] != 0) {
-                const long long g = cls[i] == 1 ? (long long)C.img0 + img_b : (long long)C.vid0 + vid_b;
+                const long long g = cls[i] == 1 ? (long long)X.IMG + img_b : (long long)X.VID + vid_b;
                 RiGrid gr;
                 rec_grid[r] = (int)g;
                 if (run_grid(a, cls[i], g, gr)) vadv += gr.adv;
@@ -563,9 +726,13 @@ __global__ void __launch_bounds__(kRiThreads) ri_write_kernel(const __grid_const
     }
     __syncthreads();
 
-    // pass 2: vision slots from their run's record
-    int rk = C.open_k, rgrid = C.open_grid, rcls = C.prev_cls > 0 ? C.prev_cls : 0;
-    long long rstart = C.open_start;
+    // pass 2: vision slots from their run's record (or the run open at the
+    // tile's first slot)
+    int rk = X.open_cls >= 0 ? X.open_k : 0;
+    int rgrid = X.open_cls == 1 ? X.open_ib : X.open_cls == 2 ? X.open_vb : -1;
+    int rcls = X.PC > 0 ? X.PC : 0;
+    long long rstart = X.open_cls >= 0 ? X.open_tx + img_adv_before(a, X.open_ib) + vid_adv_before(a, X.open_vb) - base_adv
+                                       : 0;
     if (ex.last > 0) {
         const int r = ex.last - 1;
         rk = rec_k[r];
@@ -575,6 +742,7 @@ __global__ void __launch_bounds__(kRiThreads) ri_write_kernel(const __grid_const
     }
     RiGrid gr{0, 0, 0, 0};
     bool have = rcls != 0 && run_grid(a, rcls, rgrid, gr);
+    const int tile_last = tot1.last ? (tot1.last >> 2) - 1 : -1;   // local index of the tile's last kept slot
     kept_b = ex.kept;
     prev = prev0;
 #pragma unroll
@@ -582,7 +750,7 @@ __global__ void __launch_bounds__(kRiThreads) ri_write_kernel(const __grid_const
         const long long l = l0 + i;
         if (l >= a.L) break;
         if (!kept[i]) continue;
-        const int k = C.k0 + kept_b;
+        const int k = X.K + kept_b;
         if (cls[i] != prev) {
             // the run that ends here must have filled its grid
             if (rcls != 0 && (!have || (long long)(k - rk) != (long long)gr.t * gr.h * gr.w))
@@ -609,7 +777,9 @@ __global__ void __launch_bounds__(kRiThreads) ri_write_kernel(const __grid_const
             } else if (have) {
                 record_fault(a.status, kRiRunLength);
             }
-            if (have && k == sample_kept - 1 && off + 1 != cells) record_fault(a.status, kRiRunLength);
+            // a run still short of its grid at the tile's last kept slot: a
+            // fault if that slot turns out to be the sample's last
+            if (have && local0 + i == tile_last && off + 1 != cells) atomicMax(&smp[b].tail_bad1, k + 1);
             const long long pt = rstart + tt, ph = rstart + row, pw = rstart + col;
             const long long top = max(pt, max(ph, pw));
             if (top > INT_MAX) record_fault(a.status, kRiOverflow);
@@ -622,7 +792,7 @@ __global__ void __launch_bounds__(kRiThreads) ri_write_kernel(const __grid_const
         prev = cls[i];
     }
 
-    // the tile's largest coordinate; the sample's last tile writes the delta
+    // the tile's largest coordinate; the sample's last tile to finish writes the delta
     int m = (int)mx;
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, d));
@@ -630,12 +800,15 @@ __global__ void __launch_bounds__(kRiThreads) ri_write_kernel(const __grid_const
     __syncthreads();
     if (threadIdx.x == 0) {
         for (int w = 1; w < kRiThreads / 32; ++w) m = max(m, warp_max[w]);
-        if (m >= 0) atomicMax(&smp[b].max_pos, m);
+        if (m >= 0) atomicMax(&smp[b].max_pos1, m + 1);
         __threadfence();
         if (atomicAdd(&smp[b].done, 1u) == (unsigned)a.tiles_per_row - 1) {
             __threadfence();
-            const int top = atomicAdd(&smp[b].max_pos, 0);
-            a.deltas[b] = sample_kept > 0 ? top + 1 - sample_kept : 0;
+            const int kept_n = __ldcg(&smp[b].kept);
+            const int top = atomicAdd(&smp[b].max_pos1, 0) - 1;
+            const int bad = atomicAdd(&smp[b].tail_bad1, 0) - 1;
+            if (kept_n > 0 && bad == kept_n - 1) record_fault(a.status, kRiRunLength);
+            a.deltas[b] = kept_n > 0 ? top + 1 - kept_n : 0;
         }
     }
 }
@@ -643,9 +816,12 @@ __global__ void __launch_bounds__(kRiThreads) ri_write_kernel(const __grid_const
 cudaError_t launch_rope_index(const RopeIndexArgs &a, cudaStream_t s)
 {
     const long long tiles = a.B * a.tiles_per_row;
-    if (tiles > 0) ri_tile_kernel<<<(unsigned)tiles, kRiThreads, 0, s>>>(a);
-    ri_carry_kernel<<<1, kRiCarryThreads, 0, s>>>(a);
-    if (tiles > 0) ri_write_kernel<<<(unsigned)tiles, kRiThreads, 0, s>>>(a);
+    if (tiles == 0) return cudaMemsetAsync(a.deltas, 0, (size_t)a.B * sizeof(int32_t), s);   // L = 0
+    // flags, sample records and ticket are one contiguous run of the workspace
+    const size_t zero = (size_t)(reinterpret_cast<char *>(a.ticket) - reinterpret_cast<char *>(a.flags)) + 256;
+    cudaError_t e = cudaMemsetAsync(a.flags, 0, zero, s);
+    if (e != cudaSuccess) return e;
+    ri_scan_kernel<<<(unsigned)tiles, kRiThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -1,8 +1,9 @@
-"""Failure path of the TMA-fed kernels: a bounded wait that runs out.
+"""Failure path of the kernels that wait: a bounded wait that runs out.
 
-The test hook makes the producer skip one tile's loads, so the consumers
-waiting for that stage give up after a short limit, record a fault in the
-device status word and return.  Nothing faults or hangs: the host reads the
+The test hook makes the producer of a TMA-fed kernel skip one tile's loads
+(or one tile of the position-table scan publish nothing), so the warps
+waiting for it give up after a short limit, record a fault in the device
+status word and return.  Nothing faults or hangs: the host reads the
 status, the context stays usable, and the next launch is correct.
 """
 import numpy as np
@@ -72,3 +73,26 @@ def test_skipped_tile_times_out_and_recovers(path):
     ipe.device_status()
     assert torch.equal(good_a, ref_a) and torch.equal(good_b, ref_b)
     assert not torch.equal(bad_a, ref_a) or not torch.equal(bad_b, ref_b)
+
+
+def test_position_table_look_back_times_out_and_recovers():
+    # the position-table scan: tile 1 publishes nothing, so the tiles after it
+    # give up their look-back, report code 23 and mark themselves failed
+    L = 3 * 1024 + 17
+    types = torch.zeros(1, L, dtype=torch.int32, device="cuda")
+    types[0, 1500:1524] = 1                         # a (1, 8, 12) image across tiles 1 and 2
+    img = torch.tensor([[1, 8, 12]], dtype=torch.int32, device="cuda")
+    ref_pos, ref_d = ipe.mrope_rope_index(types, img, None, None, 2)
+    ipe.device_status()
+    ipe.debug_inject(1, SHORT_WAIT)
+    try:
+        ipe.mrope_rope_index(types, img, None, None, 2)
+        with pytest.raises(ipe.IpeError) as err:
+            ipe.device_status()
+        assert err.value.status == ipe.IPE_EDEVICE and "device fault 23:" in str(err.value)
+    finally:
+        ipe.debug_inject(-1, 0)
+    ipe.device_status()
+    pos, d = ipe.mrope_rope_index(types, img, None, None, 2)
+    ipe.device_status()
+    assert torch.equal(pos, ref_pos) and torch.equal(d, ref_d)
