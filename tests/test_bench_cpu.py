@@ -58,3 +58,17 @@ def test_kernel_source_hash_covers_every_kernel_file(tmp_path, monkeypatch):
     h0 = bench.kernel_source_sha()
     (csrc / "b.cuh").write_text("two!")
     assert bench.kernel_source_sha() != h0
+
+
+def test_cpu_baseline_runs_on_every_core():
+    # the oracle baseline: one single-threaded oracle process per host core
+    # (bounded by memory), each on its own slice, and the single-thread figure
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as wl
+    d = bench.cpu_baseline(wl.WORKLOADS[bench.WORKLOAD], rounds=1)
+    n, cores = bench.oracle_workers()
+    assert d["kind"] == "oracle" and d["cores"] == n and d["host_cores"] == cores
+    assert d["single_thread"]["cores"] == 1 and d["single_thread"]["value"] > 0
+    if n >= 2:
+        assert d["value"] > d["single_thread"]["value"]

@@ -415,3 +415,26 @@ def test_kernels_built_for_sm100a():
     binary, ptx = ipe.kernel_arch()
     assert binary == 100, (binary, ptx)
     assert torch.cuda.get_device_capability() == (10, 0)
+
+
+@pytest.mark.parametrize("grids,merge,C,heads,D", [
+    ([(1, 48, 48)], 2, 64, 2, 72), ([(1, 1, 5), (1, 3, 1)], 1, 1152, 3, 16), ([(1, 6, 9)], 3, 100, 1, 12),
+    ([(2, 4, 6), (1, 2, 2), (3, 6, 4)], 2, 1000, 4, 72), ([(1, 2, 4)] * 20, 2, 132, 2, 8),
+    ([(1, 2, 1030), (1, 4, 4)], 2, 64, 1, 72), ([(1, 24, 4)] * 100, 2, 1000, 2, 16)])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_vis_fused_edges(grids, merge, C, heads, D, dtype, orc):
+    # the one-call entry on ragged shapes: the same interpolation and rotary
+    # as the separate calls, bit for bit, and the oracle's values
+    rng = GEN(C * 3 + D)
+    gen = wl.normal_bf16 if dtype == "bf16" else wl.normal_f32
+    N = sum(t * h * w for t, h, w in grids)
+    table = gen(rng, (48 * 48, C), 0.02)
+    q, k = gen(rng, (N, heads, D)), gen(rng, (N, heads, D))
+    gt, gq, gk = to_gpu(table, dtype), to_gpu(q, dtype), to_gpu(k, dtype)
+    q2, k2 = gq.clone(), gk.clone()
+    out, _, _ = ipe.vis_pos_interp_rope2d(gt, grids, gq, gk, merge, 1e4)
+    out2 = ipe.vis_pos_interp(gt, grids, merge)
+    ipe.vis_rope2d(q2, k2, grids, merge, 1e4)
+    assert torch.equal(out, out2) and torch.equal(gq, q2) and torch.equal(gk, k2)
+    _interp_check(table, grids, merge, dtype, out, orc, f"{grids} {dtype}")
+    _rope_check(q, grids, merge, 1e4, dtype, gq, orc, f"{grids} {dtype} q")
