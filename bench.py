@@ -137,8 +137,8 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def dram_traffic(kernel):
-    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or
+def traffic_entry(kernel):
+    """The committed ncu summary of `kernel` (profiles/dram_traffic.json), or
     None when the kernels changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
@@ -148,7 +148,14 @@ def dram_traffic(kernel):
     e = d.get(WORKLOAD, {}).get(kernel)
     if not e or e.get("source_sha") != kernel_source_sha():
         return None
-    return e.get("bytes_per_launch")
+    return e
+
+
+def dram_traffic(kernel):
+    """Per-launch DRAM bytes (read + write) of `kernel` from the committed
+    ncu summary, or None when the kernels changed since it was taken."""
+    e = traffic_entry(kernel)
+    return None if e is None else e.get("bytes_per_launch")
 
 
 class ClockSampler:
@@ -683,11 +690,18 @@ def main():
     kernels = {n: {"ms": kernel_ms[n], "alg_bytes": alg[n], "gbs": alg[n] / kernel_ms[n] / 1e6,
                    "frac": alg[n] / kernel_ms[n] / 1e6 / peak} for n in names}
     dom = max(names, key=lambda n: kernel_ms[n])
+    tr = traffic_entry(dom) if args.scale_down == 1 else None
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak, "unit": "GB/s",
-                "frac": kernels[dom]["frac"], "traffic": dram_traffic(dom) if args.scale_down == 1 else None,
+                "frac": kernels[dom]["frac"], "traffic": None if tr is None else tr.get("bytes_per_launch"),
                 "alg_bytes": alg[dom],
                 "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured" else
                 "fallback 6650 GB/s"}
+    if tr is not None and "l2_write_mb_full" in tr:
+        roofline["traffic_dram_read"] = int(round(tr["dram_read_mb_full"] * 1e6))
+        roofline["traffic_l2_write"] = int(round(tr["l2_write_mb_full"] * 1e6))
+        roofline["traffic_note"] = ("traffic = ncu DRAM read + write per launch (1/4-size capture x 4); the DRAM writes "
+                                    "undercount (lines still dirty in L2 when the kernel ends); traffic_l2_write = L2 "
+                                    "write sectors x 32 B / 1.5 (calibrated on a plain fill), the bytes written")
 
     # ---- side measurements (after the timed region)
     extras = {}
