@@ -16,16 +16,17 @@
 //
 // The default kernel (vis_interp_kernel) evaluates the separable form in
 // fp32 with one rounding; this one evaluates the four-corner sum directly.
-// A block takes one merge-row strip of an image, 32 chunks of 16 bytes of
-// the channels and a range of the video's frames:
-//   * set-up: each patch of the strip gets its four corner rows and four
+// A block takes a range of the patches of one merge-row strip of an image
+// and 32 chunks of 16 bytes of the channels:
+//   * set-up: each patch of its range gets its four corner rows and four
 //     weights (rounded to the dtype) once, in shared memory;
 //   * each warp then takes two output rows at a time (eight 16-byte table
 //     loads in flight per lane), forms the four products and the
 //     left-to-right sums, and writes each result chunk to every frame of
-//     its range (frames repeat frame 0).
-// The frame ranges split a video over more blocks, so that a request of few
-// strips still puts about four blocks on every SM.  For bf16 the products
+//     the video (frames repeat frame 0).
+// The patch ranges split a strip over more blocks, so that a request of few
+// strips still puts about four blocks on every SM, while every block still
+// reads each table value once for all of a video's frames.  For bf16 the products
 // and sums run as packed bf16x2 operations, which round exactly where the
 // fp32-then-round steps above do (mul_bf16x2 / add_bf16x2).
 #include "ipe_internal.h"
@@ -119,20 +120,21 @@ __device__ __forceinline__ uint4 hf_blend(const uint4 (&c)[4], const uint4 &w)
 
 template <typename T>
 __global__ void __launch_bounds__(32 * kHfWarps) vis_interp_hf_kernel(const __grid_constant__ VisDesc<1024> d,
-                                                                      const __grid_constant__ InterpArgs ia, int fpb)
+                                                                      const __grid_constant__ InterpArgs ia, int parts)
 {
     __shared__ HfPatch plan[kHfPlanCache];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int s = blockIdx.x;
     const VisImage im = d.img[find_image_of_strip(d, s)];
-    const int f0 = blockIdx.z * fpb, f1 = min(im.t, f0 + fpb);
-    if (f0 >= f1) return;                             // this image has fewer frames (whole block: no barrier yet)
     const int m = d.merge, G = d.grid_side, h = im.h, w = im.w;
     const int sl = s - im.strip0;                     // merge-row strip within the frame
     const int nq = m * w;                             // patches of the strip
-    const bool cached = nq <= kHfPlanCache;
+    const int per = (nq + parts - 1) / parts;         // this block's patches: [qa, qb)
+    const int qa = blockIdx.z * per, qb = min(nq, qa + per);
+    if (qa >= qb) return;                             // a narrow strip has fewer parts (whole block: no barrier yet)
+    const bool cached = qb - qa <= kHfPlanCache;
     if (cached)
-        for (int q = threadIdx.x; q < nq; q += blockDim.x) plan[q] = hf_patch<T>(q, sl, m, h, w, G);
+        for (int q = qa + threadIdx.x; q < qb; q += blockDim.x) plan[q - qa] = hf_patch<T>(q, sl, m, h, w, G);
     __syncthreads();
     constexpr int EC = 16 / sizeof(T);
     const int chunks = ia.hidden / EC;
@@ -143,11 +145,11 @@ __global__ void __launch_bounds__(32 * kHfWarps) vis_interp_hf_kernel(const __gr
     uint4 *out = reinterpret_cast<uint4 *>(ia.out) + ch;
     const long long rstride = chunks;                 // uint4 per table / output row
     const long long row0 = im.row0 + (long long)sl * nq;
-    for (int q = warp; q < nq; q += 2 * kHfWarps) {
-        const int qb = q + kHfWarps;
-        const bool two = qb < nq;
-        const HfPatch pa = cached ? plan[q] : hf_patch<T>(q, sl, m, h, w, G);
-        const HfPatch pb = two ? (cached ? plan[qb] : hf_patch<T>(qb, sl, m, h, w, G)) : pa;
+    for (int q = qa + warp; q < qb; q += 2 * kHfWarps) {
+        const int q2 = q + kHfWarps;
+        const bool two = q2 < qb;
+        const HfPatch pa = cached ? plan[q - qa] : hf_patch<T>(q, sl, m, h, w, G);
+        const HfPatch pb = two ? (cached ? plan[q2 - qa] : hf_patch<T>(q2, sl, m, h, w, G)) : pa;
         uint4 ca[4], cb[4];
         const int ia4[4] = {pa.idx.x, pa.idx.y, pa.idx.z, pa.idx.w};
         const int ib4[4] = {pb.idx.x, pb.idx.y, pb.idx.z, pb.idx.w};
@@ -157,37 +159,34 @@ __global__ void __launch_bounds__(32 * kHfWarps) vis_interp_hf_kernel(const __gr
         for (int k = 0; k < 4; ++k) cb[k] = tab[ib4[k] * rstride];
         const uint4 oa = hf_blend<T>(ca, pa.w), ob = hf_blend<T>(cb, pb.w);
 #pragma unroll 1
-        for (int f = f0; f < f1; ++f) {
+        for (int f = 0; f < im.t; ++f) {
             out[(row0 + q + f * hw) * rstride] = oa;
-            if (two) out[(row0 + qb + f * hw) * rstride] = ob;
+            if (two) out[(row0 + q2 + f * hw) * rstride] = ob;
         }
     }
 }
 
-// Frames per block: enough blocks for about four per SM, each block taking
-// a whole range of a video's frames.
-static int hf_frames_per_block(const VisDesc<1024> &d, long long blocks_xy)
+// Parts per strip: enough blocks for about four per SM.
+static int hf_parts(const VisDesc<1024> &d, long long blocks_xy)
 {
-    int max_t = 1;
-    for (int i = 0; i < d.n_images; ++i) max_t = std::max(max_t, d.img[i].t);
+    int max_nq = 1;
+    for (int i = 0; i < d.n_images; ++i) max_nq = std::max(max_nq, d.merge * d.img[i].w);
     const long long want = 4LL * sm_count();
-    long long groups = (want + blocks_xy - 1) / std::max<long long>(blocks_xy, 1);
-    groups = std::max<long long>(1, std::min<long long>(groups, std::min(max_t, 65535)));
-    return (max_t + (int)groups - 1) / (int)groups;
+    long long parts = (want + blocks_xy - 1) / std::max<long long>(blocks_xy, 1);
+    parts = std::max<long long>(1, std::min<long long>(parts, std::min(max_nq, 65535)));
+    return (int)parts;
 }
 
 cudaError_t launch_vis_interp_hf(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, cudaStream_t s)
 {
     const int ec = bf16 ? 8 : 4;
     const unsigned gy = (unsigned)((ia.hidden / ec + 31) / 32);
-    const int fpb = hf_frames_per_block(d, (long long)d.n_strips * gy);
-    int max_t = 1;
-    for (int i = 0; i < d.n_images; ++i) max_t = std::max(max_t, d.img[i].t);
-    const dim3 grid((unsigned)d.n_strips, gy, (unsigned)((max_t + fpb - 1) / fpb));
+    const int parts = hf_parts(d, (long long)d.n_strips * gy);
+    const dim3 grid((unsigned)d.n_strips, gy, (unsigned)parts);
     if (bf16)
-        vis_interp_hf_kernel<__nv_bfloat16><<<grid, 32 * kHfWarps, 0, s>>>(d, ia, fpb);
+        vis_interp_hf_kernel<__nv_bfloat16><<<grid, 32 * kHfWarps, 0, s>>>(d, ia, parts);
     else
-        vis_interp_hf_kernel<float><<<grid, 32 * kHfWarps, 0, s>>>(d, ia, fpb);
+        vis_interp_hf_kernel<float><<<grid, 32 * kHfWarps, 0, s>>>(d, ia, parts);
     return cudaGetLastError();
 }
 
