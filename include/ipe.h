@@ -94,7 +94,8 @@ int ipe_kernel_arch(int *binary_version, int *ptx_version);
  * code in a device status word and lets the kernel return instead of spinning.
  * This call synchronises `stream`, reads and clears that word, and returns
  * IPE_OK, or IPE_EDEVICE with a message naming the wait that gave up (the
- * results of the failed launch are then incomplete).  ipe_mrope_rope_index
+ * results of the failed launch are then incomplete).  The position-table
+ * scan's waits are bounded the same way (code 23).  ipe_mrope_rope_index
  * and ipe_mrope_decode report inputs that only the device can see the same
  * way (codes 16 .. 22, listed there).  Not part of any page: failure
  * reporting of this library.

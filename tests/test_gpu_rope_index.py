@@ -124,10 +124,19 @@ def _many_images_batch(rng, B, L):
 
 
 def test_carry_scan_over_many_chunks(orc):
-    # more than 1024 tiles (the carry pass scans them 1024 at a time) and
-    # runs, padding and samples crossing those chunk boundaries
+    # more than 1024 tiles, with runs, padding and samples crossing tile
+    # edges and many look-back windows
     types, mask, img, vid = _long_batch(np.random.default_rng(77), 520, 2100, 400)
     assert 520 * 3 > 1024
+    check(orc, types, mask, img, vid)
+
+
+def test_scan_over_many_waves_of_tiles(orc):
+    # more tiles than the GPU holds at once (several waves of blocks): tiles
+    # look back across windows whose blocks have finished or not yet
+    # started, and samples and runs cross tile edges
+    types, mask, img, vid = _long_batch(np.random.default_rng(79), 2100, 3100, 500)
+    assert 2100 * 4 > 6000
     check(orc, types, mask, img, vid)
 
 
