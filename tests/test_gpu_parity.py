@@ -118,6 +118,32 @@ def test_cos_sin_tiles_and_tail(T, half, section, interleaved, orc):
     assert np.array_equal(c[:, :half], c[:, half:])
 
 
+def test_cos_sin_ulp_bound(orc):
+    # The tables' sine / cosine (sincosf of the fp32 angle) against the
+    # oracle's double values of the same angle: within 4 fp32 units in the
+    # last place of the exact value (CUDA documents 2 for sinf and cosf),
+    # over positions up to 2^24, where the angles of the lowest frequencies
+    # take the large-argument reduction.  Each axis gets its own positions,
+    # so every frequency sees large angles.
+    T, half = 4096, 32
+    rng = GEN(4242)
+    pos = rng.integers(0, 1 << 23, size=(3, T))
+    pos[:, :64] = rng.integers(1 << 23, 1 << 24, size=(3, 64))
+    # integers next to multiples of pi/2: tiny reduced arguments
+    k = rng.integers(1, 5_000_000, size=256)
+    pos[0, 64:320] = np.rint(k * (np.pi / 2)).astype(np.int64)
+    pos[:, 320:330] = np.arange(10)[None, :]
+    pos = pos.astype(np.int32)
+    inv = ipe.rope_inv_freq(2 * half, 1e6)
+    for interleaved in (True, False):
+        cos, sin = ipe.mrope_cos_sin(torch.from_numpy(pos).cuda(), inv, (11, 11, 10), interleaved)
+        rc, rs = orc.mrope_cos_sin(pos, orc.rope_inv_freq(2 * half, 1e6), (11, 11, 10), interleaved)
+        for name, got, ref in (("cos", cos.cpu().numpy(), rc), ("sin", sin.cpu().numpy(), rs)):
+            ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
+            err = np.abs(got.astype(np.float64) - ref) / ulp
+            assert err.max() <= 4.0, (name, interleaved, float(err.max()), np.unravel_index(err.argmax(), err.shape))
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_apply_rotary_partial_independent_tables(dtype, orc):
     # cos / sin are inputs: arbitrary tables whose halves differ exercise the
