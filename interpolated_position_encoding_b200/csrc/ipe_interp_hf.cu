@@ -25,7 +25,7 @@
 //     left-to-right sums, and writes each result chunk to every frame of
 //     the video (frames repeat frame 0).
 // The patch ranges split a strip over more blocks, so that a request of few
-// strips still puts about four blocks on every SM, while every block still
+// strips still puts about eight blocks on every SM, while every block still
 // reads each table value once for all of a video's frames.  For bf16 the products
 // and sums run as packed bf16x2 operations, which round exactly where the
 // fp32-then-round steps above do (mul_bf16x2 / add_bf16x2).
@@ -166,12 +166,15 @@ __global__ void __launch_bounds__(32 * kHfWarps) vis_interp_hf_kernel(const __gr
     }
 }
 
-// Parts per strip: enough blocks for about four per SM.
+// Parts per strip: enough blocks for about eight per SM.  Four left the
+// last partial wave a fifth of the time on the 16 x 64 x 64 video (640
+// blocks on 148 SMs: 33.3 us against 31.9 us at eight; 30.7 against 28.8 us
+// on a batch of 8 single images).
 static int hf_parts(const VisDesc<1024> &d, long long blocks_xy)
 {
     int max_nq = 1;
     for (int i = 0; i < d.n_images; ++i) max_nq = std::max(max_nq, d.merge * d.img[i].w);
-    const long long want = 4LL * sm_count();
+    const long long want = 8LL * sm_count();
     long long parts = (want + blocks_xy - 1) / std::max<long long>(blocks_xy, 1);
     parts = std::max<long long>(1, std::min<long long>(parts, std::min(max_nq, 65535)));
     return (int)parts;
