@@ -8,10 +8,15 @@
 // q and k of every full-attention layer.
 //
 // One warp per token (for short sequences, per token and group of head rows).
-// The warp writes the token's (cos, sin) pairs into its shared-memory slot once; each head row is then held by LPR = D / EC lanes
-// (EC elements = 16 bytes per lane), its sum of squares reduced with
-// shuffles inside those lanes, and the rotary partner of a chunk fetched from
-// the lane half a rotary slice away.  All D channels are written back.
+// The warp writes the token's (cos, sin) pairs into its shared-memory slot
+// once.  Two lane layouts of a head row (EC elements = 16 bytes per chunk):
+//   * qk_norm_mrope_kernel: LPR = D / EC lanes, one chunk each;
+//   * qk_norm_mrope_split_kernel, for a rotary slice narrower than the row:
+//     rot / EC lanes, D / rot chunks each, so that only a lane's first chunk
+//     is rotated.
+// The row's sum of squares is reduced with shuffles inside its lanes, and
+// the rotary partner of a chunk is fetched from the lane half a rotary slice
+// away.  All D channels are written back.
 #include "ipe_chunk.cuh"
 
 namespace ipe {
@@ -56,30 +61,30 @@ __global__ void __launch_bounds__(32 * kQkWarps, qk_min_blocks(LPR))
     const int hbeg = (gw % n.groups) * n.rows_per_item;
     const int hend = min(H, hbeg + n.rows_per_item);
     const long long tstride = (long long)gridDim.x * kQkWarps / n.groups;
-    for (long long t = gw / n.groups; t < n.T; t += tstride) {
-        Pack<uint32_t, 4> x[kQkUnroll];
-        // this lane's chunk of head row h of token t
-        auto chunk_ptr = [&](int h) {
-            T *row = h < n.hq ? static_cast<T *>(n.q) + t * n.q_stride + (long long)h * D
-                              : static_cast<T *>(n.k) + t * n.k_stride + (long long)(h - n.hq) * D;
-            return reinterpret_cast<uint32_t *>(row + e0);
-        };
-        // rows h0 + u * RPW + sub of token t (zeros past the item's last row)
-        auto load_group = [&](int h0) {
+    // x[u] holds row hbeg + u RPW + sub (+ a multiple of RPW x unroll) of the
+    // token in hand; as soon as a slot's row is written back the slot loads
+    // its row of the next group, or of this warp's next token, so the loads
+    // stay in flight while the norms, rotations and stores run.
+    Pack<uint32_t, 4> x[kQkUnroll];
+    // this lane's chunk of head row h of token t
+    auto chunk_ptr = [&](long long t, int h) {
+        T *row = h < n.hq ? static_cast<T *>(n.q) + t * n.q_stride + (long long)h * D
+                          : static_cast<T *>(n.k) + t * n.k_stride + (long long)(h - n.hq) * D;
+        return reinterpret_cast<uint32_t *>(row + e0);
+    };
+    auto load_row = [&](long long t, int h, Pack<uint32_t, 4> &v) {
+        if (t < n.T && h < hend) {
+            v = ld_pack<uint32_t, 4>(chunk_ptr(t, h));
+        } else {
 #pragma unroll
-            for (int u = 0; u < kQkUnroll; ++u) {
-                const int h = h0 + u * RPW + sub;
-                if (h < hend) {
-                    x[u] = ld_pack<uint32_t, 4>(chunk_ptr(h));
-                } else {
+            for (int i = 0; i < 4; ++i) v.v[i] = 0u;   // past the item's last row: zeros, never stored
+        }
+    };
+    long long t = gw / n.groups;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) x[u].v[i] = 0u;
-                }
-            }
-        };
-        // the first rows are in flight while the angles are computed
-        load_group(hbeg);
-        // (cos, sin) of every frequency of token t
+    for (int u = 0; u < kQkUnroll; ++u) load_row(t, hbeg + u * RPW + sub, x[u]);
+    for (; t < n.T; t += tstride) {
+        // (cos, sin) of every frequency of token t, while its rows load
         for (int j = lane; j < half; j += 32) {
             const int ax = mrope_axis(j, a.section, a.interleaved);
             const int pos = __ldg(a.positions + (long long)ax * a.T + t);
@@ -96,7 +101,7 @@ __global__ void __launch_bounds__(32 * kQkWarps, qk_min_blocks(LPR))
             si[i] = first_half ? make_float2(-sv.x, -sv.y) : sv;
         }
         for (int h0 = hbeg; h0 < hend; h0 += RPW * kQkUnroll) {
-            if (h0 > hbeg) load_group(h0);
+            const bool last = h0 + RPW * kQkUnroll >= hend;
 #pragma unroll
             for (int u = 0; u < kQkUnroll; ++u) {
                 // every lane of the warp takes part in the shuffles, rows past
@@ -108,11 +113,188 @@ __global__ void __launch_bounds__(32 * kQkWarps, qk_min_blocks(LPR))
                 for (int i = 0; i < 4; ++i) w[i] = is_q ? wq.v[i] : wk.v[i];
                 const Pack<uint32_t, 4> y = rms_norm_chunk<T, LPR>(x[u], w, inv_d, n.eps);
                 const Pack<uint32_t, 4> o = rotate_row_chunk<T>(y, co, si, partner);
-                if (h < hend) st_pack<uint32_t, 4>(chunk_ptr(h), o);
+                if (h < hend) st_pack<uint32_t, 4>(chunk_ptr(t, h), o);
+                if (last)
+                    load_row(t + tstride, hbeg + u * RPW + sub, x[u]);
+                else
+                    load_row(t, h + RPW * kQkUnroll, x[u]);
             }
         }
         __syncwarp();
     }
+}
+
+// Rows whose rotary slice is narrower than the row (rot < D, rot / EC a
+// power of two): LPR = rot / EC lanes per head row, each holding the CPL =
+// D / rot chunks c, c + LPR, ... of it (a stride of rot channels).  A lane's
+// first chunk lies in the rotary slice and the others pass through, so the
+// rotation (partner shuffle and arithmetic) runs on one chunk in CPL instead
+// of on every chunk, and the sum of squares is reduced over LPR lanes.  Each
+// chunk's norm, cast and weight product are those of the kernel above; only
+// the order in which the row's squares are summed differs.  The norm weights
+// sit in shared memory; the next row of a lane's CPL chunks is loaded while
+// the current one is worked on.  MINB blocks per SM: three keep more warps
+// on short sequences, two leave bf16 rows of four chunks per lane their
+// registers (at three they spill) for long ones.  Measured on B200, bf16
+// D = 256, rot 64: 131072 tokens 606 us at three against 584 us at two;
+// 4096 tokens 24.3 us against 33.5 us.
+template <typename T, int LPR, int CPL, int MINB>
+__global__ void __launch_bounds__(32 * kQkWarps, MINB)
+    qk_norm_mrope_split_kernel(const __grid_constant__ QkNormArgs n, const __grid_constant__ MropeAngles a)
+{
+    constexpr int EC = QkElem<T>::EC;
+    constexpr int NP = EC / 2;                        // fp32 pairs of a 16-byte chunk
+    constexpr int RPW = 32 / LPR;                     // head rows per warp access
+    constexpr int ROT = LPR * EC;                     // rotary channels
+    constexpr int D = ROT * CPL;
+    constexpr int WCH = D / EC;                       // chunks of one weight vector
+    extern __shared__ float4 qk_smem[];
+    uint4 *wsm = reinterpret_cast<uint4 *>(qk_smem);  // q weights, then k weights
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float *cs_c = reinterpret_cast<float *>(wsm + 2 * WCH) + (size_t)warp * 2 * n.half_pad;
+    float *cs_s = cs_c + n.half_pad;
+    for (int i = threadIdx.x; i < 2 * WCH; i += blockDim.x)
+        wsm[i] = *reinterpret_cast<const uint4 *>(i < WCH ? static_cast<const T *>(n.q_weight) + i * EC
+                                                          : static_cast<const T *>(n.k_weight) + (i - WCH) * EC);
+    __syncthreads();
+    constexpr int half = ROT / 2;
+    const int c = lane % LPR;                         // this lane's rotary chunk
+    const int sub = lane / LPR;                       // which of the RPW rows
+    const int e0 = c * EC;
+    const bool first_half = e0 < half;
+    const int j0 = first_half ? e0 : e0 - half;       // frequency of element e0
+    const int partner = first_half ? lane + half / EC : lane - half / EC;
+    const float inv_d = __frcp_rn((float)D);          // D a power of two: exact
+    const int H = n.hq + n.hk;
+    const int gw = blockIdx.x * kQkWarps + warp;
+    const int hbeg = (gw % n.groups) * n.rows_per_item;
+    const int hend = min(H, hbeg + n.rows_per_item);
+    const long long tstride = (long long)gridDim.x * kQkWarps / n.groups;
+    auto row_ptr = [&](long long t, int h) {
+        T *row = h < n.hq ? static_cast<T *>(n.q) + t * n.q_stride + (long long)h * D
+                          : static_cast<T *>(n.k) + t * n.k_stride + (long long)(h - n.hq) * D;
+        return reinterpret_cast<uint32_t *>(row + e0);
+    };
+    // this lane's CPL chunks of row h of token t (zeros past the item's rows)
+    auto load_row = [&](long long t, int h, Pack<uint32_t, 4> *v) {
+        if (t < n.T && h < hend) {
+            const uint32_t *p = row_ptr(t, h);
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) v[k] = ld_pack<uint32_t, 4>(p + k * (ROT * (int)sizeof(T) / 4));
+        } else {
+#pragma unroll
+            for (int k = 0; k < CPL; ++k)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) v[k].v[i] = 0u;
+        }
+    };
+    long long t = gw / n.groups;
+    Pack<uint32_t, 4> x[CPL];
+    load_row(t, hbeg + sub, x);
+    for (; t < n.T; t += tstride) {
+        // (cos, sin) of every frequency of token t
+        for (int j = lane; j < half; j += 32) {
+            const int ax = mrope_axis(j, a.section, a.interleaved);
+            const int pos = __ldg(a.positions + (long long)ax * a.T + t);
+            const float angle = __fmul_rn(__int2float_rn(pos), a.inv[j]);
+            sincosf(angle, &cs_s[j], &cs_c[j]);
+        }
+        __syncwarp();
+        float2 co[NP], si[NP];
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+            co[i] = make_float2(cs_c[j0 + 2 * i], cs_c[j0 + 2 * i + 1]);
+            const float2 sv = make_float2(cs_s[j0 + 2 * i], cs_s[j0 + 2 * i + 1]);
+            si[i] = first_half ? make_float2(-sv.x, -sv.y) : sv;
+        }
+        for (int h0 = hbeg; h0 < hend; h0 += RPW) {
+            const int h = h0 + sub;
+            // the next row (of this token, or of the next one) is loaded now
+            Pack<uint32_t, 4> nx[CPL];
+            if (h0 + RPW < hend)
+                load_row(t, h + RPW, nx);
+            else
+                load_row(t + tstride, hbeg + sub, nx);
+            // every lane of the warp takes part in the shuffles
+            float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+                float2 xv[NP];
+                chunk_to_pairs<T>(x[k].v, xv);
+#pragma unroll
+                for (int i = 0; i < NP; ++i) acc = (k == 0 && i == 0) ? mul2(xv[0], xv[0]) : fma2(xv[i], xv[i], acc);
+            }
+            float ss = __fadd_rn(acc.x, acc.y);
+#pragma unroll
+            for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off, LPR);
+            const float r = __frsqrt_rn(__fadd_rn(__fmul_rn(ss, inv_d), n.eps));
+            const float2 r2 = make_float2(r, r);
+            const uint4 *wrow = wsm + (h < n.hq ? 0 : WCH) + c;
+            Pack<uint32_t, 4> y[CPL];
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+                // cast back first, then the weight
+                float2 xv[NP];
+                chunk_to_pairs<T>(x[k].v, xv);
+#pragma unroll
+                for (int i = 0; i < NP; ++i) xv[i] = mul2(xv[i], r2);
+                pairs_to_chunk<T>(xv, y[k].v);
+                const uint4 wv = wrow[k * LPR];
+                const uint32_t w[4] = {wv.x, wv.y, wv.z, wv.w};
+                if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) y[k].v[i] = mul_bf16x2(y[k].v[i], w[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        y[k].v[i] = __float_as_uint(__fmul_rn(__uint_as_float(y[k].v[i]), __uint_as_float(w[i])));
+                }
+            }
+            y[0] = rotate_row_chunk<T>(y[0], co, si, partner);
+            if (h < hend) {
+                uint32_t *p = row_ptr(t, h);
+#pragma unroll
+                for (int k = 0; k < CPL; ++k) st_pack<uint32_t, 4>(p + k * (ROT * (int)sizeof(T) / 4), y[k]);
+            }
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) x[k] = nx[k];
+        }
+        __syncwarp();
+    }
+}
+
+// Warps over tokens and head-row groups (shared by both kernels): a token's
+// head rows are split over several warps (whole passes of `unit` rows each)
+// until there are about four warps per resident warp slot; long sequences
+// keep one warp per token.
+static void qk_grid(QkNormArgs &m, int unit, int per_sm, long long &blocks)
+{
+    const int H = m.hq + m.hk;
+    const int max_groups = (H + unit - 1) / unit;
+    const long long want = 4LL * sm_count() * std::max(per_sm, 1) * kQkWarps;
+    int groups = 1;
+    while (groups < max_groups && m.T * groups < want) ++groups;
+    m.rows_per_item = ((H + groups - 1) / groups + unit - 1) / unit * unit;
+    m.groups = (H + m.rows_per_item - 1) / m.rows_per_item;
+    const long long need = (m.T * m.groups + kQkWarps - 1) / kQkWarps;
+    blocks = std::max<long long>(1, std::min(need, (long long)sm_count() * std::max(per_sm, 1)));
+    blocks = (blocks + m.groups - 1) / m.groups * m.groups;   // a whole number of groups per stride
+}
+
+template <typename T, int LPR, int CPL, int MINB>
+static cudaError_t qk_launch_split(const QkNormArgs &n, const MropeAngles &a, cudaStream_t s)
+{
+    constexpr int EC = QkElem<T>::EC;
+    const size_t smem = 2 * (size_t)LPR * CPL * EC * sizeof(T) + (size_t)kQkWarps * 2 * n.half_pad * sizeof(float);
+    auto kern = qk_norm_mrope_split_kernel<T, LPR, CPL, MINB>;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32 * kQkWarps, smem);
+    if (e != cudaSuccess) return e;
+    QkNormArgs m = n;
+    long long blocks = 0;
+    qk_grid(m, 32 / LPR, per_sm, blocks);
+    kern<<<(unsigned)blocks, 32 * kQkWarps, smem, s>>>(m, a);
+    return cudaGetLastError();
 }
 
 template <typename T, int LPR>
@@ -123,29 +305,37 @@ static cudaError_t qk_launch(const QkNormArgs &n, const MropeAngles &a, cudaStre
     int per_sm = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32 * kQkWarps, smem);
     if (e != cudaSuccess) return e;
-    // Short sequences: a token's head rows are split over several warps
-    // (whole passes of RPW x unroll rows each) until there are about four
-    // warps per resident warp slot; long ones keep one warp per token.
     QkNormArgs m = n;
-    const int unit = (32 / LPR) * qk_unroll(LPR);
-    const int H = n.hq + n.hk;
-    const int max_groups = (H + unit - 1) / unit;
-    const long long want = 4LL * sm_count() * std::max(per_sm, 1) * kQkWarps;
-    int groups = 1;
-    while (groups < max_groups && n.T * groups < want) ++groups;
-    m.rows_per_item = ((H + groups - 1) / groups + unit - 1) / unit * unit;
-    m.groups = (H + m.rows_per_item - 1) / m.rows_per_item;
-    const long long need = (n.T * m.groups + kQkWarps - 1) / kQkWarps;
-    long long blocks = std::max<long long>(1, std::min(need, (long long)sm_count() * std::max(per_sm, 1)));
-    blocks = (blocks + m.groups - 1) / m.groups * m.groups;   // a whole number of groups per stride
+    long long blocks = 0;
+    qk_grid(m, (32 / LPR) * qk_unroll(LPR), per_sm, blocks);
     kern<<<(unsigned)blocks, 32 * kQkWarps, smem, s>>>(m, a);
     return cudaGetLastError();
+}
+
+// Sequences of at least this many tokens take two blocks per SM for rows
+// of four chunks per lane.
+constexpr long long kQkLongT = 16384;
+
+template <typename T, int LPR>
+static cudaError_t qk_split_cpl(int cpl, const QkNormArgs &n, const MropeAngles &a, cudaStream_t s)
+{
+    if (cpl == 2) return qk_launch_split<T, LPR, 2, 3>(n, a, s);
+    if (n.T >= kQkLongT) return qk_launch_split<T, LPR, 4, 2>(n, a, s);
+    return qk_launch_split<T, LPR, 4, 3>(n, a, s);
 }
 
 template <typename T>
 static cudaError_t qk_dispatch(const QkNormArgs &n, const MropeAngles &a, cudaStream_t s)
 {
-    switch (n.head_dim / QkElem<T>::EC) {
+    constexpr int EC = QkElem<T>::EC;
+    // a rotary slice of 4, 8 or 16 lanes and 2 or 4 of its widths per row
+    const int lr = 2 * n.half / EC, cpl = n.head_dim / (2 * n.half);
+    if (2 * n.half < n.head_dim && n.head_dim % (2 * n.half) == 0 && (cpl == 2 || cpl == 4)) {
+        if (lr == 4) return qk_split_cpl<T, 4>(cpl, n, a, s);
+        if (lr == 8) return qk_split_cpl<T, 8>(cpl, n, a, s);
+        if (lr == 16) return qk_split_cpl<T, 16>(cpl, n, a, s);
+    }
+    switch (n.head_dim / EC) {
     case 32: return qk_launch<T, 32>(n, a, s);
     case 16: return qk_launch<T, 16>(n, a, s);
     case 8: return qk_launch<T, 8>(n, a, s);

@@ -97,7 +97,26 @@ def test_qk_norm_mrope_small(case, dtype, orc):
                  f"{case} {dtype} {nm}")
 
 
-@pytest.mark.parametrize("name,layout", [("text_t4096_qwen35", "interleaved"), ("text_t32768_omni", "chunked")])
+def test_qk_norm_mrope_long_sequence(orc):
+    # 16411 tokens (past the length where rows of four 16-byte chunks per
+    # lane take the two-blocks-per-SM form; not a multiple of the warp
+    # count), D = 256 with a 64-channel rotary slice: every token compared
+    T, hq, hk, D, rot, section = 16411, 5, 3, 256, 64, (11, 11, 10)
+    rng = GEN(16411)
+    q, k = wl.normal_bf16(rng, (T, hq, D), 3.0), wl.normal_bf16(rng, (T, hk, D), 3.0)
+    wq, wk = wl.normal_bf16(rng, (D,), 0.5), wl.normal_bf16(rng, (D,), 0.5)
+    p = rng.integers(0, 200000, (3, T)).astype(np.int32)
+    gq, gk = to_gpu(q, "bf16"), to_gpu(k, "bf16")
+    ipe.qk_norm_mrope(gq, gk, to_gpu(wq, "bf16"), to_gpu(wk, "bf16"), torch.from_numpy(p).cuda(),
+                      ipe.rope_inv_freq(rot, 1e7), section, True, eps=1e-6)
+    oinv = orc.rope_inv_freq(rot, 1e7)
+    for nm, x, w, g in (("q", q, wq, gq), ("k", k, wk, gk)):
+        check_qk(gpu_to_f64(g), host_f64(x, "bf16"), host_f64(w, "bf16"), 1e-6, "bf16", p, oinv, section, True, orc,
+                 f"long {nm}")
+
+
+@pytest.mark.parametrize("name,layout", [("text_t4096_qwen35", "interleaved"), ("text_t32768_omni", "chunked"),
+                                         ("prefill_t131072_video", "interleaved")])
 def test_qk_norm_mrope_workload(name, layout, orc):
     w = wl.WORKLOADS[name]
     t = w.text
