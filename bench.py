@@ -439,6 +439,8 @@ CASES = {
     "mrope_apply_prefill": "fused MRoPE of the large-prefill request (Q [131072, 24, 256], K [131072, 4, 256])",
     "mrope_apply_short": "fused MRoPE on the 4096-token prompt (text_t4096_qwen35: Q [4096, 24, 256], K [4096, 4, 256])",
     "qk_norm_mrope_short": "fused QK-RMSNorm + MRoPE on the 4096-token prompt (text_t4096_qwen35)",
+    "qk_norm_mrope_prefill_quarter": "fused QK-RMSNorm + MRoPE on the first 32768 tokens of the large-prefill "
+                                     "request (Q [32768, 24, 256], K [32768, 4, 256] bf16, 470 MB)",
     "vis_fused_batch8": "interpolation and vision rotary in one call on the batch of 8 single images (N = 26528)",
     "vis_fused_prefill": "interpolation and vision rotary in one call on the 16 x 64 x 64 video of the large prefill",
     "vis_pos_interp_hf": "interpolation in HF rounding mode, 16 x 64 x 64 video of the large-prefill request",
@@ -513,21 +515,23 @@ def run_case(args):
         out = torch.empty(wl.n_patches(v), v.hidden, dtype=torch.bfloat16, device=dev)
         fn = lambda: ipe.vis_pos_interp(table, v.grid_thw, v.merge, out=out, stream=stream)  # noqa: E731
         nbytes = algorithmic_bytes_vision(v)
-    elif name in ("mrope_apply_short", "qk_norm_mrope_short", "mrope_apply_prefill"):
-        w = wl.WORKLOADS["prefill_t131072_video" if name == "mrope_apply_prefill" else "text_t4096_qwen35"]
+    elif name in ("mrope_apply_short", "qk_norm_mrope_short", "mrope_apply_prefill", "qk_norm_mrope_prefill_quarter"):
+        big = name in ("mrope_apply_prefill", "qk_norm_mrope_prefill_quarter")
+        w = wl.WORKLOADS["prefill_t131072_video" if big else "text_t4096_qwen35"]
         t = w.text
         tin = wl.text_inputs(w)
-        Q = torch.from_numpy(tin["q"].view(np.int16)).view(torch.bfloat16).to(dev)
-        K = torch.from_numpy(tin["k"].view(np.int16)).view(torch.bfloat16).to(dev)
-        pos = torch.from_numpy(tin["positions"]).to(dev)
+        T = t.T // 4 if name == "qk_norm_mrope_prefill_quarter" else t.T
+        Q = torch.from_numpy(tin["q"][:T].view(np.int16)).view(torch.bfloat16).to(dev)
+        K = torch.from_numpy(tin["k"][:T].view(np.int16)).view(torch.bfloat16).to(dev)
+        pos = torch.from_numpy(np.ascontiguousarray(tin["positions"][:, :T])).to(dev)
         inv = ipe.rope_inv_freq(t.rot_dim, t.theta)
-        if name != "qk_norm_mrope_short":
+        if name.startswith("mrope_apply"):
             fn = lambda: ipe.mrope_apply(Q, K, pos, inv, t.section, True, stream=stream)  # noqa: E731
-            nbytes = (t.hq + t.hk) * t.T * t.rot_dim * 2 * 2 + 3 * t.T * 4
+            nbytes = (t.hq + t.hk) * T * t.rot_dim * 2 * 2 + 3 * T * 4
         else:
             wq = torch.ones(t.head_dim, dtype=torch.bfloat16, device=dev)
             fn = lambda: ipe.qk_norm_mrope(Q, K, wq, wq, pos, inv, t.section, True, stream=stream)  # noqa: E731
-            nbytes = (t.hq + t.hk) * t.T * t.head_dim * 2 * 2 + 3 * t.T * 4
+            nbytes = (t.hq + t.hk) * T * t.head_dim * 2 * 2 + 3 * T * 4
     elif name == "fill_reference":
         t = wl.WORKLOADS[WORKLOAD].text
         buf = torch.empty(2 * t.T * t.rot_dim, dtype=torch.float32, device=dev)
