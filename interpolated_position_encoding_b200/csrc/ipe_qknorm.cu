@@ -9,11 +9,14 @@
 //
 // One warp per token (for short sequences, per token and group of head rows).
 // The warp writes the token's (cos, sin) pairs into its shared-memory slot
-// once.  Two lane layouts of a head row (EC elements = 16 bytes per chunk):
-//   * qk_norm_mrope_kernel: LPR = D / EC lanes, one chunk each;
+// once.  Three lane layouts of a head row (EC elements = 16 bytes per chunk):
 //   * qk_norm_mrope_split_kernel, for a rotary slice narrower than the row:
 //     rot / EC lanes, D / rot chunks each, so that only a lane's first chunk
-//     is rotated.
+//     is rotated;
+//   * qk_norm_mrope_pair_kernel, for a rotary slice as wide as the row:
+//     D / (2 EC) lanes, each with a chunk of either half, so that both
+//     members of a rotation pair sit in one lane;
+//   * qk_norm_mrope_kernel otherwise: LPR = D / EC lanes, one chunk each.
 // The row's sum of squares is reduced with shuffles inside its lanes, and
 // the rotary partner of a chunk is fetched from the lane half a rotary slice
 // away.  All D channels are written back.
@@ -281,6 +284,164 @@ static void qk_grid(QkNormArgs &m, int unit, int per_sm, long long &blocks)
     blocks = (blocks + m.groups - 1) / m.groups * m.groups;   // a whole number of groups per stride
 }
 
+// Rows whose rotary slice is the whole row (rot = D, Qwen3-Omni): LPR =
+// half / EC lanes per head row, each holding chunk c of the first half and
+// chunk c of the second half (elements e0 + j and e0 + half + j).  Both
+// members of every rotation pair then sit in the same lane, so the rotation
+// needs no partner shuffle, and the sum of squares is reduced over LPR
+// lanes instead of D / EC.  The norm, cast, weight product and rotation are
+// those of the kernels above; only the order in which the row's squares are
+// summed differs.
+template <typename T, int LPR>
+__global__ void __launch_bounds__(32 * kQkWarps, 4)
+    qk_norm_mrope_pair_kernel(const __grid_constant__ QkNormArgs n, const __grid_constant__ MropeAngles a)
+{
+    constexpr int EC = QkElem<T>::EC;
+    constexpr int NP = EC / 2;                        // fp32 pairs of a 16-byte chunk
+    constexpr int RPW = 32 / LPR;                     // head rows per warp access
+    constexpr int HALF = LPR * EC;
+    constexpr int D = 2 * HALF;
+    constexpr int WCH = D / EC;                       // chunks of one weight vector
+    extern __shared__ float4 qk_smem[];
+    uint4 *wsm = reinterpret_cast<uint4 *>(qk_smem);  // q weights, then k weights
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float *cs_c = reinterpret_cast<float *>(wsm + 2 * WCH) + (size_t)warp * 2 * n.half_pad;
+    float *cs_s = cs_c + n.half_pad;
+    for (int i = threadIdx.x; i < 2 * WCH; i += blockDim.x)
+        wsm[i] = *reinterpret_cast<const uint4 *>(i < WCH ? static_cast<const T *>(n.q_weight) + i * EC
+                                                          : static_cast<const T *>(n.k_weight) + (i - WCH) * EC);
+    __syncthreads();
+    const int c = lane % LPR;                         // this lane's chunk of each half
+    const int sub = lane / LPR;                       // which of the RPW rows
+    const int e0 = c * EC;
+    const float inv_d = __frcp_rn((float)D);          // D a power of two: exact
+    const int H = n.hq + n.hk;
+    const int gw = blockIdx.x * kQkWarps + warp;
+    const int hbeg = (gw % n.groups) * n.rows_per_item;
+    const int hend = min(H, hbeg + n.rows_per_item);
+    const long long tstride = (long long)gridDim.x * kQkWarps / n.groups;
+    constexpr int kHalfWords = HALF * (int)sizeof(T) / 4;
+    auto row_ptr = [&](long long t, int h) {
+        T *row = h < n.hq ? static_cast<T *>(n.q) + t * n.q_stride + (long long)h * D
+                          : static_cast<T *>(n.k) + t * n.k_stride + (long long)(h - n.hq) * D;
+        return reinterpret_cast<uint32_t *>(row + e0);
+    };
+    auto load_row = [&](long long t, int h, Pack<uint32_t, 4> *v) {
+        if (t < n.T && h < hend) {
+            const uint32_t *p = row_ptr(t, h);
+            v[0] = ld_pack<uint32_t, 4>(p);
+            v[1] = ld_pack<uint32_t, 4>(p + kHalfWords);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) v[k].v[i] = 0u;
+        }
+    };
+    long long t = gw / n.groups;
+    Pack<uint32_t, 4> x[2];
+    load_row(t, hbeg + sub, x);
+    for (; t < n.T; t += tstride) {
+        // (cos, sin) of every frequency of token t
+        for (int j = lane; j < HALF; j += 32) {
+            const int ax = mrope_axis(j, a.section, a.interleaved);
+            const int pos = __ldg(a.positions + (long long)ax * a.T + t);
+            const float angle = __fmul_rn(__int2float_rn(pos), a.inv[j]);
+            sincosf(angle, &cs_s[j], &cs_c[j]);
+        }
+        __syncwarp();
+        float2 co[NP], sn[NP];
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+            co[i] = make_float2(cs_c[e0 + 2 * i], cs_c[e0 + 2 * i + 1]);
+            sn[i] = make_float2(cs_s[e0 + 2 * i], cs_s[e0 + 2 * i + 1]);
+        }
+        for (int h0 = hbeg; h0 < hend; h0 += RPW) {
+            const int h = h0 + sub;
+            Pack<uint32_t, 4> nx[2];
+            if (h0 + RPW < hend)
+                load_row(t, h + RPW, nx);
+            else
+                load_row(t + tstride, hbeg + sub, nx);
+            float2 xa[NP], xb[NP];
+            chunk_to_pairs<T>(x[0].v, xa);
+            chunk_to_pairs<T>(x[1].v, xb);
+            float2 acc = mul2(xa[0], xa[0]);
+#pragma unroll
+            for (int i = 1; i < NP; ++i) acc = fma2(xa[i], xa[i], acc);
+#pragma unroll
+            for (int i = 0; i < NP; ++i) acc = fma2(xb[i], xb[i], acc);
+            float ss = __fadd_rn(acc.x, acc.y);
+#pragma unroll
+            for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off, LPR);
+            const float r = __frsqrt_rn(__fadd_rn(__fmul_rn(ss, inv_d), n.eps));
+            const float2 r2 = make_float2(r, r);
+            const uint4 *wrow = wsm + (h < n.hq ? 0 : WCH) + c;
+            // cast back first, then the weight (both halves)
+            Pack<uint32_t, 4> ya, yb;
+#pragma unroll
+            for (int i = 0; i < NP; ++i) {
+                xa[i] = mul2(xa[i], r2);
+                xb[i] = mul2(xb[i], r2);
+            }
+            pairs_to_chunk<T>(xa, ya.v);
+            pairs_to_chunk<T>(xb, yb.v);
+            const uint4 wa = wrow[0], wb = wrow[LPR];
+            const uint32_t wav[4] = {wa.x, wa.y, wa.z, wa.w}, wbv[4] = {wb.x, wb.y, wb.z, wb.w};
+            if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    ya.v[i] = mul_bf16x2(ya.v[i], wav[i]);
+                    yb.v[i] = mul_bf16x2(yb.v[i], wbv[i]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    ya.v[i] = __float_as_uint(__fmul_rn(__uint_as_float(ya.v[i]), __uint_as_float(wav[i])));
+                    yb.v[i] = __float_as_uint(__fmul_rn(__uint_as_float(yb.v[i]), __uint_as_float(wbv[i])));
+                }
+            }
+            // x'[j] = x[j] cos_j - x[j+h] sin_j,  x'[j+h] = x[j+h] cos_j + x[j] sin_j
+            float2 va[NP], vb[NP], oa[NP], ob[NP];
+            chunk_to_pairs<T>(ya.v, va);
+            chunk_to_pairs<T>(yb.v, vb);
+#pragma unroll
+            for (int i = 0; i < NP; ++i) {
+                const float2 ns = make_float2(-sn[i].x, -sn[i].y);
+                oa[i] = fma2(va[i], co[i], mul2(vb[i], ns));
+                ob[i] = fma2(vb[i], co[i], mul2(va[i], sn[i]));
+            }
+            Pack<uint32_t, 4> pa, pb;
+            pairs_to_chunk<T>(oa, pa.v);
+            pairs_to_chunk<T>(ob, pb.v);
+            if (h < hend) {
+                uint32_t *p = row_ptr(t, h);
+                st_pack<uint32_t, 4>(p, pa);
+                st_pack<uint32_t, 4>(p + kHalfWords, pb);
+            }
+            x[0] = nx[0];
+            x[1] = nx[1];
+        }
+        __syncwarp();
+    }
+}
+
+template <typename T, int LPR>
+static cudaError_t qk_launch_pair(const QkNormArgs &n, const MropeAngles &a, cudaStream_t s)
+{
+    constexpr int EC = QkElem<T>::EC;
+    const size_t smem = 2 * (size_t)2 * LPR * EC * sizeof(T) + (size_t)kQkWarps * 2 * n.half_pad * sizeof(float);
+    auto kern = qk_norm_mrope_pair_kernel<T, LPR>;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32 * kQkWarps, smem);
+    if (e != cudaSuccess) return e;
+    QkNormArgs m = n;
+    long long blocks = 0;
+    qk_grid(m, 32 / LPR, per_sm, blocks);
+    kern<<<(unsigned)blocks, 32 * kQkWarps, smem, s>>>(m, a);
+    return cudaGetLastError();
+}
+
 template <typename T, int LPR, int CPL, int MINB>
 static cudaError_t qk_launch_split(const QkNormArgs &n, const MropeAngles &a, cudaStream_t s)
 {
@@ -334,6 +495,11 @@ static cudaError_t qk_dispatch(const QkNormArgs &n, const MropeAngles &a, cudaSt
         if (lr == 4) return qk_split_cpl<T, 4>(cpl, n, a, s);
         if (lr == 8) return qk_split_cpl<T, 8>(cpl, n, a, s);
         if (lr == 16) return qk_split_cpl<T, 16>(cpl, n, a, s);
+    }
+    if (2 * n.half == n.head_dim) {
+        if (lr == 8) return qk_launch_pair<T, 4>(n, a, s);
+        if (lr == 16) return qk_launch_pair<T, 8>(n, a, s);
+        if (lr == 32) return qk_launch_pair<T, 16>(n, a, s);
     }
     switch (n.head_dim / EC) {
     case 32: return qk_launch<T, 32>(n, a, s);

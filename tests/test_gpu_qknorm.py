@@ -59,12 +59,17 @@ def check_qk(got, x, w, eps, dtype, pos, inv, section, interleaved, orc, what):
     return {"flips": flips, "beyond": beyond}
 
 
+# (T, hq, hk, D, rot, section).  The library picks a lane layout by shape:
+# rot < D with rot / 16 bytes a power of two takes rot / 16 bytes lanes per
+# row (several chunks each); rot = D takes D / 32 bytes lanes (a chunk of
+# each half); any other slice, one chunk per lane.  The cases reach all three.
 CASES = [  # (T, hq, hk, D, rot, section)
     (37, 3, 2, 128, 64, (12, 10, 10)),
     (64, 24, 4, 256, 64, (11, 11, 10)),    # Qwen3.5 heads
     (33, 4, 4, 128, 128, (24, 20, 20)),    # full-dim rotary (Qwen3-Omni)
     (19, 2, 1, 64, 32, (6, 5, 5)),
     (8, 5, 3, 256, 256, (44, 42, 42)),
+    (21, 3, 2, 128, 96, (16, 16, 16)),    # rotary slice of 12 (bf16) or 24 (fp32) chunks: one chunk per lane
 ]
 
 
