@@ -82,7 +82,8 @@ int ipe_version(void);
  * for, as the CUDA runtime loaded it on the current device
  * (cudaFuncGetAttributes: binaryVersion and ptxVersion, major * 10 + minor;
  * 100 for sm_100a).  Needs a CUDA device; IPE_ECUDA when the library's code
- * cannot run on it.  Not part of any page: a check of this build.
+ * cannot run on it.  No counterpart on the pages: it reports which GPU
+ * architecture the library's kernels were compiled for.
  *   binary_version, ptx_version   host int*, written.
  * ------------------------------------------------------------------------- */
 int ipe_kernel_arch(int *binary_version, int *ptx_version);
