@@ -197,10 +197,13 @@ cudaError_t launch_rotary_table(bool bf16, const RotArgs &r, const TableAngles &
 
 cudaError_t launch_vis_plan(const VisDesc<1024> &d, int32_t *idx4, float *w4, int32_t *rowcol,
                             cudaStream_t s);
+// Shared memory of one interpolation block for this request.
+size_t vis_interp_block_smem(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia);
 cudaError_t launch_vis_interp(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, cudaStream_t s);
 cudaError_t launch_vis_interp_hf(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, cudaStream_t s);
+// `budget`: shared memory per rotary block to aim for (0: the default).
 cudaError_t launch_vis_rope(bool bf16, const VisDesc<1024> &d, const RotArgs &r,
-                            const VisAngleFreqs &f, cudaStream_t s);
+                            const VisAngleFreqs &f, cudaStream_t s, size_t budget = 0);
 
 // Widest vector (elements, <= 16 bytes) that divides half, head_dim and both
 // strides of `r` and that both base pointers are aligned to.

@@ -509,9 +509,11 @@ inline int best_swap_shift(unsigned row_bytes, unsigned half_bytes, unsigned acc
 }
 
 // Fills the stage layout of `a` and picks the stage count for the
-// shared-memory budget.
+// shared-memory budget: the deepest ring within `first` bytes (a caller
+// that shares the SMs with another kernel passes less than the default)
+// when two stages fit there, else as below.
 template <typename T, int VEC, class Src>
-void tma_layout(TmaRotArgs &a)
+void tma_layout(TmaRotArgs &a, size_t first = kTmaBlockSmem)
 {
     const unsigned eb = sizeof(T);
     const unsigned rot = 2u * a.half;
@@ -531,7 +533,7 @@ void tma_layout(TmaRotArgs &a)
     a.swap_shift = best_swap_shift(rot * eb, a.half * eb, VEC * eb);
     // deepest ring within ~112 KB (two blocks per SM); rows too wide for two
     // stages there get up to ~220 KB (one block per SM)
-    for (size_t budget : {kTmaBlockSmem, size_t(220 * 1024)}) {
+    for (size_t budget : {first, kTmaBlockSmem, size_t(220 * 1024)}) {
         a.stages = 2;
         for (int st = kTmaMaxStages; st >= 2; --st) {
             a.stages = st;
@@ -543,9 +545,9 @@ void tma_layout(TmaRotArgs &a)
 
 // Lays out `a` and launches the pipeline on the SMs.
 template <typename T, int VEC, class Src>
-cudaError_t launch_rotary_tma_vec(TmaRotArgs a, const Src &src, cudaStream_t s)
+cudaError_t launch_rotary_tma_vec(TmaRotArgs a, const Src &src, cudaStream_t s, size_t first = kTmaBlockSmem)
 {
-    tma_layout<T, VEC, Src>(a);
+    tma_layout<T, VEC, Src>(a, first);
     const size_t smem = tma_smem_bytes(a, Src::kHi);
     auto kern = rotary_tma_kernel<T, VEC, Src>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

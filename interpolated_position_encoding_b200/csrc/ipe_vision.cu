@@ -311,6 +311,11 @@ static cudaError_t interp_impl(const VisDesc<1024> &d, const InterpArgs &ia, cud
     return m2 ? interp_slices<T, 4, 2, MAXIMG>(u, d, ia, s) : interp_slices<T, 4, 0, MAXIMG>(u, d, ia, s);
 }
 
+size_t vis_interp_block_smem(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia)
+{
+    return interp_smem_bytes(bf16, d.merge, d.grid_side, interp_pick_slices(bf16, d, ia));
+}
+
 cudaError_t launch_vis_interp(bool bf16, const VisDesc<1024> &d, const InterpArgs &ia, cudaStream_t s)
 {
     if (bf16)
@@ -319,7 +324,8 @@ cudaError_t launch_vis_interp(bool bf16, const VisDesc<1024> &d, const InterpArg
 }
 
 template <typename T, int MAXIMG>
-static cudaError_t rope_impl(const VisDesc<1024> &d, const RotArgs &r, const VisAngleFreqs &f, cudaStream_t s)
+static cudaError_t rope_impl(const VisDesc<1024> &d, const RotArgs &r, const VisAngleFreqs &f, cudaStream_t s,
+                             size_t budget)
 {
     TmaRotArgs t;
     if (tma_rot_args(r, sizeof(T), t)) {
@@ -327,21 +333,22 @@ static cudaError_t rope_impl(const VisDesc<1024> &d, const RotArgs &r, const Vis
         VisTmaSrc<MAXIMG> src{shrink<MAXIMG>(d), f};
         const int v = pick_vec(r, sizeof(T));
         if constexpr (sizeof(T) == 2) {
-            if (v == 8) return launch_rotary_tma_vec<T, 8>(t, src, s);
+            if (v == 8) return launch_rotary_tma_vec<T, 8>(t, src, s, budget);
         }
-        if (v >= 4) return launch_rotary_tma_vec<T, 4>(t, src, s);
-        return launch_rotary_tma_vec<T, 2>(t, src, s);   // VEC >= 2 on the TMA path
+        if (v >= 4) return launch_rotary_tma_vec<T, 4>(t, src, s, budget);
+        return launch_rotary_tma_vec<T, 2>(t, src, s, budget);   // VEC >= 2 on the TMA path
     }
     VisSrc<MAXIMG> src{shrink<MAXIMG>(d), f};
     return dispatch_vec<T>(r, src, s);
 }
 
 cudaError_t launch_vis_rope(bool bf16, const VisDesc<1024> &d, const RotArgs &r, const VisAngleFreqs &f,
-                            cudaStream_t s)
+                            cudaStream_t s, size_t budget)
 {
+    if (budget == 0) budget = kTmaBlockSmem;
     if (bf16)
-        return d.n_images <= 16 ? rope_impl<__nv_bfloat16, 16>(d, r, f, s) : rope_impl<__nv_bfloat16, 1024>(d, r, f, s);
-    return d.n_images <= 16 ? rope_impl<float, 16>(d, r, f, s) : rope_impl<float, 1024>(d, r, f, s);
+        return d.n_images <= 16 ? rope_impl<__nv_bfloat16, 16>(d, r, f, s, budget) : rope_impl<__nv_bfloat16, 1024>(d, r, f, s, budget);
+    return d.n_images <= 16 ? rope_impl<float, 16>(d, r, f, s, budget) : rope_impl<float, 1024>(d, r, f, s, budget);
 }
 
 }  // namespace ipe
