@@ -121,8 +121,11 @@ struct MropeTmaSrc {
     {
         tma_load_2d(stage + r.off_aux0, &r.taux0, r0, 0, bar);      // positions [3, P]
     }
-    __device__ __forceinline__ void angles(const TmaRotArgs &r, const unsigned char *stage, int c, long long row,
-                                           int lane, const CsSlot &cs) const
+    // `round` maps each cos / sin value before it is stored (the HF mode
+    // rounds to the activation dtype here, in the one write of the slot)
+    template <class Round>
+    __device__ __forceinline__ void angles_rounded(const TmaRotArgs &r, const unsigned char *stage, int c,
+                                                   long long row, int lane, const CsSlot &cs, Round round) const
     {
         const int32_t *spos = reinterpret_cast<const int32_t *>(stage + r.off_aux0);
         for (int j = lane; j < r.half; j += 32) {
@@ -132,10 +135,16 @@ struct MropeTmaSrc {
             const float angle = __fmul_rn(__int2float_rn(pos), a.inv[j]);
             float sn, cn;
             sincosf(angle, &sn, &cn);
-            cs.c[j] = cn;
+            sn = round(sn);
+            cs.c[j] = round(cn);
             cs.s[j] = sn;
             cs.ns[j] = -sn;
         }
+    }
+    __device__ __forceinline__ void angles(const TmaRotArgs &r, const unsigned char *stage, int c, long long row,
+                                           int lane, const CsSlot &cs) const
+    {
+        angles_rounded(r, stage, c, row, lane, cs, [](float v) { return v; });
     }
 };
 
@@ -200,6 +209,11 @@ struct HfTmaSrc : Base {
     __device__ __forceinline__ void angles(const TmaRotArgs &r, const unsigned char *stage, int c, long long row,
                                            int lane, const CsSlot &cs) const
     {
+        if constexpr (!Base::kHi) {
+            // the fused MRoPE rounds as it writes the slot
+            Base::angles_rounded(r, stage, c, row, lane, cs, [](float v) { return round_to_dtype<T>(v); });
+            return;
+        }
         Base::angles(r, stage, c, row, lane, cs);
         for (int j = lane; j < r.half; j += 32) {
             const float sn = round_to_dtype<T>(cs.s[j]);
