@@ -146,6 +146,34 @@ struct MropeTmaSrc {
     {
         angles_rounded(r, stage, c, row, lane, cs, [](float v) { return v; });
     }
+    // HF mode, bf16: cos, sin and -sin rounded to bf16 and stored as bf16x2
+    // words of the frequency pairs (2i, 2i+1), word i at the front of each
+    // array; lane j takes frequency j and its odd neighbour's values by
+    // shuffle, so the slot is written once.  -sin flips the sign bit (exact).
+    __device__ __forceinline__ void angles_bf16_words(const TmaRotArgs &r, const unsigned char *stage, int c,
+                                                      long long row, int lane, const CsSlot &cs) const
+    {
+        const int32_t *spos = reinterpret_cast<const int32_t *>(stage + r.off_aux0);
+        for (int j0 = 0; j0 < r.half; j0 += 32) {   // every lane takes part in the shuffles
+            const int j = j0 + lane;
+            float sn = 0.f, cn = 0.f;
+            if (j < r.half) {
+                const int ax = mrope_axis(j, a.section, a.interleaved);
+                const int pos = r.aux_tma ? spos[ax * r.P + c] : __ldg(a.positions + (long long)ax * a.T + row);
+                const float angle = __fmul_rn(__int2float_rn(pos), a.inv[j]);
+                sincosf(angle, &sn, &cn);
+            }
+            const uint32_t cb = __bfloat16_as_ushort(__float2bfloat16_rn(cn));
+            const uint32_t sb = __bfloat16_as_ushort(__float2bfloat16_rn(sn));
+            const uint32_t cb1 = __shfl_down_sync(0xffffffffu, cb, 1), sb1 = __shfl_down_sync(0xffffffffu, sb, 1);
+            if (!(lane & 1) && j < r.half) {
+                const int i = j >> 1;
+                reinterpret_cast<uint32_t *>(cs.c)[i] = cb | (cb1 << 16);
+                reinterpret_cast<uint32_t *>(cs.s)[i] = sb | (sb1 << 16);
+                reinterpret_cast<uint32_t *>(cs.ns)[i] = (sb ^ 0x8000u) | ((sb1 ^ 0x8000u) << 16);
+            }
+        }
+    }
 };
 
 struct TableTmaSrc {
@@ -210,8 +238,11 @@ struct HfTmaSrc : Base {
                                            int lane, const CsSlot &cs) const
     {
         if constexpr (!Base::kHi) {
-            // the fused MRoPE rounds as it writes the slot
-            Base::angles_rounded(r, stage, c, row, lane, cs, [](float v) { return round_to_dtype<T>(v); });
+            // the fused MRoPE rounds as it writes the slot (bf16: as words)
+            if constexpr (sizeof(T) == 2)
+                Base::angles_bf16_words(r, stage, c, row, lane, cs);
+            else
+                Base::angles_rounded(r, stage, c, row, lane, cs, [](float v) { return round_to_dtype<T>(v); });
             return;
         }
         Base::angles(r, stage, c, row, lane, cs);
@@ -231,9 +262,8 @@ struct HfTmaSrc : Base {
             // already), read that way by every chunk's packed products; each
             // round of 32 words is read in full before any of it is written.
             // Measured on B200 (large prefill): the HF table rotation 178.1
-            // -> 171.7 us; for the fused MRoPE's three arrays the extra pass
-            // per row cost more than it saved (172.2 -> 184.0 us), so its
-            // chunks pack their coefficients themselves.
+            // -> 171.7 us.  (The fused MRoPE packs as it writes instead: a
+            // second pass over its three arrays cost more than it saved.)
             float *arr[5] = {cs.c, cs.s, cs.ns, cs.ch, cs.sh};
             constexpr int NA = 5;
             const int nw = r.half / 2;
@@ -292,40 +322,22 @@ __device__ __forceinline__ void rotate_chunk(T *p, int half, int u, bool swap, c
     if constexpr (HF && sizeof(T) == 2) {
         // bf16 HF: every product and the sum as one packed bf16x2 operation
         // each, rounding where the fp32-then-cast steps do (mul_bf16x2 /
-        // add_bf16x2).  Tables (HI): the slot holds cos / sin as bf16x2
-        // words (the HF angle source packs them once per row), word o / 2
-        // for element o; otherwise the chunk packs its fp32 coefficients
-        // (exact: they hold bf16 values).
+        // add_bf16x2).  The slot holds cos / sin as bf16x2 words (the HF
+        // angle sources store them so, once per row), word o / 2 for
+        // element o.
         using W = Pack<uint32_t, VEC / 2>;
+        auto words = [&](const float *a) {
+            return ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(a - o) + o / 2);
+        };
+        const W C1w = words(C1), S1w = words(S1), S2w = words(S2);
+        const W C2w = HI ? words(C2) : C1w;
+        const W r1 = ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(p1));
+        const W r2 = ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(p2));
         W o1, o2;
-        if constexpr (HI) {
-            auto words = [&](const float *a) {
-                return ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(a - o) + o / 2);
-            };
-            const W C1w = words(C1), S1w = words(S1), S2w = words(S2), C2w = words(C2);
-            const W r1 = ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(p1));
-            const W r2 = ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(p2));
 #pragma unroll
-            for (int i = 0; i < VEC / 2; ++i) {
-                o1.v[i] = add_bf16x2(mul_bf16x2(r1.v[i], C1w.v[i]), mul_bf16x2(r2.v[i], S1w.v[i]));
-                o2.v[i] = add_bf16x2(mul_bf16x2(r2.v[i], C2w.v[i]), mul_bf16x2(r1.v[i], S2w.v[i]));
-            }
-        } else {
-            load_coef<VEC>(C1, c1);
-            load_coef<VEC>(S1, s1);
-            load_coef<VEC>(S2, s2);
-            const W r1 = ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(p1));
-            const W r2 = ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(p2));
-            auto bf2 = [](float2 f) {
-                const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
-                return *reinterpret_cast<const uint32_t *>(&b);
-            };
-#pragma unroll
-            for (int i = 0; i < VEC / 2; ++i) {
-                const uint32_t C1w = bf2(c1[i]), S1w = bf2(s1[i]), S2w = bf2(s2[i]);
-                o1.v[i] = add_bf16x2(mul_bf16x2(r1.v[i], C1w), mul_bf16x2(r2.v[i], S1w));
-                o2.v[i] = add_bf16x2(mul_bf16x2(r2.v[i], C1w), mul_bf16x2(r1.v[i], S2w));
-            }
+        for (int i = 0; i < VEC / 2; ++i) {
+            o1.v[i] = add_bf16x2(mul_bf16x2(r1.v[i], C1w.v[i]), mul_bf16x2(r2.v[i], S1w.v[i]));
+            o2.v[i] = add_bf16x2(mul_bf16x2(r2.v[i], C2w.v[i]), mul_bf16x2(r1.v[i], S2w.v[i]));
         }
         st_pack<uint32_t, VEC / 2>(reinterpret_cast<uint32_t *>(p1), o1);
         st_pack<uint32_t, VEC / 2>(reinterpret_cast<uint32_t *>(p2), o2);
