@@ -116,6 +116,7 @@ __device__ __forceinline__ void load_coef(const float *p, float2 *v)
 struct MropeTmaSrc {
     static constexpr bool kHi = false;
     static constexpr bool kHf = false;
+    static constexpr bool kTwoBlockBound = true;
     MropeAngles a;
     __device__ __forceinline__ void issue_aux(const TmaRotArgs &r, uint32_t stage, int r0, uint32_t bar) const
     {
@@ -179,6 +180,7 @@ struct MropeTmaSrc {
 struct TableTmaSrc {
     static constexpr bool kHi = true;
     static constexpr bool kHf = false;
+    static constexpr bool kTwoBlockBound = false;
     TableAngles a;
     __device__ __forceinline__ void issue_aux(const TmaRotArgs &r, uint32_t stage, int r0, uint32_t bar) const
     {
@@ -207,6 +209,7 @@ template <int MAXIMG>
 struct VisTmaSrc {
     static constexpr bool kHi = false;
     static constexpr bool kHf = false;
+    static constexpr bool kTwoBlockBound = true;
     VisDesc<MAXIMG> d;
     VisAngleFreqs f;
     __device__ __forceinline__ void issue_aux(const TmaRotArgs &, uint32_t, int, uint32_t) const {}
@@ -544,18 +547,37 @@ __device__ __forceinline__ void rotary_tma_block(const TmaRotArgs &a, const Src 
     if (lane == 0) bulk_wait_all();
 }
 
-// Two blocks per SM as the bound: ptxas then gives the consumers up to 113
-// registers (88-96 for bf16 rows), against 66-96 with the thread count alone.
-// Measured on B200: HF fused MRoPE 165.4 -> 161.2 us, Qwen3-Omni MRoPE
-// 121.1 -> 118.1 us, the one-call vision pair 129.7 -> 127.2 us (video) and
-// 71.5 -> 68.7 us (batch of 8); the vision rotary alone on the video 100.8
-// -> 103.5 us; the fused MRoPE and the table rotation unchanged.
+// Launch bounds by angle source (Src::kTwoBlockBound).  With two blocks per
+// SM as the bound ptxas gives the consumers up to 113 registers (88-96 for
+// bf16 rows), against 66-96 with the thread count alone.  Measured on B200:
+// HF fused MRoPE 165.4 -> 161.2 us, Qwen3-Omni MRoPE 121.1 -> 118.1 us, the
+// one-call vision pair 129.7 -> 127.2 us (video) and 71.5 -> 68.7 us (batch
+// of 8), the vision rotary alone on the video 100.8 -> 103.5 us, the fused
+// MRoPE unchanged; the table rotation slower (Omni 119.2 -> 128.3 us), so
+// table sources keep the thread count alone.
 template <typename T, int VEC, class Src>
 __global__ void __launch_bounds__(kTmaThreads, 2) rotary_tma_kernel(const __grid_constant__ TmaRotArgs a,
-                                                                 const __grid_constant__ Src src)
+                                                                    const __grid_constant__ Src src)
 {
     extern __shared__ unsigned char smem_raw[];
     rotary_tma_block<T, VEC, Src>(a, src, smem_raw, blockIdx.x, gridDim.x);
+}
+
+template <typename T, int VEC, class Src>
+__global__ void __launch_bounds__(kTmaThreads) rotary_tma_kernel_tb(const __grid_constant__ TmaRotArgs a,
+                                                                    const __grid_constant__ Src src)
+{
+    extern __shared__ unsigned char smem_raw[];
+    rotary_tma_block<T, VEC, Src>(a, src, smem_raw, blockIdx.x, gridDim.x);
+}
+
+template <typename T, int VEC, class Src>
+constexpr auto rotary_tma_entry()
+{
+    if constexpr (Src::kTwoBlockBound)
+        return &rotary_tma_kernel<T, VEC, Src>;
+    else
+        return &rotary_tma_kernel_tb<T, VEC, Src>;
 }
 
 // --------------------------------------------------------------- launch
@@ -627,7 +649,7 @@ cudaError_t launch_rotary_tma_vec(TmaRotArgs a, const Src &src, cudaStream_t s, 
 {
     tma_layout<T, VEC, Src>(a, first);
     const size_t smem = tma_smem_bytes(a, Src::kHi);
-    auto kern = rotary_tma_kernel<T, VEC, Src>;
+    auto kern = rotary_tma_entry<T, VEC, Src>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
