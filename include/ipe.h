@@ -439,9 +439,11 @@ int ipe_vis_rope2d(void *q, void *k, ipe_dtype dtype, int64_t n_patch, int heads
  * ipe_vis_pos_interp_rope2d -- ipe_vis_pos_interp and ipe_vis_rope2d on the
  * same images in one call: the interpolation runs on a second stream of the
  * library (one per device, created on first use) while the rotation runs on
- * `stream`, so the two kernels share the SMs; `stream` waits for both.  Same
- * results as the two calls.  Arguments as for the two calls; one dtype for
- * table, out, q and k.
+ * `stream`, so the two kernels share the SMs; `stream` waits for both.  The
+ * rotation is launched first, with shared-memory blocks small enough to
+ * leave room for two interpolation blocks on every SM where that still
+ * gives it a two-stage ring.  Same results as the two calls.  Arguments as
+ * for the two calls; one dtype for table, out, q and k.
  * ------------------------------------------------------------------------- */
 int ipe_vis_pos_interp_rope2d(const void *table, int grid_side, int hidden, void *out, void *q,
                               void *k, int heads, int head_dim, int64_t q_stride, int64_t k_stride,

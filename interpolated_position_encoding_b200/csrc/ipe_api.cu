@@ -901,9 +901,15 @@ int ipe_vis_pos_interp_rope2d(const void *table, int grid_side, int hidden, void
     if (int rc = aux_stream(&aux)) return rc;
     cudaEvent_t fork = aux->ring[aux->next++ % 64], join = aux->ring[aux->next++ % 64];
     const bool bf16 = dtype == IPE_BF16;
-    constexpr size_t kSmemPerSm = 233472, kBlockReserve = 1024;   // B200: 228 KB per SM, 1 KB per block
-    const size_t ib = vis_interp_block_smem(bf16, d, ia) + kBlockReserve;
-    const size_t budget = 2 * ib < kSmemPerSm ? (kSmemPerSm - 2 * ib) / 2 - kBlockReserve : 0;
+    // shared memory of an SM (228 KB on B200) and the 1 KB the runtime
+    // reserves per block
+    int dev = 0, per_sm = 0, reserve = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&reserve, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+        per_sm = reserve = 0;
+    const size_t ib = vis_interp_block_smem(bf16, d, ia) + (size_t)reserve;
+    const size_t budget = 2 * ib + reserve < (size_t)per_sm ? ((size_t)per_sm - 2 * ib) / 2 - reserve : 0;
     cudaError_t e;
     if ((e = cudaEventRecord(fork, s)) != cudaSuccess) return cuda_fail(e, "vis_pos_interp_rope2d fork");
     if ((e = launch_vis_rope(bf16, d, r, f, s, budget)) != cudaSuccess)
