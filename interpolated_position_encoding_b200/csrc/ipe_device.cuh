@@ -114,13 +114,25 @@ __device__ __forceinline__ void patch_row_col(const VisDesc<MAXIMG> &d, long lon
 {
     const VisImage &im = d.img[find_image(d, k)];
     const int m = d.merge;
-    const long long hw = (long long)im.h * im.w;
-    const int q = (int)((k - im.row0) % hw);       // index within the frame
-    const int blk = q / (m * m), r = q - blk * m * m;
+    // 32-bit from here: a request holds fewer than 2^31 patches (the host
+    // checks), so the patch's offset in its image and h * w fit in an int
+    const int hw = im.h * im.w;
+    const int q = (int)(k - im.row0) % hw;         // index within the frame
+    int blk, iy, ix;                                // merge block, row and column inside it
+    if (m == 2) {
+        blk = q >> 2;
+        iy = (q >> 1) & 1;
+        ix = q & 1;
+    } else {
+        blk = q / (m * m);
+        const int r = q - blk * m * m;
+        iy = r / m;
+        ix = r - iy * m;
+    }
     const int wb = im.w / m;
     const int by = blk / wb, bx = blk - by * wb;
-    row = by * m + r / m;
-    col = bx * m + r % m;
+    row = by * m + iy;
+    col = bx * m + ix;
 }
 
 // Sample point i of n on a grid of side G: floor index i0, clipped ceiling
