@@ -81,6 +81,7 @@ CASES = [  # (T, hq, hk, D, rot, section, dtype, stride_pad)
     (97, 8, 2, 128, 128, (24, 20, 20), "bf16", 0),
     (64, 4, 2, 64, 32, (6, 5, 5), "f32", 0),
     (45, 3, 1, 64, 64, (12, 10, 10), "bf16", 2),    # 4-byte token stride: the vector-load engine
+    (40, 4, 2, 256, 256, (44, 42, 42), "bf16", 0),  # 128 frequencies: several 32-word rounds of the bf16 slot
 ]
 
 
@@ -114,6 +115,23 @@ def test_apply_rotary_partial_hf_matches_torch(case):
     ipe.apply_rotary_partial(gq, gk, cos, sin, rounding="hf")
     ipe.device_status()
     assert torch.equal(gq, want_q) and torch.equal(gk, want_k)
+
+
+@pytest.mark.parametrize("rot", [64, 128, 256])
+def test_apply_rotary_partial_hf_unequal_halves(rot):
+    # tables whose two halves differ (the literal formula reads cos / sin at
+    # j + rot/2 for the second half): every coefficient array of the slot,
+    # bit for bit against torch running the listing's steps
+    T, hq, hk, D = 77, 5, 3, 256
+    g = torch.Generator("cuda").manual_seed(rot)
+    q = (torch.randn(T, hq, D, device="cuda", generator=g) * 2).to(torch.bfloat16)
+    k = (torch.randn(T, hk, D, device="cuda", generator=g) * 2).to(torch.bfloat16)
+    cos = torch.rand(T, rot, device="cuda", generator=g) * 2 - 1
+    sin = torch.rand(T, rot, device="cuda", generator=g) * 2 - 1
+    want_q, want_k = _torch_rotation(q.clone(), cos, sin, rot), _torch_rotation(k.clone(), cos, sin, rot)
+    ipe.apply_rotary_partial(q, k, cos, sin, rounding="hf")
+    ipe.device_status()
+    assert torch.equal(q, want_q) and torch.equal(k, want_k)
 
 
 def _torch_mrope_tables(pos, inv, section, interleaved, orc):
