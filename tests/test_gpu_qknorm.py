@@ -70,6 +70,7 @@ CASES = [  # (T, hq, hk, D, rot, section)
     (19, 2, 1, 64, 32, (6, 5, 5)),
     (8, 5, 3, 256, 256, (44, 42, 42)),
     (21, 3, 2, 128, 96, (16, 16, 16)),    # rotary slice of 12 (bf16) or 24 (fp32) chunks: one chunk per lane
+    (29, 3, 2, 64, 64, (12, 10, 10)),     # whole-row slice of 64 channels: 4 (bf16) or 8 (fp32) lanes per row
 ]
 
 
