@@ -552,9 +552,9 @@ __device__ __forceinline__ void rotary_tma_block(const TmaRotArgs &a, const Src 
 // bf16 rows), against 66-96 with the thread count alone.  Measured on B200:
 // HF fused MRoPE 165.4 -> 161.2 us, Qwen3-Omni MRoPE 121.1 -> 118.1 us, the
 // one-call vision pair 129.7 -> 127.2 us (video) and 71.5 -> 68.7 us (batch
-// of 8), the vision rotary alone on the video 100.8 -> 103.5 us, the fused
-// MRoPE unchanged; the table rotation slower (Omni 119.2 -> 128.3 us), so
-// table sources keep the thread count alone.
+// of 8), the vision rotary on the batch of 8 47.0 -> 45.1 us and on the video
+// unchanged (102 us), the fused MRoPE unchanged; the table rotation slower
+// (Omni 119.2 -> 128.3 us), so table sources keep the thread count alone.
 template <typename T, int VEC, class Src>
 __global__ void __launch_bounds__(kTmaThreads, 2) rotary_tma_kernel(const __grid_constant__ TmaRotArgs a,
                                                                     const __grid_constant__ Src src)
