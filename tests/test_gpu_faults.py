@@ -33,19 +33,30 @@ def test_status_is_clean_after_normal_launches():
     ipe.device_status()
 
 
-@pytest.mark.parametrize("path", ["mrope_apply", "vis_rope2d", "apply_rotary_partial"])
+@pytest.mark.parametrize("path", ["mrope_apply", "vis_rope2d", "apply_rotary_partial", "mrope_apply_wide"])
 def test_skipped_tile_times_out_and_recovers(path):
+    # the first three take a ring of three or more stages (a stage freed one
+    # row late); the wide rows (9 KB: 36 heads of 128 channels, rotated
+    # whole) take two stages at one block per SM (a stage freed at once)
     inv = ipe.rope_inv_freq(64, 1e7)
     pos, q, k = _text_case()
+    if path == "mrope_apply_wide":
+        rng = np.random.default_rng([6, 2048])
+        pos = torch.from_numpy(np.tile(np.arange(2048, dtype=np.int32), (3, 1))).cuda()
+        q = bf16_to_gpu(wl.normal_bf16(rng, (2048, 32, 128)))
+        k = bf16_to_gpu(wl.normal_bf16(rng, (2048, 4, 128)))
+        inv = ipe.rope_inv_freq(128, 1e6)
     grid = [(4, 16, 32)]
     rng = np.random.default_rng(11)
     vq = bf16_to_gpu(wl.normal_bf16(rng, (2048, 16, 72)))
     vk = bf16_to_gpu(wl.normal_bf16(rng, (2048, 16, 72)))
-    cos, sin = ipe.mrope_cos_sin(pos, inv, (11, 11, 10))
+    cos, sin = ipe.mrope_cos_sin(pos, inv, (11, 11, 10)) if path == "apply_rotary_partial" else (None, None)
 
     def run(a, b):
         if path == "mrope_apply":
             ipe.mrope_apply(a, b, pos, inv, (11, 11, 10))
+        elif path == "mrope_apply_wide":
+            ipe.mrope_apply(a, b, pos, inv, (24, 20, 20))
         elif path == "apply_rotary_partial":
             ipe.apply_rotary_partial(a, b, cos, sin)
         else:
