@@ -302,68 +302,98 @@ __device__ __forceinline__ float2 hf_pair(float2 a, float2 b)
     return make_float2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y));
 }
 
-// One chunk: elements [u VEC, u VEC + VEC) of the first half of head row `p`
-// and the matching chunk of the second half, rotated in place.  With `swap`
-// the lane reads (and writes) the second half first, which spreads
-// neighbouring rows over the banks; the formula is the same either way:
-//   x'[j]     = x[j] cos_j         - x[j+h] sin_j
-//   x'[j + h] = x[j + h] cos_{j+h} + x[j] sin_{j+h}
-// written as  w1 = v1 C1 + v2 S1,  w2 = v2 C2 + v1 S2  on the values v1, v2
-// at the first and second address, with C / S chosen (not computed) per lane.
+// The coefficients of one chunk: fp32 pairs, or bf16x2 words in the bf16 HF
+// mode (the slot holds words there).
 template <typename T, int VEC, bool HI, bool HF>
-__device__ __forceinline__ void rotate_chunk(T *p, int half, int u, bool swap, const CsSlot &cs)
+struct RotCoef {
+    static constexpr bool kWords = HF && sizeof(T) == 2;
+    Pack<uint32_t, VEC / 2> c1w, c2w, s1w, s2w;
+    float2 c1[VEC / 2], c2[VEC / 2], s1[VEC / 2], s2[VEC / 2];
+};
+
+// Coefficients of chunk u with the lane's swap bit: C1 / S1 for the values
+// at the first address, C2 / S2 for the second (see rotate_chunk_with).
+template <typename T, int VEC, bool HI, bool HF>
+__device__ __forceinline__ void load_rot_coef(const CsSlot &cs, int u, bool swap, RotCoef<T, VEC, HI, HF> &k)
 {
-    static_assert(VEC >= 2, "pairs");
-    T *pa = p + u * VEC, *pb = pa + half;
-    T *p1 = swap ? pb : pa, *p2 = swap ? pa : pb;
     const int o = u * VEC;
     const float *C1 = HI ? (swap ? cs.ch : cs.c) + o : cs.c + o;
     const float *C2 = HI ? (swap ? cs.c : cs.ch) + o : cs.c + o;
     const float *S1 = (swap ? (HI ? cs.sh : cs.s) : cs.ns) + o;
     const float *S2 = (swap ? cs.ns : (HI ? cs.sh : cs.s)) + o;
-    float2 v1[VEC / 2], v2[VEC / 2], c1[VEC / 2], c2[VEC / 2], s1[VEC / 2], s2[VEC / 2], w1[VEC / 2], w2[VEC / 2];
-    if constexpr (HF && sizeof(T) == 2) {
-        // bf16 HF: every product and the sum as one packed bf16x2 operation
-        // each, rounding where the fp32-then-cast steps do (mul_bf16x2 /
-        // add_bf16x2).  The slot holds cos / sin as bf16x2 words (the HF
-        // angle sources store them so, once per row), word o / 2 for
-        // element o.
-        using W = Pack<uint32_t, VEC / 2>;
+    if constexpr (RotCoef<T, VEC, HI, HF>::kWords) {
+        // word o / 2 of an array holds elements o and o + 1
         auto words = [&](const float *a) {
             return ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(a - o) + o / 2);
         };
-        const W C1w = words(C1), S1w = words(S1), S2w = words(S2);
-        const W C2w = HI ? words(C2) : C1w;
+        k.c1w = words(C1);
+        k.s1w = words(S1);
+        k.s2w = words(S2);
+        k.c2w = HI ? words(C2) : k.c1w;
+    } else {
+        load_coef<VEC>(C1, k.c1);
+        load_coef<VEC>(S1, k.s1);
+        load_coef<VEC>(S2, k.s2);
+        if constexpr (HI) load_coef<VEC>(C2, k.c2);
+    }
+}
+
+// One chunk: elements [u VEC, u VEC + VEC) of the first half of head row `p`
+// and the matching chunk of the second half, rotated in place with the
+// coefficients `k` of that chunk.  With `swap` the lane reads (and writes)
+// the second half first, which spreads neighbouring rows over the banks;
+// the formula is the same either way:
+//   x'[j]     = x[j] cos_j         - x[j+h] sin_j
+//   x'[j + h] = x[j + h] cos_{j+h} + x[j] sin_{j+h}
+// written as  w1 = v1 C1 + v2 S1,  w2 = v2 C2 + v1 S2  on the values v1, v2
+// at the first and second address, with C / S chosen (not computed) per lane.
+template <typename T, int VEC, bool HI, bool HF>
+__device__ __forceinline__ void rotate_chunk_with(T *p, int half, int u, bool swap, const RotCoef<T, VEC, HI, HF> &k)
+{
+    static_assert(VEC >= 2, "pairs");
+    T *pa = p + u * VEC, *pb = pa + half;
+    T *p1 = swap ? pb : pa, *p2 = swap ? pa : pb;
+    if constexpr (RotCoef<T, VEC, HI, HF>::kWords) {
+        // bf16 HF: every product and the sum as one packed bf16x2 operation
+        // each, rounding where the fp32-then-cast steps do (mul_bf16x2 /
+        // add_bf16x2).
+        using W = Pack<uint32_t, VEC / 2>;
         const W r1 = ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(p1));
         const W r2 = ld_pack<uint32_t, VEC / 2>(reinterpret_cast<const uint32_t *>(p2));
         W o1, o2;
 #pragma unroll
         for (int i = 0; i < VEC / 2; ++i) {
-            o1.v[i] = add_bf16x2(mul_bf16x2(r1.v[i], C1w.v[i]), mul_bf16x2(r2.v[i], S1w.v[i]));
-            o2.v[i] = add_bf16x2(mul_bf16x2(r2.v[i], C2w.v[i]), mul_bf16x2(r1.v[i], S2w.v[i]));
+            o1.v[i] = add_bf16x2(mul_bf16x2(r1.v[i], k.c1w.v[i]), mul_bf16x2(r2.v[i], k.s1w.v[i]));
+            o2.v[i] = add_bf16x2(mul_bf16x2(r2.v[i], k.c2w.v[i]), mul_bf16x2(r1.v[i], k.s2w.v[i]));
         }
         st_pack<uint32_t, VEC / 2>(reinterpret_cast<uint32_t *>(p1), o1);
         st_pack<uint32_t, VEC / 2>(reinterpret_cast<uint32_t *>(p2), o2);
         return;
     }
+    float2 v1[VEC / 2], v2[VEC / 2], w1[VEC / 2], w2[VEC / 2];
     load_pairs<T, VEC>(p1, v1);
     load_pairs<T, VEC>(p2, v2);
-    load_coef<VEC>(C1, c1);
-    load_coef<VEC>(S1, s1);
-    load_coef<VEC>(S2, s2);
-    if constexpr (HI) load_coef<VEC>(C2, c2);
 #pragma unroll
     for (int i = 0; i < VEC / 2; ++i) {
+        const float2 c2 = HI ? k.c2[i] : k.c1[i];
         if constexpr (HF) {
-            w1[i] = hf_pair<T>(mul2(v1[i], c1[i]), mul2(v2[i], s1[i]));
-            w2[i] = hf_pair<T>(mul2(v2[i], HI ? c2[i] : c1[i]), mul2(v1[i], s2[i]));
+            w1[i] = hf_pair<T>(mul2(v1[i], k.c1[i]), mul2(v2[i], k.s1[i]));
+            w2[i] = hf_pair<T>(mul2(v2[i], c2), mul2(v1[i], k.s2[i]));
         } else {
-            w1[i] = fma2(v1[i], c1[i], mul2(v2[i], s1[i]));
-            w2[i] = fma2(v2[i], HI ? c2[i] : c1[i], mul2(v1[i], s2[i]));
+            w1[i] = fma2(v1[i], k.c1[i], mul2(v2[i], k.s1[i]));
+            w2[i] = fma2(v2[i], c2, mul2(v1[i], k.s2[i]));
         }
     }
     store_pairs<T, VEC>(p1, w1);
     store_pairs<T, VEC>(p2, w2);
+}
+
+template <typename T, int VEC, bool HI, bool HF>
+__device__ __forceinline__ void rotate_chunk(T *p, int half, int u, bool swap, const CsSlot &cs)
+{
+    RotCoef<T, VEC, HI, HF> k;
+    load_rot_coef<T, VEC, HI, HF>(cs, u, swap, k);
+    rotate_chunk_with<T, VEC, HI, HF>(p, half, u, swap, k);
 }
 
 // Rotate the head rows of one tile row (q slot then k slot) in shared memory.
@@ -385,6 +415,18 @@ __device__ __forceinline__ void rotate_slots(const TmaRotArgs &a, unsigned char 
         // lanes sweep (head, chunk) with the chunk fastest; odd heads swap
         int h = lane / nvec, u = lane - h * nvec;
         const int dh = 32 / nvec, du = 32 - dh * nvec;
+        if (du == 0 && !(dh & 1)) {
+            // the lane keeps its chunk and its swap bit for every head it
+            // visits: the chunk's coefficients are read once per row
+            const bool swap = h & 1;
+            RotCoef<T, VEC, HI, HF> kc;
+            load_rot_coef<T, VEC, HI, HF>(cs, u, swap, kc);
+            for (; h < H; h += dh) {
+                T *p = h < a.hq ? q + h * rot : k + (h - a.hq) * rot;
+                rotate_chunk_with<T, VEC, HI, HF>(p, half, u, swap, kc);
+            }
+            return;
+        }
         while (h < H) {
             T *p = h < a.hq ? q + h * rot : k + (h - a.hq) * rot;
             rotate_chunk<T, VEC, HI, HF>(p, half, u, h & 1, cs);
