@@ -112,11 +112,37 @@ __device__ __forceinline__ void load_coef(const float *p, float2 *v)
 // ------------------------------------------------------------ angle sources
 // angles(): (cos, sin) of every frequency of tile row c (global row `row`)
 // into the warp's slot.  issue_aux(): TMA loads of per-tile side data.
+// Sources with kEarlyAngles also offer angles_early(), the same values for
+// frequencies lane + 32 i computed into registers from global memory only
+// (so a warp can work out its next row's while that row's stage is still
+// loading), and angles_store(), which writes them to the slot.
+
+constexpr int kEarlyRounds = 4;   // half <= 128 on the TMA path
+struct AngleRegs {
+    float c[kEarlyRounds], s[kEarlyRounds];
+};
+
+__device__ __forceinline__ void store_angle_regs(const TmaRotArgs &r, int lane, const CsSlot &cs, const AngleRegs &g)
+{
+#pragma unroll
+    for (int i = 0; i < kEarlyRounds; ++i) {
+        const int j = lane + 32 * i;
+        if (j < r.half) {
+            cs.c[j] = g.c[i];
+            cs.s[j] = g.s[i];
+            cs.ns[j] = -g.s[i];
+        }
+    }
+}
 
 struct MropeTmaSrc {
     static constexpr bool kHi = false;
     static constexpr bool kHf = false;
     static constexpr bool kTwoBlockBound = true;
+    // early angles would read the positions from global memory on the
+    // row's critical path instead of from the stage: slower (the large
+    // prefill 162.6 -> 164 us, Omni 107.6 -> 118 us)
+    static constexpr bool kEarlyAngles = false;
     MropeAngles a;
     __device__ __forceinline__ void issue_aux(const TmaRotArgs &r, uint32_t stage, int r0, uint32_t bar) const
     {
@@ -181,6 +207,7 @@ struct TableTmaSrc {
     static constexpr bool kHi = true;
     static constexpr bool kHf = false;
     static constexpr bool kTwoBlockBound = false;
+    static constexpr bool kEarlyAngles = false;
     TableAngles a;
     __device__ __forceinline__ void issue_aux(const TmaRotArgs &r, uint32_t stage, int r0, uint32_t bar) const
     {
@@ -210,26 +237,33 @@ struct VisTmaSrc {
     static constexpr bool kHi = false;
     static constexpr bool kHf = false;
     static constexpr bool kTwoBlockBound = true;
+    // the angles need only the row index: worked out a row ahead (the
+    // one-call vision pair 67.2 -> 65.9 us on the batch of 8 and 127.1 ->
+    // 125.3 us on the video; the rotary alone on the video 103.1 -> 104.2 us)
+    static constexpr bool kEarlyAngles = true;
     VisDesc<MAXIMG> d;
     VisAngleFreqs f;
-    __device__ __forceinline__ void issue_aux(const TmaRotArgs &, uint32_t, int, uint32_t) const {}
-    __device__ __forceinline__ void angles(const TmaRotArgs &r, const unsigned char *, int, long long row, int lane,
-                                           const CsSlot &cs) const
+    __device__ __forceinline__ void angles_early(const TmaRotArgs &r, long long row, int lane, AngleRegs &g) const
     {
         int prow, pcol;
         patch_row_col(d, row, prow, pcol);
         const int nf = f.nf;
-        for (int j = lane; j < r.half; j += 32) {
-            // angles [row * inv (nf) | col * inv (nf)]
-            const int v = j < nf ? prow : pcol;
-            const float angle = __fmul_rn(__int2float_rn(v), f.inv[j < nf ? j : j - nf]);
-            float sn, cn;
-            sincosf(angle, &sn, &cn);
-            cs.c[j] = cn;
-            cs.s[j] = sn;
-            cs.ns[j] = -sn;
+#pragma unroll
+        for (int i = 0; i < kEarlyRounds; ++i) {
+            const int j = lane + 32 * i;
+            if (j < r.half) {
+                // angles [row * inv (nf) | col * inv (nf)]
+                const int v = j < nf ? prow : pcol;
+                sincosf(__fmul_rn(__int2float_rn(v), f.inv[j < nf ? j : j - nf]), &g.s[i], &g.c[i]);
+            }
         }
     }
+    __device__ __forceinline__ void angles_store(const TmaRotArgs &r, int lane, const CsSlot &cs,
+                                                 const AngleRegs &g) const
+    {
+        store_angle_regs(r, lane, cs, g);
+    }
+    __device__ __forceinline__ void issue_aux(const TmaRotArgs &, uint32_t, int, uint32_t) const {}
 };
 
 // HF rounding mode of a source: its cos / sin cast to the activation dtype T
@@ -237,6 +271,7 @@ struct VisTmaSrc {
 template <class Base, typename T>
 struct HfTmaSrc : Base {
     static constexpr bool kHf = true;
+    static constexpr bool kEarlyAngles = false;
     __device__ __forceinline__ void angles(const TmaRotArgs &r, const unsigned char *stage, int c, long long row,
                                            int lane, const CsSlot &cs) const
     {
@@ -546,6 +581,13 @@ __device__ __forceinline__ void rotary_tma_block(const TmaRotArgs &a, const Src 
     const bool late = S >= 3;
     int pending = -1;   // stage whose row store may still be reading it
     long long it = 0;
+    // Sources with kEarlyAngles: a warp works out its next row's (cos, sin)
+    // into registers while its current row's store reads the stage and the
+    // next stage loads, then only writes them to its slot.
+    AngleRegs ang;
+    if constexpr (Src::kEarlyAngles) {
+        if (bid < ntiles && bid * a.P + c < a.rows) src.angles_early(a, bid * a.P + c, lane, ang);
+    }
     for (long long tile = bid; tile < ntiles; tile += nb, ++it) {
         const int s = (int)(it % S);
         bool ok = mbar_wait(smem_addr(&bars[s]), (uint32_t)((it / S) & 1), a.wait_limit, abort);
@@ -562,7 +604,10 @@ __device__ __forceinline__ void rotary_tma_block(const TmaRotArgs &a, const Src 
         if (row < a.rows) {
             unsigned char *sq = stage + (size_t)c * a.slot_q;
             unsigned char *sk = stage + a.off_k + (size_t)c * a.slot_k;
-            src.angles(a, stage, c, row, lane, cs);
+            if constexpr (Src::kEarlyAngles)
+                src.angles_store(a, lane, cs, ang);
+            else
+                src.angles(a, stage, c, row, lane, cs);
             __syncwarp();
             rotate_slots<T, VEC, Src::kHi, Src::kHf>(a, sq, sk, lane, cs);
             fence_proxy_async_smem();
@@ -585,6 +630,11 @@ __device__ __forceinline__ void rotary_tma_block(const TmaRotArgs &a, const Src 
             }
         }
         pending = s;
+        if constexpr (Src::kEarlyAngles) {
+            // the next row's angles, after the stage release
+            const long long nrow = (tile + nb) * a.P + c;
+            if (tile + nb < ntiles && nrow < a.rows) src.angles_early(a, nrow, lane, ang);
+        }
     }
     if (lane == 0) bulk_wait_all();
 }
