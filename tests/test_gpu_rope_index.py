@@ -1,7 +1,7 @@
 """Position table on the device (through the C ABI) against the oracle.
 
 Integer work: positions and deltas must match the oracle bit for bit.  Inputs
-that only the device can judge (a run longer or shorter than its grid, grids
+that only the device can detect (a run longer or shorter than its grid, grids
 that run out, unknown types) must be reported through the device status word.
 """
 import numpy as np
