@@ -60,6 +60,7 @@ struct MropeAngles {               // angle = fl32(pos[axis(j)]) * inv[j]
     int section[3];
     int interleaved;
     float inv[kMaxHalf];
+    int row_shift = 0;             // rotary rows per token = 1 << row_shift (the TMA ring's head split)
 };
 
 struct TableAngles {               // cos / sin read from [T, 2*half] tables

@@ -146,7 +146,16 @@ struct MropeTmaSrc {
     MropeAngles a;
     __device__ __forceinline__ void issue_aux(const TmaRotArgs &r, uint32_t stage, int r0, uint32_t bar) const
     {
-        tma_load_2d(stage + r.off_aux0, &r.taux0, r0, 0, bar);      // positions [3, P]
+        tma_load_2d(stage + r.off_aux0, &r.taux0, r0 >> a.row_shift, 0, bar);   // positions [3, P >> row_shift]
+    }
+    // position on axis ax of the token of tile row c (global row `row`):
+    // from the stage when the positions came with it, else from memory
+    __device__ __forceinline__ int pos_of(const TmaRotArgs &r, const unsigned char *stage, int c, long long row,
+                                          int ax) const
+    {
+        const int32_t *spos = reinterpret_cast<const int32_t *>(stage + r.off_aux0);
+        return r.aux_tma ? spos[ax * (r.P >> a.row_shift) + (c >> a.row_shift)]
+                         : __ldg(a.positions + (long long)ax * a.T + (row >> a.row_shift));
     }
     // `round` maps each cos / sin value before it is stored (the HF mode
     // rounds to the activation dtype here, in the one write of the slot)
@@ -154,10 +163,8 @@ struct MropeTmaSrc {
     __device__ __forceinline__ void angles_rounded(const TmaRotArgs &r, const unsigned char *stage, int c,
                                                    long long row, int lane, const CsSlot &cs, Round round) const
     {
-        const int32_t *spos = reinterpret_cast<const int32_t *>(stage + r.off_aux0);
         for (int j = lane; j < r.half; j += 32) {
-            const int ax = mrope_axis(j, a.section, a.interleaved);
-            const int pos = r.aux_tma ? spos[ax * r.P + c] : __ldg(a.positions + (long long)ax * a.T + row);
+            const int pos = pos_of(r, stage, c, row, mrope_axis(j, a.section, a.interleaved));
             // fl32(fl32(pos) * inv_freq[j]): one rounded product, no contraction
             const float angle = __fmul_rn(__int2float_rn(pos), a.inv[j]);
             float sn, cn;
@@ -180,13 +187,11 @@ struct MropeTmaSrc {
     __device__ __forceinline__ void angles_bf16_words(const TmaRotArgs &r, const unsigned char *stage, int c,
                                                       long long row, int lane, const CsSlot &cs) const
     {
-        const int32_t *spos = reinterpret_cast<const int32_t *>(stage + r.off_aux0);
         for (int j0 = 0; j0 < r.half; j0 += 32) {   // every lane takes part in the shuffles
             const int j = j0 + lane;
             float sn = 0.f, cn = 0.f;
             if (j < r.half) {
-                const int ax = mrope_axis(j, a.section, a.interleaved);
-                const int pos = r.aux_tma ? spos[ax * r.P + c] : __ldg(a.positions + (long long)ax * a.T + row);
+                const int pos = pos_of(r, stage, c, row, mrope_axis(j, a.section, a.interleaved));
                 const float angle = __fmul_rn(__int2float_rn(pos), a.inv[j]);
                 sincosf(angle, &sn, &cn);
             }
