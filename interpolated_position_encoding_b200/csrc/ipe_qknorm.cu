@@ -25,6 +25,12 @@
 namespace ipe {
 
 constexpr int kQkWarps = 8;
+// Pair layout: row groups in flight per warp (U) and blocks per SM.
+// Measured on B200 (Qwen3-Omni, T = 32768, 36 rows of 128 channels): one
+// group at four blocks per SM 106.2 us, two at three 103.7 us, three at
+// three 101.7 us, three at two 100.7 us; four or six (rows padded to 48)
+// 113 us.
+constexpr int qk_pair_min_blocks(int u) { return u >= 3 ? 2 : 3; }
 // Rows in flight per lane and blocks per SM, by lanes per row (measured:
 // 256-channel bf16 rows prefer four rows at three blocks per SM, narrower
 // rows two rows at four blocks per SM).
@@ -292,8 +298,8 @@ static void qk_grid(QkNormArgs &m, int unit, int per_sm, long long &blocks)
 // lanes instead of D / EC.  The norm, cast, weight product and rotation are
 // those of the kernels above; only the order in which the row's squares are
 // summed differs.
-template <typename T, int LPR>
-__global__ void __launch_bounds__(32 * kQkWarps, 4)
+template <typename T, int LPR, int U>
+__global__ void __launch_bounds__(32 * kQkWarps, qk_pair_min_blocks(U))
     qk_norm_mrope_pair_kernel(const __grid_constant__ QkNormArgs n, const __grid_constant__ MropeAngles a)
 {
     constexpr int EC = QkElem<T>::EC;
@@ -338,9 +344,14 @@ __global__ void __launch_bounds__(32 * kQkWarps, 4)
                 for (int i = 0; i < 4; ++i) v[k].v[i] = 0u;
         }
     };
+    // U slots of row groups: slot u holds row h0 + u RPW + sub of the token
+    // in hand and, as soon as it is taken for the norm, loads the row it will
+    // hold next (U RPW rows further, or the next token's), so U groups of
+    // loads stay in flight per warp
     long long t = gw / n.groups;
-    Pack<uint32_t, 4> x[2];
-    load_row(t, hbeg + sub, x);
+    Pack<uint32_t, 4> x[U][2];
+#pragma unroll
+    for (int u = 0; u < U; ++u) load_row(t, hbeg + u * RPW + sub, x[u]);
     for (; t < n.T; t += tstride) {
         // (cos, sin) of every frequency of token t
         for (int j = lane; j < HALF; j += 32) {
@@ -356,16 +367,17 @@ __global__ void __launch_bounds__(32 * kQkWarps, 4)
             co[i] = make_float2(cs_c[e0 + 2 * i], cs_c[e0 + 2 * i + 1]);
             sn[i] = make_float2(cs_s[e0 + 2 * i], cs_s[e0 + 2 * i + 1]);
         }
-        for (int h0 = hbeg; h0 < hend; h0 += RPW) {
-            const int h = h0 + sub;
-            Pack<uint32_t, 4> nx[2];
-            if (h0 + RPW < hend)
-                load_row(t, h + RPW, nx);
-            else
-                load_row(t + tstride, hbeg + sub, nx);
+        for (int h0 = hbeg; h0 < hend; h0 += RPW * U)
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int h = h0 + u * RPW + sub;
             float2 xa[NP], xb[NP];
-            chunk_to_pairs<T>(x[0].v, xa);
-            chunk_to_pairs<T>(x[1].v, xb);
+            chunk_to_pairs<T>(x[u][0].v, xa);
+            chunk_to_pairs<T>(x[u][1].v, xb);
+            if (h0 + RPW * U < hend)
+                load_row(t, h + RPW * U, x[u]);
+            else
+                load_row(t + tstride, hbeg + u * RPW + sub, x[u]);
             float2 acc = mul2(xa[0], xa[0]);
 #pragma unroll
             for (int i = 1; i < NP; ++i) acc = fma2(xa[i], xa[i], acc);
@@ -419,27 +431,36 @@ __global__ void __launch_bounds__(32 * kQkWarps, 4)
                 st_pack<uint32_t, 4>(p, pa);
                 st_pack<uint32_t, 4>(p + kHalfWords, pb);
             }
-            x[0] = nx[0];
-            x[1] = nx[1];
         }
         __syncwarp();
     }
 }
 
-template <typename T, int LPR>
-static cudaError_t qk_launch_pair(const QkNormArgs &n, const MropeAngles &a, cudaStream_t s)
+template <typename T, int LPR, int U>
+static cudaError_t qk_launch_pair_u(const QkNormArgs &n, const MropeAngles &a, cudaStream_t s)
 {
     constexpr int EC = QkElem<T>::EC;
     const size_t smem = 2 * (size_t)2 * LPR * EC * sizeof(T) + (size_t)kQkWarps * 2 * n.half_pad * sizeof(float);
-    auto kern = qk_norm_mrope_pair_kernel<T, LPR>;
+    auto kern = qk_norm_mrope_pair_kernel<T, LPR, U>;
     int per_sm = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32 * kQkWarps, smem);
     if (e != cudaSuccess) return e;
     QkNormArgs m = n;
     long long blocks = 0;
-    qk_grid(m, 32 / LPR, per_sm, blocks);
+    qk_grid(m, (32 / LPR) * U, per_sm, blocks);
     kern<<<(unsigned)blocks, 32 * kQkWarps, smem, s>>>(m, a);
     return cudaGetLastError();
+}
+
+// Three groups in flight unless two pad the head rows less (the rows past
+// the last are zeros that are never stored, but still cost their work).
+template <typename T, int LPR>
+static cudaError_t qk_launch_pair(const QkNormArgs &n, const MropeAngles &a, cudaStream_t s)
+{
+    constexpr int RPW = 32 / LPR;
+    const int H = n.hq + n.hk;
+    auto pad = [&](int u) { return (H + RPW * u - 1) / (RPW * u) * (RPW * u) - H; };
+    return pad(2) < pad(3) ? qk_launch_pair_u<T, LPR, 2>(n, a, s) : qk_launch_pair_u<T, LPR, 3>(n, a, s);
 }
 
 template <typename T, int LPR, int CPL, int MINB>

@@ -71,6 +71,8 @@ CASES = [  # (T, hq, hk, D, rot, section)
     (8, 5, 3, 256, 256, (44, 42, 42)),
     (21, 3, 2, 128, 96, (16, 16, 16)),    # rotary slice of 12 (bf16) or 24 (fp32) chunks: one chunk per lane
     (29, 3, 2, 64, 64, (12, 10, 10)),     # whole-row slice of 64 channels: 4 (bf16) or 8 (fp32) lanes per row
+    (23, 9, 3, 128, 128, (24, 20, 20)),   # 12 whole rows: three row groups in flight per warp (both dtypes)
+    (17, 10, 2, 64, 64, (12, 10, 10)),    # 12 rows of 64: two groups in flight (bf16), three (fp32)
 ]
 
 
@@ -103,22 +105,33 @@ def test_qk_norm_mrope_small(case, dtype, orc):
                  f"{case} {dtype} {nm}")
 
 
-def test_qk_norm_mrope_long_sequence(orc):
-    # 16411 tokens (past the length where rows of four 16-byte chunks per
-    # lane take the two-blocks-per-SM form; not a multiple of the warp
-    # count), D = 256 with a 64-channel rotary slice: every token compared
-    T, hq, hk, D, rot, section = 16411, 5, 3, 256, 64, (11, 11, 10)
-    rng = GEN(16411)
-    q, k = wl.normal_bf16(rng, (T, hq, D), 3.0), wl.normal_bf16(rng, (T, hk, D), 3.0)
-    wq, wk = wl.normal_bf16(rng, (D,), 0.5), wl.normal_bf16(rng, (D,), 0.5)
+LONG = [  # (T, hq, hk, D, rot, section, dtype, theta)
+    # past the length where rows of four 16-byte chunks per lane take the
+    # two-blocks-per-SM form; not a multiple of the warp count
+    (16411, 5, 3, 256, 64, (11, 11, 10), "bf16", 1e7),
+    # whole rows, several tokens per warp: two row groups in flight (bf16)
+    # and three (fp32)
+    (20011, 4, 4, 128, 128, (24, 20, 20), "bf16", 1e6),
+    (12007, 9, 3, 128, 128, (24, 20, 20), "f32", 1e6),
+]
+
+
+@pytest.mark.parametrize("case", LONG, ids=lambda c: "T%d_h%d_%d_D%d_r%d" % c[:5])
+def test_qk_norm_mrope_long_sequence(case, orc):
+    # every token compared
+    T, hq, hk, D, rot, section, dtype, theta = case
+    rng = GEN(T)
+    gen = wl.normal_bf16 if dtype == "bf16" else wl.normal_f32
+    q, k = gen(rng, (T, hq, D), 3.0), gen(rng, (T, hk, D), 3.0)
+    wq, wk = gen(rng, (D,), 0.5), gen(rng, (D,), 0.5)
     p = rng.integers(0, 200000, (3, T)).astype(np.int32)
-    gq, gk = to_gpu(q, "bf16"), to_gpu(k, "bf16")
-    ipe.qk_norm_mrope(gq, gk, to_gpu(wq, "bf16"), to_gpu(wk, "bf16"), torch.from_numpy(p).cuda(),
-                      ipe.rope_inv_freq(rot, 1e7), section, True, eps=1e-6)
-    oinv = orc.rope_inv_freq(rot, 1e7)
+    gq, gk = to_gpu(q, dtype), to_gpu(k, dtype)
+    ipe.qk_norm_mrope(gq, gk, to_gpu(wq, dtype), to_gpu(wk, dtype), torch.from_numpy(p).cuda(),
+                      ipe.rope_inv_freq(rot, theta), section, True, eps=1e-6)
+    oinv = orc.rope_inv_freq(rot, theta)
     for nm, x, w, g in (("q", q, wq, gq), ("k", k, wk, gk)):
-        check_qk(gpu_to_f64(g), host_f64(x, "bf16"), host_f64(w, "bf16"), 1e-6, "bf16", p, oinv, section, True, orc,
-                 f"long {nm}")
+        check_qk(gpu_to_f64(g), host_f64(x, dtype), host_f64(w, dtype), 1e-6, dtype, p, oinv, section, True, orc,
+                 f"long {case[:5]} {nm}")
 
 
 @pytest.mark.parametrize("name,layout", [("text_t4096_qwen35", "interleaved"), ("text_t32768_omni", "chunked"),
