@@ -31,6 +31,21 @@ struct VisDesc {
     VisImage img[MAXIMG];
 };
 
+// The first MAXIMG images of a descriptor (MAXIMG = 16: a 400-byte kernel
+// parameter block instead of about 25 KB, for calls of at most 16 images).
+template <int MAXIMG>
+inline VisDesc<MAXIMG> shrink(const VisDesc<1024> &d)
+{
+    VisDesc<MAXIMG> s;
+    s.n_images = d.n_images;
+    s.merge = d.merge;
+    s.grid_side = d.grid_side;
+    s.n_strips = d.n_strips;
+    s.n_patch = d.n_patch;
+    for (int i = 0; i < d.n_images && i < MAXIMG; ++i) s.img[i] = d.img[i];
+    return s;
+}
+
 // Interpolation output / table of one call.
 struct InterpArgs {
     const void *table;   // [G*G, hidden]

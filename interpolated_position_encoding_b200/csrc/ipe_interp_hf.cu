@@ -118,8 +118,8 @@ __device__ __forceinline__ uint4 hf_blend(const uint4 (&c)[4], const uint4 &w)
     }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(32 * kHfWarps) vis_interp_hf_kernel(const __grid_constant__ VisDesc<1024> d,
+template <typename T, int MAXIMG>
+__global__ void __launch_bounds__(32 * kHfWarps) vis_interp_hf_kernel(const __grid_constant__ VisDesc<MAXIMG> d,
                                                                       const __grid_constant__ InterpArgs ia, int parts)
 {
     __shared__ HfPatch plan[kHfPlanCache];
@@ -186,10 +186,18 @@ cudaError_t launch_vis_interp_hf(bool bf16, const VisDesc<1024> &d, const Interp
     const unsigned gy = (unsigned)((ia.hidden / ec + 31) / 32);
     const int parts = hf_parts(d, (long long)d.n_strips * gy);
     const dim3 grid((unsigned)d.n_strips, gy, (unsigned)parts);
-    if (bf16)
-        vis_interp_hf_kernel<__nv_bfloat16><<<grid, 32 * kHfWarps, 0, s>>>(d, ia, parts);
-    else
-        vis_interp_hf_kernel<float><<<grid, 32 * kHfWarps, 0, s>>>(d, ia, parts);
+    const bool small = d.n_images <= 16;
+    if (bf16) {
+        if (small)
+            vis_interp_hf_kernel<__nv_bfloat16, 16><<<grid, 32 * kHfWarps, 0, s>>>(shrink<16>(d), ia, parts);
+        else
+            vis_interp_hf_kernel<__nv_bfloat16, 1024><<<grid, 32 * kHfWarps, 0, s>>>(d, ia, parts);
+    } else {
+        if (small)
+            vis_interp_hf_kernel<float, 16><<<grid, 32 * kHfWarps, 0, s>>>(shrink<16>(d), ia, parts);
+        else
+            vis_interp_hf_kernel<float, 1024><<<grid, 32 * kHfWarps, 0, s>>>(d, ia, parts);
+    }
     return cudaGetLastError();
 }
 

@@ -236,18 +236,6 @@ static bool interp_wide(const InterpArgs &ia)
 }
 
 // ------------------------------------------------------------- launches
-template <int MAXIMG>
-static VisDesc<MAXIMG> shrink(const VisDesc<1024> &d)
-{
-    VisDesc<MAXIMG> s;
-    s.n_images = d.n_images;
-    s.merge = d.merge;
-    s.grid_side = d.grid_side;
-    s.n_strips = d.n_strips;
-    s.n_patch = d.n_patch;
-    for (int i = 0; i < d.n_images && i < MAXIMG; ++i) s.img[i] = d.img[i];
-    return s;
-}
 
 template <int MAXIMG>
 static cudaError_t plan_impl(const VisDesc<1024> &d, int32_t *idx4, float *w4, int32_t *rowcol, cudaStream_t s)
