@@ -805,9 +805,33 @@ def _time_flushed(torch, stream, fn, reps, flush):
     return total / reps
 
 
+def _time_resident(torch, stream, fn, reps):
+    """Mean device time of fn over back-to-back calls with nothing flushed,
+    so inputs and outputs that fit stay in L2 between calls.  The stream is
+    held by a device sleep while the host queues the calls, so the time is
+    the GPU's, not the host's launch rate."""
+    fn()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(5_000_000)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+# Algorithmic bytes below which a call's tensors can stay in the 126 MB L2:
+# such calls are reported both flushed and resident.
+L2_RESIDENT_BYTES = 64 << 20
+
+
 def per_workload(ipe, dev, stream, peak, reps):
     """Every kernel of the library on each of the five workloads (L2 flushed
-    between timed calls): ms, algorithmic GB/s and fraction of the peak."""
+    between timed calls): ms, algorithmic GB/s and fraction of the peak;
+    calls small enough to stay in L2 also carry the same figures timed back
+    to back without a flush ("resident")."""
     import numpy as np
     import torch
     import workloads as wl
@@ -822,6 +846,12 @@ def per_workload(ipe, dev, stream, peak, reps):
     def entry(ms, nbytes):
         return {"ms": ms, "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / peak}
 
+    def timed(fn, nbytes):
+        e = entry(_time_flushed(torch, stream, fn, reps, flush), nbytes)
+        if nbytes < L2_RESIDENT_BYTES:
+            e["resident"] = entry(_time_resident(torch, stream, fn, reps), nbytes)
+        return e
+
     for name, w in wl.WORKLOADS.items():
         r = {}
         if w.vision is not None:
@@ -833,15 +863,12 @@ def per_workload(ipe, dev, stream, peak, reps):
             out = torch.empty(N, v.hidden, dtype=table.dtype, device=dev)
             ib = algorithmic_bytes_vision(v)
             rb = 2 * N * v.heads * v.head_dim * eb * 2
-            r["vis_pos_interp"] = entry(_time_flushed(
-                torch, stream, lambda: ipe.vis_pos_interp(table, v.grid_thw, v.merge, out=out, stream=stream), reps,
-                flush), ib)
-            r["vis_rope2d"] = entry(_time_flushed(
-                torch, stream, lambda: ipe.vis_rope2d(q, k, v.grid_thw, v.merge, v.theta, stream=stream), reps,
-                flush), rb)
-            r["vis_pos_interp_rope2d"] = entry(_time_flushed(
-                torch, stream, lambda: ipe.vis_pos_interp_rope2d(table, v.grid_thw, q, k, v.merge, v.theta, out=out,
-                                                                 stream=stream), reps, flush), ib + rb)
+            r["vis_pos_interp"] = timed(
+                lambda: ipe.vis_pos_interp(table, v.grid_thw, v.merge, out=out, stream=stream), ib)
+            r["vis_rope2d"] = timed(lambda: ipe.vis_rope2d(q, k, v.grid_thw, v.merge, v.theta, stream=stream), rb)
+            r["vis_pos_interp_rope2d"] = timed(
+                lambda: ipe.vis_pos_interp_rope2d(table, v.grid_thw, q, k, v.merge, v.theta, out=out, stream=stream),
+                ib + rb)
             r["patches"] = N
         if w.text is not None:
             t = w.text
@@ -854,21 +881,18 @@ def per_workload(ipe, dev, stream, peak, reps):
             rot = (t.hq + t.hk) * t.T * t.rot_dim * 2 * 2
             for layout in t.layouts:
                 il = layout == "interleaved"
-                r[f"mrope_apply/{layout}"] = entry(_time_flushed(
-                    torch, stream, lambda: ipe.mrope_apply(Q, K, pos, inv, t.section, il, stream=stream), reps,
-                    flush), rot + 3 * t.T * 4)
-                r[f"mrope_cos_sin/{layout}"] = entry(_time_flushed(
-                    torch, stream, lambda: ipe.mrope_cos_sin(pos, inv, t.section, il, cos, sin, stream=stream), reps,
-                    flush), 3 * t.T * 4 + 2 * t.T * t.rot_dim * 4)
-                r[f"apply_rotary_partial/{layout}"] = entry(_time_flushed(
-                    torch, stream, lambda: ipe.apply_rotary_partial(Q, K, cos, sin, stream=stream), reps, flush),
-                    rot + 2 * t.T * t.rot_dim * 4)
+                r[f"mrope_apply/{layout}"] = timed(
+                    lambda: ipe.mrope_apply(Q, K, pos, inv, t.section, il, stream=stream), rot + 3 * t.T * 4)
+                r[f"mrope_cos_sin/{layout}"] = timed(
+                    lambda: ipe.mrope_cos_sin(pos, inv, t.section, il, cos, sin, stream=stream),
+                    3 * t.T * 4 + 2 * t.T * t.rot_dim * 4)
+                r[f"apply_rotary_partial/{layout}"] = timed(
+                    lambda: ipe.apply_rotary_partial(Q, K, cos, sin, stream=stream), rot + 2 * t.T * t.rot_dim * 4)
                 if layout == t.layouts[0]:
                     wq = torch.ones(t.head_dim, dtype=torch.bfloat16, device=dev)
                     full = (t.hq + t.hk) * t.T * t.head_dim * 2 * 2 + 3 * t.T * 4 + 2 * t.head_dim * 2
-                    r["qk_norm_mrope"] = entry(_time_flushed(
-                        torch, stream, lambda: ipe.qk_norm_mrope(Q, K, wq, wq, pos, inv, t.section, il, stream=stream),
-                        reps, flush), full)
+                    r["qk_norm_mrope"] = timed(
+                        lambda: ipe.qk_norm_mrope(Q, K, wq, wq, pos, inv, t.section, il, stream=stream), full)
             r["tokens"] = t.T
         res[name] = r
         torch.cuda.empty_cache()
