@@ -917,7 +917,8 @@ def _segment_types(segments, merge):
 
 def next_rows(ipe, dev, stream, peak, reps):
     """The rows beyond the path: the device position table (get_rope_index)
-    and the decode step, L2 flushed between timed calls."""
+    and the decode step, L2 flushed between timed calls (and, when they fit
+    in L2, also back to back: "resident")."""
     import numpy as np
     import torch
     import workloads as wl
@@ -926,6 +927,12 @@ def next_rows(ipe, dev, stream, peak, reps):
 
     def entry(ms, nbytes, **kw):
         return {"ms": ms, "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / peak, **kw}
+
+    def timed(fn, nbytes, **kw):
+        e = entry(_time_flushed(torch, stream, fn, reps, flush), nbytes, **kw)
+        if nbytes < L2_RESIDENT_BYTES:
+            e["resident"] = entry(_time_resident(torch, stream, fn, reps), nbytes)
+        return e
 
     # position table: the prefill request (B = 1) and a padded batch of 16
     t = wl.WORKLOADS[WORKLOAD].text
@@ -947,9 +954,9 @@ def next_rows(ipe, dev, stream, peak, reps):
         dl = torch.empty(Bn, dtype=torch.int32, device=dev)
         ws = torch.empty(ipe.rope_index_workspace_bytes(Bn, Ln, 0, vg.shape[0]), dtype=torch.uint8, device=dev)
         nbytes = Bn * Ln * 4 * (1 + (mk is not None) + 3) + Bn * 4
-        ms = _time_flushed(torch, stream, lambda: ipe.mrope_rope_index(gty, None, gvg, gmk, t.merge, posb, dl, ws,
-                                                                       stream=stream), reps, flush)
-        res[f"rope_index/{name}"] = entry(ms, nbytes, slots=Bn * Ln, launches=2)
+        res[f"rope_index/{name}"] = timed(
+            lambda: ipe.mrope_rope_index(gty, None, gvg, gmk, t.merge, posb, dl, ws, stream=stream), nbytes,
+            slots=Bn * Ln, launches=2)
 
     # decode step with the prefill model's heads: norm, rotation, cache write
     D, hq, hk, rot = t.head_dim, t.hq, t.hk, t.rot_dim
@@ -967,10 +974,9 @@ def next_rows(ipe, dev, stream, peak, reps):
         dl = torch.randint(-2000, 0, (B,), dtype=torch.int32, device=dev, generator=g)
         sm = (torch.arange(B, device=dev, dtype=torch.int64) * 1024 + seq.long() % 1024).contiguous()
         nbytes = B * (hq + hk) * D * 2 * 2 + B * hk * D * 2 * 3 + B * 16 + 2 * D * 2
-        ms = _time_flushed(torch, stream, lambda: ipe.mrope_decode(q, k, seq, inv, dl, v=v, q_weight=wq, k_weight=wq,
-                                                                   k_cache=kc, v_cache=vc, slot_mapping=sm,
-                                                                   stream=stream), reps, flush)
-        res[f"mrope_decode/b{B}_norm_cache"] = entry(ms, nbytes, tokens=B, launches=1)
+        res[f"mrope_decode/b{B}_norm_cache"] = timed(
+            lambda: ipe.mrope_decode(q, k, seq, inv, dl, v=v, q_weight=wq, k_weight=wq, k_cache=kc, v_cache=vc,
+                                     slot_mapping=sm, stream=stream), nbytes, tokens=B, launches=1)
         del kc, vc
     # HF rounding mode: interpolation (four-corner sum) and the fused MRoPE
     for name in ("prefill_t131072_video", "vision_batch8_bf16"):
