@@ -367,69 +367,70 @@ __global__ void __launch_bounds__(32 * kQkWarps, qk_pair_min_blocks(U))
             co[i] = make_float2(cs_c[e0 + 2 * i], cs_c[e0 + 2 * i + 1]);
             sn[i] = make_float2(cs_s[e0 + 2 * i], cs_s[e0 + 2 * i + 1]);
         }
-        for (int h0 = hbeg; h0 < hend; h0 += RPW * U)
+        for (int h0 = hbeg; h0 < hend; h0 += RPW * U) {
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int h = h0 + u * RPW + sub;
-            float2 xa[NP], xb[NP];
-            chunk_to_pairs<T>(x[u][0].v, xa);
-            chunk_to_pairs<T>(x[u][1].v, xb);
-            if (h0 + RPW * U < hend)
-                load_row(t, h + RPW * U, x[u]);
-            else
-                load_row(t + tstride, hbeg + u * RPW + sub, x[u]);
-            float2 acc = mul2(xa[0], xa[0]);
+            for (int u = 0; u < U; ++u) {
+                const int h = h0 + u * RPW + sub;
+                float2 xa[NP], xb[NP];
+                chunk_to_pairs<T>(x[u][0].v, xa);
+                chunk_to_pairs<T>(x[u][1].v, xb);
+                if (h0 + RPW * U < hend)
+                    load_row(t, h + RPW * U, x[u]);
+                else
+                    load_row(t + tstride, hbeg + u * RPW + sub, x[u]);
+                float2 acc = mul2(xa[0], xa[0]);
 #pragma unroll
-            for (int i = 1; i < NP; ++i) acc = fma2(xa[i], xa[i], acc);
+                for (int i = 1; i < NP; ++i) acc = fma2(xa[i], xa[i], acc);
 #pragma unroll
-            for (int i = 0; i < NP; ++i) acc = fma2(xb[i], xb[i], acc);
-            float ss = __fadd_rn(acc.x, acc.y);
+                for (int i = 0; i < NP; ++i) acc = fma2(xb[i], xb[i], acc);
+                float ss = __fadd_rn(acc.x, acc.y);
 #pragma unroll
-            for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off, LPR);
-            const float r = __frsqrt_rn(__fadd_rn(__fmul_rn(ss, inv_d), n.eps));
-            const float2 r2 = make_float2(r, r);
-            const uint4 *wrow = wsm + (h < n.hq ? 0 : WCH) + c;
-            // cast back first, then the weight (both halves)
-            Pack<uint32_t, 4> ya, yb;
+                for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off, LPR);
+                const float r = __frsqrt_rn(__fadd_rn(__fmul_rn(ss, inv_d), n.eps));
+                const float2 r2 = make_float2(r, r);
+                const uint4 *wrow = wsm + (h < n.hq ? 0 : WCH) + c;
+                // cast back first, then the weight (both halves)
+                Pack<uint32_t, 4> ya, yb;
 #pragma unroll
-            for (int i = 0; i < NP; ++i) {
-                xa[i] = mul2(xa[i], r2);
-                xb[i] = mul2(xb[i], r2);
-            }
-            pairs_to_chunk<T>(xa, ya.v);
-            pairs_to_chunk<T>(xb, yb.v);
-            const uint4 wa = wrow[0], wb = wrow[LPR];
-            const uint32_t wav[4] = {wa.x, wa.y, wa.z, wa.w}, wbv[4] = {wb.x, wb.y, wb.z, wb.w};
-            if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    ya.v[i] = mul_bf16x2(ya.v[i], wav[i]);
-                    yb.v[i] = mul_bf16x2(yb.v[i], wbv[i]);
+                for (int i = 0; i < NP; ++i) {
+                    xa[i] = mul2(xa[i], r2);
+                    xb[i] = mul2(xb[i], r2);
                 }
-            } else {
+                pairs_to_chunk<T>(xa, ya.v);
+                pairs_to_chunk<T>(xb, yb.v);
+                const uint4 wa = wrow[0], wb = wrow[LPR];
+                const uint32_t wav[4] = {wa.x, wa.y, wa.z, wa.w}, wbv[4] = {wb.x, wb.y, wb.z, wb.w};
+                if constexpr (std::is_same<T, __nv_bfloat16>::value) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    ya.v[i] = __float_as_uint(__fmul_rn(__uint_as_float(ya.v[i]), __uint_as_float(wav[i])));
-                    yb.v[i] = __float_as_uint(__fmul_rn(__uint_as_float(yb.v[i]), __uint_as_float(wbv[i])));
+                    for (int i = 0; i < 4; ++i) {
+                        ya.v[i] = mul_bf16x2(ya.v[i], wav[i]);
+                        yb.v[i] = mul_bf16x2(yb.v[i], wbv[i]);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        ya.v[i] = __float_as_uint(__fmul_rn(__uint_as_float(ya.v[i]), __uint_as_float(wav[i])));
+                        yb.v[i] = __float_as_uint(__fmul_rn(__uint_as_float(yb.v[i]), __uint_as_float(wbv[i])));
+                    }
                 }
-            }
-            // x'[j] = x[j] cos_j - x[j+h] sin_j,  x'[j+h] = x[j+h] cos_j + x[j] sin_j
-            float2 va[NP], vb[NP], oa[NP], ob[NP];
-            chunk_to_pairs<T>(ya.v, va);
-            chunk_to_pairs<T>(yb.v, vb);
+                // x'[j] = x[j] cos_j - x[j+h] sin_j,  x'[j+h] = x[j+h] cos_j + x[j] sin_j
+                float2 va[NP], vb[NP], oa[NP], ob[NP];
+                chunk_to_pairs<T>(ya.v, va);
+                chunk_to_pairs<T>(yb.v, vb);
 #pragma unroll
-            for (int i = 0; i < NP; ++i) {
-                const float2 ns = make_float2(-sn[i].x, -sn[i].y);
-                oa[i] = fma2(va[i], co[i], mul2(vb[i], ns));
-                ob[i] = fma2(vb[i], co[i], mul2(va[i], sn[i]));
-            }
-            Pack<uint32_t, 4> pa, pb;
-            pairs_to_chunk<T>(oa, pa.v);
-            pairs_to_chunk<T>(ob, pb.v);
-            if (h < hend) {
-                uint32_t *p = row_ptr(t, h);
-                st_pack<uint32_t, 4>(p, pa);
-                st_pack<uint32_t, 4>(p + kHalfWords, pb);
+                for (int i = 0; i < NP; ++i) {
+                    const float2 ns = make_float2(-sn[i].x, -sn[i].y);
+                    oa[i] = fma2(va[i], co[i], mul2(vb[i], ns));
+                    ob[i] = fma2(vb[i], co[i], mul2(va[i], sn[i]));
+                }
+                Pack<uint32_t, 4> pa, pb;
+                pairs_to_chunk<T>(oa, pa.v);
+                pairs_to_chunk<T>(ob, pb.v);
+                if (h < hend) {
+                    uint32_t *p = row_ptr(t, h);
+                    st_pack<uint32_t, 4>(p, pa);
+                    st_pack<uint32_t, 4>(p + kHalfWords, pb);
+                }
             }
         }
         __syncwarp();
