@@ -438,6 +438,8 @@ CASES = {
     "vis_pos_interp_batch8": "interpolation of the batch of 8 single images (bf16 table, N = 26528)",
     "mrope_apply_prefill": "fused MRoPE of the large-prefill request (Q [131072, 24, 256], K [131072, 4, 256])",
     "mrope_apply_short": "fused MRoPE on the 4096-token prompt (text_t4096_qwen35: Q [4096, 24, 256], K [4096, 4, 256])",
+    "mrope_apply_omni": "fused MRoPE on text_t32768_omni (Q [32768, 32, 128], K [32768, 4, 128] bf16, rot 128: "
+                        "rows of 9 KB, rotated as two rows of half the heads)",
     "qk_norm_mrope_short": "fused QK-RMSNorm + MRoPE on the 4096-token prompt (text_t4096_qwen35)",
     "qk_norm_mrope_prefill_quarter": "fused QK-RMSNorm + MRoPE on the first 32768 tokens of the large-prefill "
                                      "request (Q [32768, 24, 256], K [32768, 4, 256] bf16, 470 MB)",
@@ -515,9 +517,11 @@ def run_case(args):
         out = torch.empty(wl.n_patches(v), v.hidden, dtype=torch.bfloat16, device=dev)
         fn = lambda: ipe.vis_pos_interp(table, v.grid_thw, v.merge, out=out, stream=stream)  # noqa: E731
         nbytes = algorithmic_bytes_vision(v)
-    elif name in ("mrope_apply_short", "qk_norm_mrope_short", "mrope_apply_prefill", "qk_norm_mrope_prefill_quarter"):
+    elif name in ("mrope_apply_short", "qk_norm_mrope_short", "mrope_apply_prefill", "qk_norm_mrope_prefill_quarter",
+                  "mrope_apply_omni"):
         big = name in ("mrope_apply_prefill", "qk_norm_mrope_prefill_quarter")
-        w = wl.WORKLOADS["prefill_t131072_video" if big else "text_t4096_qwen35"]
+        w = wl.WORKLOADS["prefill_t131072_video" if big else
+                         "text_t32768_omni" if name == "mrope_apply_omni" else "text_t4096_qwen35"]
         t = w.text
         tin = wl.text_inputs(w)
         T = t.T // 4 if name == "qk_norm_mrope_prefill_quarter" else t.T
