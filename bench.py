@@ -816,7 +816,7 @@ def _time_resident(torch, stream, fn, reps):
     the GPU's, not the host's launch rate."""
     fn()
     torch.cuda.synchronize()
-    torch.cuda._sleep(5_000_000)
+    torch.cuda._sleep(max(5_000_000, 400_000 * reps))   # about 0.2 ms of queueing per call
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(reps):
