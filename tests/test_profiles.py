@@ -58,3 +58,14 @@ def test_traffic_table_entries():
         for k, v in kernels.items():
             assert "--clock-control none" in v["capture"], (workload, k)
             assert v["bytes_per_launch"] > 0 and len(v["source_sha"]) == 16, (workload, k)
+
+
+def test_cited_bench_cases_exist():
+    import re
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    for name in SUMMARIES:
+        for c in _commands(open(os.path.join(PROFILES, name)).read()):
+            for case in re.findall(r"--case (\S+)", c):
+                assert case in bench.CASES, f"{name}: --case {case} is not a bench case"
