@@ -68,4 +68,6 @@ def test_cited_bench_cases_exist():
     for name in SUMMARIES:
         for c in _commands(open(os.path.join(PROFILES, name)).read()):
             for case in re.findall(r"--case (\S+)", c):
+                if case.isupper():
+                    continue                  # a placeholder for the cases a summary lists
                 assert case in bench.CASES, f"{name}: --case {case} is not a bench case"
